@@ -1,0 +1,343 @@
+#!/usr/bin/env python
+"""Benchmark of one MLA decode step (absorb -> paged decode -> combine -> up-project).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config v3] [--impl reference]
+
+Prints one JSON line (rank 0).  The workload is the DeepSeek-V3-shaped decode
+(batch 64, 128 heads, 4096 cached tokens per sequence, bf16 cache in 64-token
+pages with a shuffled block table); other presets can be chosen with --config.
+Under torchrun every rank runs its own batch (different seed, same shape): the
+sequences are independent, so ranks exchange nothing on the data path and the
+line reports weak scaling, timed on the device as the max over ranks.
+
+Timing: W untimed warm-up steps, then K steps; each step is bracketed by CUDA
+events on the launching stream and L2 is flushed (a 256 MB write) between steps,
+outside the events.  ``value`` is cache GB/s of the whole step (all ranks);
+``roofline`` is the decode kernel's own cache bytes over its event-timed
+duration against the measured HBM copy bandwidth.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode cache GB/s, TFLOP/s & % of B200 roofline; tokens/s per step"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def step_flops(lens, H, s_q):
+    """Algorithmic decode FLOPs: 2 * (576 + 512) per (cached token, head, query)."""
+    return sum(lens) * H * s_q * 2 * (576 + 512)
+
+
+def proj_flops(n_tok, H):
+    return 2 * (2 * n_tok * H * 128 * 512)
+
+
+def shard_seed(base_seed: int, rank: int) -> int:
+    """Each rank decodes its own batch: same shape, its own seed."""
+    return base_seed + 1000 * rank
+
+
+def reduce_max(x: float) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_cpu_baseline(spec_name: str, budget_s: float = 12.0):
+    """Times the fp64 oracle (absorbed form, the oracle's faster mode) on a bounded
+    sample of the workload: whole sequences, all heads, until the budget is used.
+    Returns (GB/s of cache processed, description, cores)."""
+    import numpy as np
+    import torch
+    from mla_inputs import make_workload, preset
+    import oracle
+    from oracle import mla_oracle as om
+    spec = preset(spec_name)
+    w = make_workload(spec)
+    inp = oracle.from_workload(w)
+    row_bytes = 1152 if spec.kv_dtype == "bf16" else 580
+    done_b, done_tokens, t0 = 0, 0, time.perf_counter()
+    while done_b < w.B and time.perf_counter() - t0 < budget_s:
+        om.decode_absorbed(inp, rows=[(done_b, i) for i in range(w.s_q)])
+        done_tokens += w.lens[done_b]
+        done_b += 1
+    dt = time.perf_counter() - t0
+    cores = torch.get_num_threads()
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        cores = max([d.get("num_threads", 0) for d in info] + [1])
+    except Exception:
+        pass
+    gbs = done_tokens * row_bytes / dt / 1e9
+    desc = (f"oracle decode_absorbed (fp64 numpy) on {done_b} of {w.B} sequences "
+            f"({done_tokens} cached tokens, all {w.H} heads, {w.s_q} queries) in {dt:.2f} s")
+    return gbs, desc, cores, dt
+
+
+def run_reference(args):
+    """The oracle timed on the host cores as the reference arm (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    vals, descs, cores = [], [], 1
+    for _ in range(args.warmup):
+        oracle_cpu_baseline(args.config, budget_s=2.0)
+    for _ in range(args.steps):
+        v, d, cores, _ = oracle_cpu_baseline(args.config, budget_s=max(2.0, 40.0 / max(1, args.steps)))
+        vals.append(v)
+        descs.append(d)
+    value = statistics.mean(vals)
+    line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": _config_dict(args.config, None),
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
+                             "kind": "oracle", "sample": descs[-1]},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config_dict(name, w, splits=None):
+    from mla_inputs import preset
+    s = preset(name)
+    d = {"workload": f"{name}: {s.note}", "B": s.B, "H": s.H, "s_q": s.s_q,
+         "kv_cache": s.kv_dtype, "page_size": 64, "d_c": 512, "d_r": 64,
+         "causal": s.causal, "l2": "flushed between timed steps (256 MB write)"}
+    if w is not None:
+        d["cached_tokens"] = sum(w.lens)
+    if splits is not None:
+        d["splits"] = splits
+    return d
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="v3")
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    import head_latent_attention_06_b200 as mla
+    from head_latent_attention_06_b200.step import step_from_workload
+    from mla_inputs import make_workload, preset
+    mla.load()
+
+    spec = preset(args.config)
+    spec = spec.with_(seed=shard_seed(spec.seed, rank))
+    w = make_workload(spec)
+    st = step_from_workload(w, num_splits=args.splits)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    cache_bytes = w.cache_bytes()
+    flops = step_flops(w.lens, w.H, w.s_q)
+
+    def timed_step(ev):
+        ev[0].record(stream)
+        st.absorb()
+        ev[1].record(stream)
+        mla.mla_decode_paged(st.args)
+        ev[2].record(stream)
+        mla.mla_combine_splits(st.args)
+        st.up_project()
+        ev[3].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        st.run()
+    torch.cuda.synchronize()
+    assert mla.mla_get_status(st.workspace) == 0
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for k in range(args.steps):
+            flush.zero_()
+            timed_step(evs[k])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    total_ms = reduce_max(sum(step_ms))
+    dec_avg_ms = reduce_max(sum(dec_ms) / len(dec_ms))
+    ms_per_step = total_ms / args.steps
+
+    # end to end through the public API: pinned host queries and metadata in,
+    # the step's output back to pinned host memory, every step.
+    h_q_nope = w.q_nope.pin_memory()
+    h_q_pe = w.q_pe.pin_memory()
+    h_bt = w.block_table.pin_memory()
+    h_len = w.seq_lens.pin_memory()
+    h_out = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+    d_bt, d_len = st._keep[2], st._keep[3]
+    h2d = sum(t.numel() * t.element_size() for t in (h_q_nope, h_q_pe, h_bt, h_len))
+    d2h = h_out.numel() * h_out.element_size()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    for k in range(args.steps + 2):
+        flush.zero_()
+        e0, e1 = e2e_ev[k - 2] if k >= 2 else (None, None)
+        if e0 is not None:
+            e0.record(stream)
+        st.q_nope.copy_(h_q_nope, non_blocking=True)
+        st.q_pe.copy_(h_q_pe, non_blocking=True)
+        d_bt.copy_(h_bt, non_blocking=True)
+        d_len.copy_(h_len, non_blocking=True)
+        st.run()
+        h_out.copy_(st.out, non_blocking=True)
+        if e1 is not None:
+            e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(sum(a.elapsed_time(b) for a, b in e2e_ev)) / args.steps
+
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    value = world * cache_bytes / (ms_per_step * 1e-3) / 1e9
+    dec_gbs = cache_bytes / (dec_avg_ms * 1e-3) / 1e9
+    dec_tflops = flops / (dec_avg_ms * 1e-3) / 1e12
+    t_mem = cache_bytes / (hbm * 1e9)
+    t_tc = flops / (float(peaks["bf16_tflops"]) * 1e12)
+    launches_per_step = 3 + (1 if st.num_splits > 1 else 0)
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8-e4m3 cache, bf16 MMA" if spec.kv_dtype == "fp8" else "bf16",
+        "data": "synthetic (seeded, N(0,1) activations and cache, N(0,1/512) weights)",
+        "config": _config_dict(args.config, w, st.num_splits),
+        "tflops": round(world * (flops + proj_flops(w.n_tok, w.H)) / (ms_per_step * 1e-3) / 1e12, 2),
+        "tokens_per_s": round(world * w.n_tok / (ms_per_step * 1e-3), 1),
+        "decode_us": round(dec_avg_ms * 1e3, 2),
+        "roofline": {
+            "bound": "hbm", "achieved": round(dec_gbs, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(dec_gbs / hbm, 4), "traffic": None,
+            "peak_kind": f"{peak_kind} HBM copy bandwidth",
+            "kernel": "mla_decode_paged",
+            "tensor": {"achieved_tflops": round(dec_tflops, 1),
+                       "peak_tflops": float(peaks["bf16_tflops"]),
+                       "frac": round(dec_tflops / float(peaks["bf16_tflops"]), 4)},
+            "binding_roofline_frac": round(max(t_mem, t_tc) / (dec_avg_ms * 1e-3), 4),
+        },
+        "e2e": {"value": round(world * cache_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 5)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, cores, _ = oracle_cpu_baseline(args.config)
+        line["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": cores,
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

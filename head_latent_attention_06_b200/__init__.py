@@ -1,0 +1,202 @@
+"""B200 (sm_100a) MLA decode over a paged latent KV cache.
+
+A thin ctypes binding over ``libmla_b200.so`` (C ABI in ``include/mla.h``).  The
+functions keep the C names and only marshal arguments: torch tensors become
+device pointers and sizes, the current torch stream becomes the CUDA stream.
+Every step of the computation runs in the library's CUDA kernels; there is no
+fallback, and calling into a missing library raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmla_b200.so")
+
+D_C, D_R, D_N, D_V, PAGE = 512, 64, 128, 128, 64
+MAX_SPLITS = 128
+KV_BF16, KV_FP8_E4M3 = 0, 1
+
+STATUS = {
+    0: "MLA_OK", 1: "MLA_ERR_INVALID_VALUE", 2: "MLA_ERR_UNSUPPORTED", 3: "MLA_ERR_MISALIGNED",
+    4: "MLA_ERR_WORKSPACE_TOO_SMALL", 5: "MLA_ERR_CUDA", 6: "MLA_ERR_DEVICE_TIMEOUT",
+    7: "MLA_ERR_BAD_BLOCK_TABLE", 8: "MLA_ERR_BAD_SEQ_LEN",
+}
+
+# Every symbol include/mla.h declares.
+EXPORTS = ("mla_absorb_q", "mla_decode_workspace_size", "mla_decode_num_splits",
+           "mla_decode_paged", "mla_combine_splits", "mla_up_proj_v", "mla_get_status",
+           "mla_status_string")
+
+
+class MlaError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class DecodeArgs(ctypes.Structure):
+    """Mirror of ``mla_decode_args_t`` (field order and types must match)."""
+    _fields_ = [
+        ("q_lat", ctypes.c_void_p), ("q_pe", ctypes.c_void_p),
+        ("kv_cache", ctypes.c_void_p), ("kv_scale", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+        ("o_lat", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("B", ctypes.c_int32), ("s_q", ctypes.c_int32), ("H", ctypes.c_int32),
+        ("d_c", ctypes.c_int32), ("d_r", ctypes.c_int32), ("page_size", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
+        ("kv_dtype", ctypes.c_int32), ("causal", ctypes.c_int32),
+        ("num_splits", ctypes.c_int32), ("max_seq_len", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float),
+    ]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (built by ``head_latent_attention_06_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: run `python -m head_latent_attention_06_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32 = ctypes.c_void_p, ctypes.c_int32
+    lib.mla_absorb_q.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
+    lib.mla_up_proj_v.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
+    pa = ctypes.POINTER(DecodeArgs)
+    lib.mla_decode_workspace_size.argtypes = [pa, ctypes.POINTER(ctypes.c_size_t)]
+    lib.mla_decode_num_splits.argtypes = [pa, ctypes.POINTER(ctypes.c_int32)]
+    lib.mla_decode_paged.argtypes = [pa, vp]
+    lib.mla_combine_splits.argtypes = [pa, vp]
+    lib.mla_get_status.argtypes = [vp, vp]
+    lib.mla_status_string.argtypes = [ctypes.c_int]
+    lib.mla_status_string.restype = ctypes.c_char_p
+    for name in EXPORTS:
+        if name != "mla_status_string":
+            getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else int(t.data_ptr())
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    return int(stream) if isinstance(stream, int) else int(stream.cuda_stream)
+
+
+def _check(fn, code):
+    if code != 0:
+        raise MlaError(fn, code)
+
+
+def _dev(t, dtype, name):
+    import torch
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+    return t
+
+
+# ------------------------------------------------------------------ entry points
+
+def mla_absorb_q(q_nope, w_uk, q_lat, stream=None):
+    """q_lat[t][h] = W_UK[h]^T q_nope[t][h]; q_nope [n_tok][H][128], w_uk [H][128][512],
+    q_lat [n_tok][H][512], all bf16 on the device."""
+    import torch
+    for t, n in ((q_nope, "q_nope"), (w_uk, "w_uk"), (q_lat, "q_lat")):
+        _dev(t, torch.bfloat16, n)
+    H = w_uk.shape[0]
+    n_tok = q_nope.numel() // (H * D_N)
+    _check("mla_absorb_q", load().mla_absorb_q(_ptr(q_nope), _ptr(w_uk), _ptr(q_lat), n_tok, H,
+                                               w_uk.shape[1], w_uk.shape[2], _stream(stream)))
+
+
+def mla_up_proj_v(o_lat, w_uv, out, stream=None):
+    """out[t][h] = W_UV[h] o_lat[t][h]; o_lat [n_tok][H][512], w_uv [H][128][512],
+    out [n_tok][H][128], all bf16 on the device."""
+    import torch
+    for t, n in ((o_lat, "o_lat"), (w_uv, "w_uv"), (out, "out")):
+        _dev(t, torch.bfloat16, n)
+    H = w_uv.shape[0]
+    n_tok = o_lat.numel() // (H * D_C)
+    _check("mla_up_proj_v", load().mla_up_proj_v(_ptr(o_lat), _ptr(w_uv), _ptr(out), n_tok, H,
+                                                 w_uv.shape[1], w_uv.shape[2], _stream(stream)))
+
+
+def make_decode_args(*, q_lat, q_pe, kv_cache, kv_scale, block_table, seq_lens, o_lat, lse,
+                     workspace=None, causal=False, softmax_scale, num_splits=0,
+                     max_seq_len=0) -> DecodeArgs:
+    """Fill a ``DecodeArgs`` from device tensors.  Shapes: q_lat [B][s_q][H][512],
+    q_pe [B][s_q][H][64], kv_cache [num_pages][64][576] (bf16 or float8_e4m3fn),
+    kv_scale [num_pages][64] fp32 or None, block_table [B][max_pages] int32,
+    seq_lens [B] int32, o_lat like q_lat, lse [B][s_q][H] fp32 or None."""
+    import torch
+    B, s_q, H, _ = q_lat.shape
+    fp8 = kv_cache.dtype == torch.float8_e4m3fn
+    a = DecodeArgs()
+    a.q_lat, a.q_pe = _ptr(q_lat), _ptr(q_pe)
+    a.kv_cache, a.kv_scale = _ptr(kv_cache), _ptr(kv_scale)
+    a.block_table, a.seq_lens = _ptr(block_table), _ptr(seq_lens)
+    a.o_lat, a.lse = _ptr(o_lat), _ptr(lse)
+    a.B, a.s_q, a.H = B, s_q, H
+    a.d_c, a.d_r, a.page_size = D_C, D_R, PAGE
+    a.num_pages = kv_cache.shape[0]
+    a.max_pages_per_seq = block_table.shape[1]
+    a.kv_dtype = KV_FP8_E4M3 if fp8 else KV_BF16
+    a.causal = int(bool(causal))
+    a.num_splits = int(num_splits)
+    a.max_seq_len = int(max_seq_len)
+    a.softmax_scale = float(softmax_scale)
+    if workspace is not None:
+        a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    return a
+
+
+def mla_decode_workspace_size(args: DecodeArgs) -> int:
+    n = ctypes.c_size_t(0)
+    _check("mla_decode_workspace_size", load().mla_decode_workspace_size(ctypes.byref(args), ctypes.byref(n)))
+    return int(n.value)
+
+
+def mla_decode_num_splits(args: DecodeArgs) -> int:
+    n = ctypes.c_int32(0)
+    _check("mla_decode_num_splits", load().mla_decode_num_splits(ctypes.byref(args), ctypes.byref(n)))
+    return int(n.value)
+
+
+def mla_decode_paged(args: DecodeArgs, stream=None):
+    _check("mla_decode_paged", load().mla_decode_paged(ctypes.byref(args), _stream(stream)))
+
+
+def mla_combine_splits(args: DecodeArgs, stream=None):
+    _check("mla_combine_splits", load().mla_combine_splits(ctypes.byref(args), _stream(stream)))
+
+
+def mla_get_status(workspace, stream=None) -> int:
+    """Waits for the stream and returns (and clears) the device status word."""
+    return int(load().mla_get_status(_ptr(workspace), _stream(stream)))
+
+
+def mla_status_string(code: int) -> str:
+    return load().mla_status_string(int(code)).decode()
+
+
+def alloc_workspace(args: DecodeArgs, device="cuda"):
+    """A zeroed workspace tensor sized for ``args``; also stored into ``args``."""
+    import torch
+    n = mla_decode_workspace_size(args)
+    ws = torch.zeros(n, dtype=torch.uint8, device=device)
+    args.workspace, args.workspace_bytes = _ptr(ws), n
+    return ws

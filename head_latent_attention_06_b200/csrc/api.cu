@@ -1,0 +1,169 @@
+// C ABI of the MLA decode library (declared in include/mla.h): host-side
+// argument validation, split selection, workspace sizing and kernel launches.
+// Nothing here allocates device memory or synchronises, except mla_get_status.
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+
+namespace mla {
+cudaError_t launch_absorb_q(const void*, const void*, void*, int, int, cudaStream_t);
+cudaError_t launch_up_proj_v(const void*, const void*, void*, int, int, cudaStream_t);
+cudaError_t launch_decode_mma(const mla_decode_args_t*, int, cudaStream_t);
+cudaError_t launch_combine(const mla_decode_args_t*, int, cudaStream_t);
+int decode_mma_tiles(int len);
+int decode_mma_ctas_per_split(int s_q, int H, int B);
+}  // namespace mla
+
+using namespace mla;
+
+namespace {
+
+constexpr int kNumSMs = 148;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+mla_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+mla_status_t check_proj(const void* x, const void* w, const void* y, int32_t n_tok, int32_t H,
+                        int32_t d_small, int32_t d_c) {
+  if (n_tok < 0 || H <= 0) return MLA_ERR_INVALID_VALUE;
+  if (d_small != 128 || d_c != kDc) return MLA_ERR_UNSUPPORTED;
+  if (n_tok == 0) return MLA_OK;
+  if (!x || !w || !y) return MLA_ERR_INVALID_VALUE;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return MLA_ERR_MISALIGNED;
+  return MLA_OK;
+}
+
+// Shape checks shared by the decode entry points (no pointer checks).
+mla_status_t check_decode_shape(const mla_decode_args_t* a) {
+  if (!a) return MLA_ERR_INVALID_VALUE;
+  if (a->B < 0 || a->H <= 0 || a->s_q <= 0 || a->num_pages < 0 || a->max_pages_per_seq <= 0)
+    return MLA_ERR_INVALID_VALUE;
+  if (a->d_c != kDc || a->d_r != kDr || a->page_size != kPage) return MLA_ERR_UNSUPPORTED;
+  if (a->H % 16 != 0 || a->H > 128 || a->s_q > 2) return MLA_ERR_UNSUPPORTED;
+  if (a->kv_dtype != MLA_KV_BF16 && a->kv_dtype != MLA_KV_FP8_E4M3) return MLA_ERR_UNSUPPORTED;
+  if (a->num_splits < 0 || a->num_splits > MLA_MAX_SPLITS) return MLA_ERR_INVALID_VALUE;
+  if (a->max_seq_len < 0) return MLA_ERR_INVALID_VALUE;
+  if (!(a->softmax_scale == a->softmax_scale)) return MLA_ERR_INVALID_VALUE;
+  return MLA_OK;
+}
+
+// Split count: enough (sequence, row-group, split) CTAs to cover the SMs, but
+// never a split shorter than 8 tiles.
+int choose_splits(const mla_decode_args_t* a) {
+  if (a->num_splits > 0) return a->num_splits;
+  const int max_len = a->max_seq_len > 0 ? a->max_seq_len : a->max_pages_per_seq * kPage;
+  const int tiles = decode_mma_tiles(max_len);
+  const int ctas = decode_mma_ctas_per_split(a->s_q, a->H, a->B > 0 ? a->B : 1);
+  int s = (kNumSMs + ctas - 1) / ctas;
+  int cap = tiles / 8;
+  if (cap < 1) cap = 1;
+  if (s > cap) s = cap;
+  if (s > MLA_MAX_SPLITS) s = MLA_MAX_SPLITS;
+  if (s < 1) s = 1;
+  return s;
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status_t mla_absorb_q(const void* q_nope, const void* w_uk, void* q_lat, int32_t n_tok,
+                          int32_t H, int32_t d_n, int32_t d_c, void* stream) {
+  mla_status_t st = check_proj(q_nope, w_uk, q_lat, n_tok, H, d_n, d_c);
+  if (st != MLA_OK || n_tok == 0) return st;
+  return from_cuda(launch_absorb_q(q_nope, w_uk, q_lat, n_tok, H, (cudaStream_t)stream));
+}
+
+mla_status_t mla_up_proj_v(const void* o_lat, const void* w_uv, void* out, int32_t n_tok, int32_t H,
+                           int32_t d_v, int32_t d_c, void* stream) {
+  mla_status_t st = check_proj(o_lat, w_uv, out, n_tok, H, d_v, d_c);
+  if (st != MLA_OK || n_tok == 0) return st;
+  return from_cuda(launch_up_proj_v(o_lat, w_uv, out, n_tok, H, (cudaStream_t)stream));
+}
+
+mla_status_t mla_decode_num_splits(const mla_decode_args_t* a, int32_t* num_splits) {
+  mla_status_t st = check_decode_shape(a);
+  if (st != MLA_OK) return st;
+  if (!num_splits) return MLA_ERR_INVALID_VALUE;
+  *num_splits = choose_splits(a);
+  return MLA_OK;
+}
+
+mla_status_t mla_decode_workspace_size(const mla_decode_args_t* a, size_t* bytes) {
+  mla_status_t st = check_decode_shape(a);
+  if (st != MLA_OK) return st;
+  if (!bytes) return MLA_ERR_INVALID_VALUE;
+  *bytes = workspace_layout(a->B * a->s_q, a->H, choose_splits(a)).total;
+  return MLA_OK;
+}
+
+static mla_status_t check_decode_ptrs(const mla_decode_args_t* a, int splits) {
+  if (!a->workspace) return MLA_ERR_INVALID_VALUE;
+  if (!aligned16(a->workspace)) return MLA_ERR_MISALIGNED;
+  if (a->workspace_bytes < workspace_layout(a->B * a->s_q, a->H, splits).total)
+    return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (a->B == 0) return MLA_OK;
+  if (!a->q_lat || !a->q_pe || !a->kv_cache || !a->block_table || !a->seq_lens || !a->o_lat)
+    return MLA_ERR_INVALID_VALUE;
+  if (a->kv_dtype == MLA_KV_FP8_E4M3 && !a->kv_scale) return MLA_ERR_INVALID_VALUE;
+  if (a->num_pages <= 0) return MLA_ERR_INVALID_VALUE;
+  if (!aligned16(a->q_lat) || !aligned16(a->q_pe) || !aligned16(a->kv_cache) ||
+      !aligned16(a->o_lat))
+    return MLA_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(a->block_table) & 3u) ||
+      (reinterpret_cast<uintptr_t>(a->seq_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(a->lse) & 3u) || (reinterpret_cast<uintptr_t>(a->kv_scale) & 3u))
+    return MLA_ERR_MISALIGNED;
+  return MLA_OK;
+}
+
+mla_status_t mla_decode_paged(const mla_decode_args_t* a, void* stream) {
+  mla_status_t st = check_decode_shape(a);
+  if (st != MLA_OK) return st;
+  const int splits = choose_splits(a);
+  st = check_decode_ptrs(a, splits);
+  if (st != MLA_OK || a->B == 0) return st;
+  return from_cuda(launch_decode_mma(a, splits, (cudaStream_t)stream));
+}
+
+mla_status_t mla_combine_splits(const mla_decode_args_t* a, void* stream) {
+  mla_status_t st = check_decode_shape(a);
+  if (st != MLA_OK) return st;
+  const int splits = choose_splits(a);
+  st = check_decode_ptrs(a, splits);
+  if (st != MLA_OK || a->B == 0 || splits == 1) return st;
+  return from_cuda(launch_combine(a, splits, (cudaStream_t)stream));
+}
+
+mla_status_t mla_get_status(void* workspace, void* stream) {
+  if (!workspace) return MLA_ERR_INVALID_VALUE;
+  uint32_t word = 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MLA_ERR_CUDA;
+  if (word != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(word), s) != cudaSuccess) return MLA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  return (mla_status_t)word;
+}
+
+const char* mla_status_string(mla_status_t s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_VALUE: return "MLA_ERR_INVALID_VALUE";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_MISALIGNED: return "MLA_ERR_MISALIGNED";
+    case MLA_ERR_WORKSPACE_TOO_SMALL: return "MLA_ERR_WORKSPACE_TOO_SMALL";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT";
+    case MLA_ERR_BAD_BLOCK_TABLE: return "MLA_ERR_BAD_BLOCK_TABLE";
+    case MLA_ERR_BAD_SEQ_LEN: return "MLA_ERR_BAD_SEQ_LEN";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,65 @@
+"""One MLA decode step through the C ABI: absorb -> paged decode -> combine -> up-project.
+
+``DecodeStep`` owns the intermediate device buffers (q_lat, o_lat, lse, out and
+the workspace) and replays the four calls on the current stream.  It does no
+arithmetic of its own.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import (D_C, D_N, D_V, alloc_workspace, make_decode_args, mla_absorb_q,
+               mla_combine_splits, mla_decode_num_splits, mla_decode_paged, mla_up_proj_v)
+
+
+class DecodeStep:
+    def __init__(self, *, q_nope, q_pe, w_uk, w_uv, kv_cache, kv_scale, block_table, seq_lens,
+                 causal, softmax_scale, num_splits=0, max_seq_len=0, out=None):
+        B, s_q, H, _ = q_nope.shape
+        dev = q_nope.device
+        self.B, self.s_q, self.H = B, s_q, H
+        self.q_nope, self.q_pe, self.w_uk, self.w_uv = q_nope, q_pe, w_uk, w_uv
+        self.q_lat = torch.empty(B, s_q, H, D_C, dtype=torch.bfloat16, device=dev)
+        self.o_lat = torch.empty(B, s_q, H, D_C, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(B, s_q, H, dtype=torch.float32, device=dev)
+        self.out = out if out is not None else torch.empty(B, s_q, H, D_V, dtype=torch.bfloat16,
+                                                           device=dev)
+        self.args = make_decode_args(q_lat=self.q_lat, q_pe=q_pe, kv_cache=kv_cache,
+                                     kv_scale=kv_scale, block_table=block_table,
+                                     seq_lens=seq_lens, o_lat=self.o_lat, lse=self.lse,
+                                     causal=causal, softmax_scale=softmax_scale,
+                                     num_splits=num_splits, max_seq_len=max_seq_len)
+        self.workspace = alloc_workspace(self.args, device=dev)
+        self.num_splits = mla_decode_num_splits(self.args)
+        self._keep = (kv_cache, kv_scale, block_table, seq_lens)
+
+    def absorb(self, stream=None):
+        n_tok = self.B * self.s_q
+        mla_absorb_q(self.q_nope.view(n_tok, self.H, D_N), self.w_uk,
+                     self.q_lat.view(n_tok, self.H, D_C), stream)
+
+    def attend(self, stream=None):
+        mla_decode_paged(self.args, stream)
+        mla_combine_splits(self.args, stream)
+
+    def up_project(self, stream=None):
+        n_tok = self.B * self.s_q
+        mla_up_proj_v(self.o_lat.view(n_tok, self.H, D_C), self.w_uv,
+                      self.out.view(n_tok, self.H, D_V), stream)
+
+    def run(self, stream=None):
+        self.absorb(stream)
+        self.attend(stream)
+        self.up_project(stream)
+        return self.out
+
+
+def step_from_workload(w, device="cuda", num_splits=0):
+    """Copy a ``mla_inputs.Workload`` to the device and build its ``DecodeStep``."""
+    d = lambda t: None if t is None else t.to(device, non_blocking=False).contiguous()
+    return DecodeStep(q_nope=d(w.q_nope), q_pe=d(w.q_pe), w_uk=d(w.w_uk), w_uv=d(w.w_uv),
+                      kv_cache=d(w.kv_cache), kv_scale=d(w.kv_scale),
+                      block_table=d(w.block_table), seq_lens=d(w.seq_lens), causal=w.causal,
+                      softmax_scale=w.softmax_scale, num_splits=num_splits,
+                      max_seq_len=max(w.lens) if w.lens else 0)

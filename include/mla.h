@@ -1,0 +1,164 @@
+/*
+ * mla.h — C ABI of the B200 (sm_100a) MLA decode library.
+ *
+ * Multi-Head Latent Attention decode over a paged latent KV cache.  Every cached
+ * token holds one latent c (d_c = 512 values) followed by a decoupled RoPE key
+ * k_pe (d_r = 64 values), shared by all heads: the 576-value record of the
+ * snowgate forum thread 35 (replies on the latent record, "512-dim + 64-dim
+ * rope").  Keys and values are up-projections of the latent, k = W_UK c and
+ * v = W_UV c ("MLA: Multi-Head Latent Attention — DeepSeek-AI Explained",
+ * section "Architecture"); decode never forms them, it folds W_UK into the query
+ * and W_UV into the output (nnets.ru article, section "Суть MLA", the weight
+ * absorbing trick).  One decode step is four calls, in order:
+ *
+ *   mla_absorb_q       q_lat = W_UK^T q_nope                 (per head)
+ *   mla_decode_paged   scores, online softmax, o_lat = P c   (split-KV partials)
+ *   mla_combine_splits log-sum-exp merge of the partials     (no-op for 1 split)
+ *   mla_up_proj_v      o = W_UV o_lat                         (per head)
+ *
+ * Conventions for every entry point:
+ *  - Pointers are DEVICE pointers unless a field says otherwise; the caller owns
+ *    every buffer.  The library allocates nothing, frees nothing and keeps no
+ *    pointer after a call returns.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL means the legacy default
+ *    stream) and the call returns without waiting, except mla_get_status.
+ *  - Tensors are dense and row-major in the index order written; bf16 is
+ *    bfloat16, e4m3 is OCP float8 e4m3fn.
+ *  - Calls return a status and never throw or abort.  Argument errors are found
+ *    on the host before anything is enqueued; problems that only the device can
+ *    see (a page id outside the cache, a length beyond the block table) are
+ *    recorded in the workspace's status word and read by mla_get_status.
+ *  - The library is built for sm_100a only; on another device the launch fails
+ *    and MLA_ERR_CUDA is returned.
+ */
+#ifndef MLA_B200_H
+#define MLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_VALUE = 1,        /* null pointer, negative or inconsistent size */
+  MLA_ERR_UNSUPPORTED = 2,          /* a dimension this build does not handle */
+  MLA_ERR_MISALIGNED = 3,           /* a pointer is not 16-byte aligned */
+  MLA_ERR_WORKSPACE_TOO_SMALL = 4,  /* workspace_bytes < mla_decode_workspace_size() */
+  MLA_ERR_CUDA = 5,                 /* a CUDA runtime call or launch failed */
+  MLA_ERR_DEVICE_TIMEOUT = 6,       /* a bounded device wait ran out (device-side) */
+  MLA_ERR_BAD_BLOCK_TABLE = 7,      /* a block-table entry outside [0, num_pages) (device-side) */
+  MLA_ERR_BAD_SEQ_LEN = 8           /* seq_lens[b] < 0 or > max_pages_per_seq*page_size (device-side) */
+} mla_status_t;
+
+typedef enum { MLA_KV_BF16 = 0, MLA_KV_FP8_E4M3 = 1 } mla_kv_dtype_t;
+
+/* Supported dimensions: d_c = 512, d_r = 64, d_n = d_v = 128, page_size = 64,
+ * H a multiple of 16 up to 128, s_q in {1, 2}. */
+#define MLA_D_C 512
+#define MLA_D_R 64
+#define MLA_D_QK_NOPE 128
+#define MLA_D_V 128
+#define MLA_PAGE_SIZE 64
+#define MLA_MAX_SPLITS 128
+
+/*
+ * mla_absorb_q — weight absorption of the query (nnets.ru article, section
+ * "Суть MLA"; snowgate thread 35, "W_UK absorbing the query").
+ *   q_lat[t][h][c] = sum_n q_nope[t][h][n] * w_uk[h][n][c]
+ * q_nope : bf16 [n_tok][H][d_n]        (n_tok = B * s_q, token t = b * s_q + i)
+ * w_uk   : bf16 [H][d_n][d_c]          (k = W_UK[h] c, so W_UK[h] is d_n x d_c)
+ * q_lat  : bf16 [n_tok][H][d_c]        (written; fp32 accumulation, rounded once)
+ * d_n must be 128 and d_c 512.  n_tok = 0 enqueues nothing and returns MLA_OK.
+ */
+mla_status_t mla_absorb_q(const void* q_nope, const void* w_uk, void* q_lat,
+                          int32_t n_tok, int32_t H, int32_t d_n, int32_t d_c, void* stream);
+
+/*
+ * Arguments of mla_decode_paged / mla_combine_splits / mla_decode_workspace_size.
+ * Zero-initialise the struct, then fill every field.
+ */
+typedef struct {
+  const void* q_lat;              /* bf16 [B][s_q][H][d_c], output of mla_absorb_q */
+  const void* q_pe;               /* bf16 [B][s_q][H][d_r], RoPE already applied */
+  const void* kv_cache;           /* [num_pages][page_size][d_c + d_r]: row = c || k_pe,
+                                     bf16 (MLA_KV_BF16) or e4m3 (MLA_KV_FP8_E4M3) */
+  const float* kv_scale;          /* fp32 [num_pages][page_size], per-token dequant scale of the
+                                     whole row (value = e4m3 * scale); NULL for bf16 */
+  const int32_t* block_table;     /* int32 [B][max_pages_per_seq]: physical page of each
+                                     64-token logical page */
+  const int32_t* seq_lens;        /* int32 [B], device: cached tokens of sequence b, including
+                                     its s_q new tokens */
+  void* o_lat;                    /* bf16 [B][s_q][H][d_c], written (latent-space output) */
+  float* lse;                     /* fp32 [B][s_q][H], natural-log partition function,
+                                     written; may be NULL */
+  void* workspace;                /* device scratch, >= mla_decode_workspace_size() bytes,
+                                     16-byte aligned; its first 16 bytes must be zero before the
+                                     first use (they hold the sticky status word) */
+  size_t workspace_bytes;
+  int32_t B, s_q, H;
+  int32_t d_c, d_r, page_size;
+  int32_t num_pages;              /* physical pages in kv_cache */
+  int32_t max_pages_per_seq;      /* row length of block_table */
+  int32_t kv_dtype;               /* mla_kv_dtype_t */
+  int32_t causal;                 /* 1: query i of sequence b sees tokens 0 .. L_b - s_q + i */
+  int32_t num_splits;             /* 0 = choose automatically; else 1 .. MLA_MAX_SPLITS */
+  int32_t max_seq_len;            /* host-known upper bound of seq_lens (0 = use
+                                     max_pages_per_seq * page_size); only steers the split count */
+  float softmax_scale;            /* e.g. 1/sqrt(d_n + d_r) */
+} mla_decode_args_t;
+
+/* Bytes of workspace mla_decode_paged needs for these arguments (host only, no
+ * device access).  Depends on B, s_q, H and the split count that will be used. */
+mla_status_t mla_decode_workspace_size(const mla_decode_args_t* args, size_t* bytes);
+
+/* The split count mla_decode_paged will use for these arguments (host only). */
+mla_status_t mla_decode_num_splits(const mla_decode_args_t* args, int32_t* num_splits);
+
+/*
+ * mla_decode_paged — latent attention over the paged cache (the absorbed form of
+ * softmax attention; FlashAttention-style on-chip tiles with an online softmax,
+ * nnets.ru article, section "MLA и FlashAttention").  For query i of sequence b,
+ * head h and visible token j (j < L_b, or j <= L_b - s_q + i when causal):
+ *   s_j   = softmax_scale * (q_lat . c_j + q_pe . k_pe_j)
+ *   o_lat = sum_j softmax(s)_j c_j ,   lse = log sum_j exp(s_j)
+ * Token j is row j % page_size of page block_table[b][j / page_size].  Rows of a
+ * last page at positions >= L_b are read but weigh nothing; they must hold finite
+ * values.  With one split the results go straight to o_lat / lse; with more,
+ * fp32 partials go to the workspace and mla_combine_splits must follow on the
+ * same stream.  A query with no visible token gets o_lat = 0 and lse = -inf.
+ */
+mla_status_t mla_decode_paged(const mla_decode_args_t* args, void* stream);
+
+/*
+ * mla_combine_splits — merges split-KV partials (flash-decoding):
+ *   lse = log sum_s exp(lse_s),  o_lat = sum_s exp(lse_s - lse) o_s
+ * Reads the workspace written by mla_decode_paged with the same args; writes
+ * o_lat (bf16) and lse.  Returns MLA_OK without enqueuing work when one split
+ * was used.
+ */
+mla_status_t mla_combine_splits(const mla_decode_args_t* args, void* stream);
+
+/*
+ * mla_up_proj_v — value up-projection on the output side ("Architecture":
+ * v = W_UV c; absorbed, o = W_UV o_lat).
+ *   out[t][h][v] = sum_c w_uv[h][v][c] * o_lat[t][h][c]
+ * o_lat : bf16 [n_tok][H][d_c];  w_uv : bf16 [H][d_v][d_c];  out : bf16 [n_tok][H][d_v]
+ * d_v must be 128 and d_c 512.
+ */
+mla_status_t mla_up_proj_v(const void* o_lat, const void* w_uv, void* out,
+                           int32_t n_tok, int32_t H, int32_t d_v, int32_t d_c, void* stream);
+
+/* Waits for `stream`, returns the sticky device status word of `workspace`
+ * (MLA_OK if no device-side problem was recorded) and clears it. */
+mla_status_t mla_get_status(void* workspace, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* mla_status_string(mla_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_B200_H */

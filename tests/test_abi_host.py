@@ -1,0 +1,137 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports every
+symbol include/mla.h declares, and rejects bad arguments before touching the
+device (no call here reaches a CUDA launch)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import head_latent_attention_06_b200 as mla
+from head_latent_attention_06_b200 import build as mla_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mla.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED, WS_SMALL = 0, 1, 2, 3, 4
+
+
+@pytest.fixture(scope="module")
+def lib():
+    mla_build.build()
+    return mla.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_what_binding_expects():
+    assert declared_functions() == sorted(mla.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", mla.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (mla_\w+)", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+
+
+def test_status_strings(lib):
+    for code, name in mla.STATUS.items():
+        assert mla.mla_status_string(code) == name
+    assert mla.mla_status_string(99) == "MLA_ERR_UNKNOWN"
+
+
+def _args(B=2, s_q=1, H=128, splits=0, max_len=4096, **kw):
+    a = mla.DecodeArgs()
+    fake = 0x10000
+    for f in ("q_lat", "q_pe", "kv_cache", "block_table", "seq_lens", "o_lat", "lse"):
+        setattr(a, f, fake)
+    a.B, a.s_q, a.H = B, s_q, H
+    a.d_c, a.d_r, a.page_size = 512, 64, 64
+    a.num_pages, a.max_pages_per_seq = 128, 64
+    a.kv_dtype, a.causal, a.num_splits, a.max_seq_len = 0, 0, splits, max_len
+    a.softmax_scale = 0.0722
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_workspace_size_is_host_only_and_grows_with_splits(lib):
+    one = mla.mla_decode_workspace_size(_args(splits=1))
+    assert one == 256
+    four = mla.mla_decode_workspace_size(_args(splits=4))
+    rows = 2 * 1 * 128 * 4
+    assert four >= 256 + rows * 512 * 4 + rows * 4
+    assert four % 256 == 0
+
+
+def test_auto_split_count(lib):
+    # few sequences, long context: many splits; many sequences: one or two
+    assert mla.mla_decode_num_splits(_args(B=4, H=16, max_len=131072)) >= 32
+    assert mla.mla_decode_num_splits(_args(B=128, H=128, max_len=8192, s_q=2)) == 1
+    assert mla.mla_decode_num_splits(_args(B=1, H=16, max_len=64)) == 1
+    assert mla.mla_decode_num_splits(_args(B=4, H=16, splits=7)) == 7
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("d_c", 256, UNSUPPORTED), ("d_r", 32, UNSUPPORTED), ("page_size", 32, UNSUPPORTED),
+    ("H", 24, UNSUPPORTED), ("H", 256, UNSUPPORTED), ("s_q", 3, UNSUPPORTED),
+    ("kv_dtype", 5, UNSUPPORTED), ("H", 0, INVALID), ("s_q", 0, INVALID), ("B", -1, INVALID),
+    ("num_splits", 129, INVALID), ("max_pages_per_seq", 0, INVALID),
+])
+def test_decode_rejects_bad_shapes(lib, field, value, code):
+    a = _args(**{field: value})
+    assert lib.mla_decode_paged(ctypes.byref(a), None) == code
+    assert lib.mla_combine_splits(ctypes.byref(a), None) == code
+    n = ctypes.c_size_t(0)
+    assert lib.mla_decode_workspace_size(ctypes.byref(a), ctypes.byref(n)) == code
+
+
+def test_decode_rejects_bad_pointers_and_workspace(lib):
+    a = _args()
+    assert lib.mla_decode_paged(ctypes.byref(a), None) == INVALID          # no workspace
+    a.workspace, a.workspace_bytes = 0x20001, 1 << 30
+    assert lib.mla_decode_paged(ctypes.byref(a), None) == MISALIGNED
+    a.workspace, a.workspace_bytes = 0x20000, 16
+    a.num_splits = 4
+    assert lib.mla_decode_paged(ctypes.byref(a), None) == WS_SMALL
+    a.workspace_bytes = 1 << 30
+    a.q_lat = None
+    assert lib.mla_decode_paged(ctypes.byref(a), None) == INVALID
+    a.q_lat = 0x10008
+    assert lib.mla_decode_paged(ctypes.byref(a), None) == MISALIGNED
+    a.q_lat = 0x10000
+    a.kv_dtype, a.kv_scale = 1, None                                       # fp8 needs scales
+    assert lib.mla_decode_paged(ctypes.byref(a), None) == INVALID
+
+
+def test_decode_with_empty_batch_enqueues_nothing(lib):
+    a = _args(B=0)
+    a.workspace, a.workspace_bytes = 0x20000, 256
+    assert lib.mla_decode_paged(ctypes.byref(a), None) == OK
+    assert lib.mla_combine_splits(ctypes.byref(a), None) == OK
+
+
+@pytest.mark.parametrize("fn", ["mla_absorb_q", "mla_up_proj_v"])
+def test_projection_argument_checks(lib, fn):
+    f = getattr(lib, fn)
+    p = 0x10000
+    assert f(p, p, p, 0, 128, 128, 512, None) == OK            # n_tok = 0: nothing to do
+    assert f(p, p, p, 4, 128, 64, 512, None) == UNSUPPORTED
+    assert f(p, p, p, 4, 128, 128, 256, None) == UNSUPPORTED
+    assert f(p, p, p, -1, 128, 128, 512, None) == INVALID
+    assert f(p, p, p, 4, 0, 128, 512, None) == INVALID
+    assert f(None, p, p, 4, 128, 128, 512, None) == INVALID
+    assert f(p, p + 2, p, 4, 128, 128, 512, None) == MISALIGNED
+
+
+def test_get_status_rejects_null(lib):
+    assert lib.mla_get_status(None, None) == INVALID
