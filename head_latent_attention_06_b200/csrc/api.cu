@@ -2,6 +2,7 @@
 // argument validation, split selection, workspace sizing and kernel launches.
 // Nothing here allocates device memory or synchronises, except mla_get_status.
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "common.cuh"
@@ -11,6 +12,9 @@ cudaError_t launch_absorb_q(const void*, const void*, void*, int, int, cudaStrea
 cudaError_t launch_up_proj_v(const void*, const void*, void*, int, int, cudaStream_t);
 cudaError_t launch_decode_mma(const mla_decode_args_t*, int, cudaStream_t);
 cudaError_t launch_combine(const mla_decode_args_t*, int, cudaStream_t);
+cudaError_t launch_decode_tc(const mla_decode_args_t*, int, cudaStream_t);
+bool decode_tc_supported(const mla_decode_args_t*);
+int decode_tc_clusters_per_split(const mla_decode_args_t*);
 int decode_mma_tiles(int len);
 int decode_mma_ctas_per_split(int s_q, int H, int B);
 }  // namespace mla
@@ -49,11 +53,36 @@ mla_status_t check_decode_shape(const mla_decode_args_t* a) {
   return MLA_OK;
 }
 
-// Split count: enough (sequence, row-group, split) CTAs to cover the SMs, but
-// never a split shorter than 8 tiles.
+// Which decode kernel runs: the tensor-memory kernel for the shapes it takes,
+// else the warp-MMA kernel.  MLA_DECODE_KERNEL=mma forces the latter (testing).
+bool use_tc(const mla_decode_args_t* a) {
+  const char* env = getenv("MLA_DECODE_KERNEL");
+  if (env && strcmp(env, "mma") == 0) return false;
+  return decode_tc_supported(a);
+}
+
+// Split count.  Tensor-memory kernel: the count that minimises the makespan
+// (waves of 74 CTA pairs x tiles per split), preferring fewer splits.  Warp-MMA
+// kernel: enough CTAs to cover the SMs, never a split shorter than 8 tiles.
 int choose_splits(const mla_decode_args_t* a) {
   if (a->num_splits > 0) return a->num_splits;
   const int max_len = a->max_seq_len > 0 ? a->max_seq_len : a->max_pages_per_seq * kPage;
+  if (use_tc(a)) {
+    const int tiles = (max_len + kPage - 1) / kPage;
+    const int units = decode_tc_clusters_per_split(a) > 0 ? decode_tc_clusters_per_split(a) : 1;
+    const int slots = kNumSMs / 2;
+    int best = 1;
+    long best_cost = -1;
+    for (int s = 1; s <= MLA_MAX_SPLITS && s <= (tiles > 0 ? tiles : 1); ++s) {
+      const long waves = ((long)units * s + slots - 1) / slots;
+      const long cost = waves * ((tiles + s - 1) / s) * 100 + s;  // + s: combine work, tie-break
+      if (best_cost < 0 || cost < best_cost) {
+        best_cost = cost;
+        best = s;
+      }
+    }
+    return best;
+  }
   const int tiles = decode_mma_tiles(max_len);
   const int ctas = decode_mma_ctas_per_split(a->s_q, a->H, a->B > 0 ? a->B : 1);
   int s = (kNumSMs + ctas - 1) / ctas;
@@ -125,6 +154,7 @@ mla_status_t mla_decode_paged(const mla_decode_args_t* a, void* stream) {
   const int splits = choose_splits(a);
   st = check_decode_ptrs(a, splits);
   if (st != MLA_OK || a->B == 0) return st;
+  if (use_tc(a)) return from_cuda(launch_decode_tc(a, splits, (cudaStream_t)stream));
   return from_cuda(launch_decode_mma(a, splits, (cudaStream_t)stream));
 }
 

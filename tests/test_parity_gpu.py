@@ -74,6 +74,15 @@ def test_small_cases_every_element(cuda_lib, kv, H, s_q, causal, lens, splits):
     check_close("o (definition)", to_np(st.out)[sel], ref2["o"][sel], kv)
 
 
+@pytest.mark.parametrize("lens,splits", [([1, 63, 64, 65, 200, 1000], 1), ([700, 3], 4)])
+def test_warp_mma_kernel_on_128_heads(cuda_lib, monkeypatch, lens, splits):
+    """The portable warp-MMA kernel, forced for a shape the tensor-memory kernel takes."""
+    monkeypatch.setenv("MLA_DECODE_KERNEL", "mma")
+    w = make_workload(_spec("bf16", 128, 1, lens))
+    st = _run(cuda_lib, w, splits)
+    compare_step(st, w, oracle_of(w, absorbed=True))
+
+
 def test_empty_and_short_contexts(cuda_lib):
     w = make_workload(_spec("bf16", 16, 2, [0, 1, 2, 70], causal=True))
     for splits in (1, 4):
@@ -85,8 +94,9 @@ def test_empty_and_short_contexts(cuda_lib):
         compare_step(st, w, ref)
 
 
-def test_split_count_invariance(cuda_lib):
-    w = make_workload(_spec("bf16", 128, 1, [3000, 4096, 17]))
+@pytest.mark.parametrize("H", [128, 64])
+def test_split_count_invariance(cuda_lib, H):
+    w = make_workload(_spec("bf16", H, 1, [3000, 4096, 17]))
     outs = [to_np(_run(cuda_lib, w, s).out) for s in (1, 2, 7, 32)]
     for o in outs[1:]:
         ma, rl = errors(o, outs[0])
@@ -94,9 +104,10 @@ def test_split_count_invariance(cuda_lib):
 
 
 @pytest.mark.parametrize("kv", ["bf16", "fp8"])
-def test_page_permutation_is_bit_exact(cuda_lib, kv):
-    a = make_workload(_spec(kv, 64, 1, [500, 129], permute=False))
-    b = make_workload(_spec(kv, 64, 1, [500, 129], permute=True))
+@pytest.mark.parametrize("H", [64, 128])
+def test_page_permutation_is_bit_exact(cuda_lib, kv, H):
+    a = make_workload(_spec(kv, H, 1, [500, 129], permute=False))
+    b = make_workload(_spec(kv, H, 1, [500, 129], permute=True))
     assert not torch.equal(a.block_table, b.block_table)
     oa, ob = _run(cuda_lib, a).out, _run(cuda_lib, b).out
     assert torch.equal(oa, ob)
@@ -124,9 +135,10 @@ def test_projections_against_oracle(cuda_lib):
     assert rl <= 4e-3 and ma <= 4e-2, (ma, rl)
 
 
-def test_device_checks_report_bad_block_table_and_length(cuda_lib):
+@pytest.mark.parametrize("H", [16, 128])
+def test_device_checks_report_bad_block_table_and_length(cuda_lib, H):
     from head_latent_attention_06_b200.step import step_from_workload
-    w = make_workload(_spec("bf16", 16, 1, [130, 64]))
+    w = make_workload(_spec("bf16", H, 1, [130, 64]))
     st = step_from_workload(w)
     bt = st._keep[2]
     bt[0, 1] = 10_000                     # page id beyond the cache: skipped, reported
