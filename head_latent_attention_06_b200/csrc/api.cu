@@ -61,8 +61,8 @@ bool use_tc(const mla_decode_args_t* a) {
   return decode_tc_supported(a);
 }
 
-// Split count.  Tensor-memory kernel: the count that minimises the makespan
-// (waves of 74 CTA pairs x tiles per split), preferring fewer splits.  Warp-MMA
+// Split count.  Tensor-memory kernel: the count that minimises the modelled
+// makespan (waves of 74 CTA pairs x per-unit work), preferring fewer splits.  Warp-MMA
 // kernel: enough CTAs to cover the SMs, never a split shorter than 8 tiles.
 int choose_splits(const mla_decode_args_t* a) {
   if (a->num_splits > 0) return a->num_splits;
@@ -75,7 +75,9 @@ int choose_splits(const mla_decode_args_t* a) {
     long best_cost = -1;
     for (int s = 1; s <= MLA_MAX_SPLITS && s <= (tiles > 0 ? tiles : 1); ++s) {
       const long waves = ((long)units * s + slots - 1) / slots;
-      const long cost = waves * ((tiles + s - 1) / s) * 100 + s;  // + s: combine work, tie-break
+      // a work unit costs its tiles plus about 8 tiles of start-up (Q load, first
+      // pages, epilogue); more than one split adds the combine pass
+      const long cost = waves * ((tiles + s - 1) / s + 8) * 100 + (s > 1 ? 400 : 0) + s;
       if (best_cost < 0 || cost < best_cost) {
         best_cost = cost;
         best = s;

@@ -13,10 +13,17 @@
 // is the paired form (cta_group::2, M = 128): CTA r holds the Q rows of heads
 // 64r .. 64r+63 and receives their S and O rows in its TMEM.  Per 64-token page:
 //   S  (M=128, N=64,  K=576): B = the page's tokens; CTA r supplies its 32
-//        tokens x 576 from its "S ring" stage (9 TMA boxes of 32 x 64).
+//        tokens x 576 (9 TMA boxes of 32 x 64).
 //   PV (M=128, N=256, K=64) twice (latent 0..255, 256..511): B = all 64 tokens x
-//        the CTA's 128-column half of each N tile, from its "V ring" stage
-//        (4 TMA boxes of 64 x 64, a second read of the page that hits L2).
+//        the CTA's 128-column half of each N tile (4 TMA boxes of 64 x 64, a
+//        second read of the page that hits L2).
+// The cache streams through two rings, one for the score operand (S stages of
+// 36 KB) and one for the value operand (V stages of 32 KB), in the order the
+// MMAs consume them.  Only the even CTA posts the expected byte count of a stage
+// (both CTAs' bytes) on its own barrier; the odd CTA's TMA completes its bytes
+// there without arriving; each slot is released by the commit of the MMAs that read it, so
+// the producer refills it at once.  Each CTA also prefetches its half of the
+// page four tiles ahead into L2 with a bulk prefetch.
 // TMEM per CTA (2x2 datapath layout of the paired M = 128 MMA): O takes 256
 // columns, each S buffer 32 columns (two buffers).  Lane l < 64 holds head row l
 // for the first half of every N tile, lane 64 + l the same row for the second.
@@ -25,8 +32,9 @@
 // the even CTA) the single MMA issuer, warps 2..5 softmax / correction /
 // epilogue, one thread per TMEM lane.  The MMA order S(0), S(1), PV(0), S(2),
 // PV(1), ... lets S(t+2) run on the tensor pipe while the softmax of t+1 runs.
-// The output rescale is lazy: the reference maximum moves only when the tile
-// maximum exceeds it by more than 2^8, so O in TMEM is rarely touched.
+// P is double-buffered in shared memory, so the softmax of t+1 never waits for
+// P.V of t.  The output rescale is lazy: the reference maximum moves only when
+// the tile maximum exceeds it by more than 2^8, so O in TMEM is rarely touched.
 //
 // Every mbarrier wait is bounded (MLA_ERR_DEVICE_TIMEOUT in the status word,
 // then an orderly exit that drains issued MMAs and frees TMEM).
@@ -45,22 +53,34 @@ constexpr int kThreads = 192;
 constexpr uint32_t kChunkQ = 64 * 128;              // 64 rows x 64 bf16
 constexpr uint32_t kQBytes = 9 * kChunkQ;           // 73728
 constexpr uint32_t kChunkS = 32 * 128;              // 32 tokens x 64 bf16
-constexpr uint32_t kSStage = 9 * kChunkS;           // 36864
+constexpr uint32_t kSStage = 9 * kChunkS;           // 36864: the CTA's 32 tokens x 576
 constexpr uint32_t kChunkV = 64 * 128;              // 64 tokens x 64 bf16
-constexpr uint32_t kVStage = 4 * kChunkV;           // 32768
+constexpr uint32_t kVStage = 4 * kChunkV;           // 32768: 64 tokens x the CTA's 4 latent chunks
+constexpr int kStages = 2;
 constexpr uint32_t kPBytes = 64 * 128;              // 64 rows x 64 tokens bf16
 constexpr uint32_t kQOff = 0;
 constexpr uint32_t kSOff = kQOff + kQBytes;
-constexpr uint32_t kVOff = kSOff + 2 * kSStage;
-constexpr uint32_t kPOff = kVOff + 2 * kVStage;
-constexpr uint32_t kBarOff = kPOff + kPBytes;
-enum Bar { Q_FULL = 0, S_FULL = 1, S_EMPTY = 3, V_FULL = 5, V_EMPTY = 7, S_READY = 9, P_READY = 11,
-           O_DONE = 12, DRAIN = 13, NBARS = 14 };
-constexpr uint32_t kMiscOff = kBarOff + 8 * 16;
+constexpr uint32_t kVOff = kSOff + kStages * kSStage;
+constexpr uint32_t kPOff = kVOff + kStages * kVStage;  // two P buffers
+constexpr uint32_t kBarOff = kPOff + 2 * kPBytes;
+// barrier indices
+constexpr int S_FULL = 0;                 // [kStages] in the even CTA: stage filled in both CTAs
+constexpr int S_EMPTY = S_FULL + kStages; // [kStages] in each CTA: stage consumed by the MMAs
+constexpr int V_FULL = S_EMPTY + kStages;
+constexpr int V_EMPTY = V_FULL + kStages;
+constexpr int Q_FULL = V_EMPTY + kStages;
+constexpr int S_READY = Q_FULL + 1;       // [2]
+constexpr int P_READY = S_READY + 2;      // [2] in the even CTA
+constexpr int O_DONE = P_READY + 2;       // [2]
+constexpr int DRAIN = O_DONE + 2;
+constexpr int NBARS = DRAIN + 1;
+constexpr int kPrefetchTiles = 4;                    // L2 prefetch distance of the cache stream
+constexpr uint32_t kMiscOff = kBarOff + 8 * NBARS;
 constexpr uint32_t kXmaxOff = kMiscOff + 16;         // float [2][128]
 constexpr uint32_t kXlOff = kXmaxOff + 2 * 128 * 4;  // float [128]
 constexpr uint32_t kSmemUsed = kXlOff + 128 * 4;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;    // + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 256;                     // S buffers at columns 256, 288
 constexpr uint64_t kWaitLimitNs = 2000000000ull;     // 2 s
@@ -70,6 +90,7 @@ constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
 
 struct TcParams {
+  const uint8_t* kv;
   const int32_t* block_table;
   const int32_t* seq_lens;
   __nv_bfloat16* o_lat;
@@ -131,16 +152,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     if (bad_len && r == 0 && g == 0 && split == 0) set_status(p.status, MLA_ERR_BAD_SEQ_LEN);
     *abort_flag = 0;
-    mbar_init(own_bar(Q_FULL), 2);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(own_bar(S_FULL + i), 2);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(own_bar(S_FULL + i), 1);
       mbar_init(own_bar(S_EMPTY + i), 1);
-      mbar_init(own_bar(V_FULL + i), 2);
+      mbar_init(own_bar(V_FULL + i), 1);
       mbar_init(own_bar(V_EMPTY + i), 1);
-      mbar_init(own_bar(S_READY + i), 1);
     }
-    mbar_init(own_bar(P_READY), 2);
-    mbar_init(own_bar(O_DONE), 1);
+    mbar_init(own_bar(Q_FULL), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(own_bar(S_READY + i), 1);
+      mbar_init(own_bar(P_READY + i), 2);
+      mbar_init(own_bar(O_DONE + i), 1);
+    }
     mbar_init(own_bar(DRAIN), 1);
     fence_mbar_init();
   }
@@ -156,6 +179,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // =========================== TMA producer ===========================
+    // Ring order = MMA order: S(0), S(1), V(0), S(2), V(1), ... where S(u) is the
+    // CTA's 32 tokens x 576 of page u (9 slots) and V(u) the page's 64 tokens x
+    // the CTA's latent columns of both P.V halves (8 slots of 16 tokens x 128).
     if (n > 0) {
       if (lane == 0) {
         prefetch_tmap(&tm_q);
@@ -164,12 +190,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_kv);
         const int qrow = (b * p.s_q + g) * p.H + 64 * (int)r;
         const uint32_t qb = lead_bar(Q_FULL);
-        mbar_arrive_expect_tx_cluster(qb, kQBytes);
+        if (r == 0) mbar_arrive_expect_tx_local(own_bar(Q_FULL), 2 * kQBytes);
         for (int c = 0; c < 8; ++c) tma_load_2d_pair(sa + kQOff + c * kChunkQ, &tm_q, qb, 64 * c, qrow);
         tma_load_2d_pair(sa + kQOff + 8 * kChunkQ, &tm_qpe, qb, 0, qrow);
       }
       // physical pages, fetched 32 at a time by the whole warp
-      int blk_s = -1, pg_s = 0, blk_v = -1, pg_v = 0;
+      int blk_s = -1, pg_s = 0, blk_v = -1, pg_v = 0, blk_p = -1, pg_p = 0;
       auto page_of = [&](int u, int& blk, int& pg) -> int {
         if ((u >> 5) != blk) {
           blk = u >> 5;
@@ -183,36 +209,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         return __shfl_sync(0xffffffffu, pg, u & 31);
       };
+      // the CTA's half page (32 contiguous rows) of tile u, into L2 ahead of its TMA
+      auto prefetch = [&](int u) {
+        const int pg = page_of(u, blk_p, pg_p);
+        if (lane == 0) prefetch_l2_bulk(p.kv + ((size_t)pg * kPage + 32 * r) * kRow * 2, kSStage);
+      };
+      for (int u = 0; u < n && u < kPrefetchTiles; ++u) prefetch(u);
       auto load_s = [&](int u) -> bool {
-        const int st = u & 1;
-        bool ok = mbar_wait(own_bar(S_EMPTY + st), ((u >> 1) & 1) ^ 1, abort_flag, p.status, kWaitLimitNs);
-        if (!__all_sync(0xffffffffu, ok)) return false;
+        const int st = u % kStages;
+        const uint32_t ph = ((u / kStages) & 1) ^ 1;
+        if (!mbar_wait_converged(own_bar(S_EMPTY + st), ph, abort_flag, p.status, kWaitLimitNs)) return false;
         const int pg = page_of(u, blk_s, pg_s);
-        if (lane == 0) {
-          const uint32_t fb = lead_bar(S_FULL + st);
-          mbar_arrive_expect_tx_cluster(fb, kSStage);
-          const uint32_t dst = sa + kSOff + st * kSStage;
-          for (int c = 0; c < 9; ++c)
-            tma_load_2d_pair(dst + c * kChunkS, &tm_ks, fb, 64 * c, pg * kPage + 32 * (int)r);
-        }
-        __syncwarp();
+        const uint32_t fb = lead_bar(S_FULL + st);
+        if (r == 0) mbar_arrive_expect_tx_local_elect(own_bar(S_FULL + st), 2 * kSStage);
+        const uint32_t dst = sa + kSOff + st * kSStage;
+        for (int c = 0; c < 9; ++c)
+          tma_load_2d_pair_elect(dst + c * kChunkS, &tm_ks, fb, 64 * c, pg * kPage + 32 * (int)r);
+        if (u + kPrefetchTiles < n) prefetch(u + kPrefetchTiles);
         return true;
       };
       auto load_v = [&](int u) -> bool {
-        const int st = u & 1;
-        bool ok = mbar_wait(own_bar(V_EMPTY + st), ((u >> 1) & 1) ^ 1, abort_flag, p.status, kWaitLimitNs);
-        if (!__all_sync(0xffffffffu, ok)) return false;
+        const int st = u % kStages;
+        const uint32_t ph = ((u / kStages) & 1) ^ 1;
+        if (!mbar_wait_converged(own_bar(V_EMPTY + st), ph, abort_flag, p.status, kWaitLimitNs)) return false;
         const int pg = page_of(u, blk_v, pg_v);
-        if (lane == 0) {
-          const uint32_t fb = lead_bar(V_FULL + st);
-          mbar_arrive_expect_tx_cluster(fb, kVStage);
-          const uint32_t dst = sa + kVOff + st * kVStage;
-          for (int j = 0; j < 4; ++j) {
-            const int lc = (j < 2) ? 2 * (int)r + j : 4 + 2 * (int)r + (j - 2);  // latent chunk
-            tma_load_2d_pair(dst + j * kChunkV, &tm_kv, fb, 64 * lc, pg * kPage);
-          }
+        const uint32_t fb = lead_bar(V_FULL + st);
+        if (r == 0) mbar_arrive_expect_tx_local_elect(own_bar(V_FULL + st), 2 * kVStage);
+        const uint32_t dst = sa + kVOff + st * kVStage;
+        for (int j = 0; j < 4; ++j) {
+          const int lc = 4 * (j >> 1) + 2 * (int)r + (j & 1);  // latent chunk: halves {2r, 2r+1}, {4+2r, 5+2r}
+          tma_load_2d_pair_elect(dst + j * kChunkV, &tm_kv, fb, 64 * lc, pg * kPage);
         }
-        __syncwarp();
         return true;
       };
       bool ok = load_s(0);
@@ -224,60 +251,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // =========================== MMA issuer (even CTA) ===========================
     if (r == 0 && n > 0) {
-      bool ok = mbar_wait(own_bar(Q_FULL), 0, abort_flag, p.status, kWaitLimitNs);
-      ok = __all_sync(0xffffffffu, ok);
+      bool ok = mbar_wait_converged(own_bar(Q_FULL), 0, abort_flag, p.status, kWaitLimitNs);
+      const uint64_t dq = desc_sw128(sa + kQOff, 16, 1024);
+      const uint64_t ds = desc_sw128(sa + kSOff, 16, 1024);
+      const uint64_t dv = desc_sw128(sa + kVOff, kChunkV, 1024);
+      const uint64_t dp = desc_sw128(sa + kPOff, 16, 1024);
       auto issue_s = [&](int u) -> bool {
-        const int st = u & 1;
-        bool w = mbar_wait(own_bar(S_FULL + st), (u >> 1) & 1, abort_flag, p.status, kWaitLimitNs);
-        if (!__all_sync(0xffffffffu, w)) return false;
-        if (lane == 0) {
-          tc_fence_after();
-          const uint32_t d = tmem + kTmemS + 32u * st;
-#pragma unroll 1
-          for (int c = 0; c < 9; ++c) {
+        const int st = u % kStages, sb = u & 1;
+        if (!mbar_wait_converged(own_bar(S_FULL + st), (u / kStages) & 1, abort_flag, p.status, kWaitLimitNs))
+          return false;
+        tc_fence_after();
+        const uint32_t d = tmem + kTmemS + 32u * sb;
+        const uint64_t bs0 = ds + ((st * kSStage) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = desc_sw128(sa + kQOff + c * kChunkQ + kk * 32, 16, 1024);
-              const uint64_t bd = desc_sw128(sa + kSOff + st * kSStage + c * kChunkS + kk * 32, 16, 1024);
-              mma_pair(d, ad, bd, kIdescS, (c | kk) != 0);
-            }
-          }
-          commit_pair_mc(own_bar(S_EMPTY + st), 0x3);
-          commit_pair_mc(own_bar(S_READY + st), 0x3);
+        for (int c = 0; c < 9; ++c) {
+          const uint64_t aq = dq + ((c * kChunkQ) >> 4), bs = bs0 + ((c * kChunkS) >> 4);
+          mma_pair_elect(d, aq, bs, kIdescS, c != 0);
+          mma_pair_elect(d, aq + 2, bs + 2, kIdescS, 1);
+          mma_pair_elect(d, aq + 4, bs + 4, kIdescS, 1);
+          mma_pair_elect(d, aq + 6, bs + 6, kIdescS, 1);
         }
-        __syncwarp();
+        commit_pair_mc_elect(own_bar(S_EMPTY + st), 0x3);
+        commit_pair_mc_elect(own_bar(S_READY + sb), 0x3);
+        return true;
+      };
+      auto issue_pv = [&](int t) -> bool {
+        const int pb = t & 1, st = t % kStages;
+        if (!mbar_wait_converged(own_bar(P_READY + pb), (t >> 1) & 1, abort_flag, p.status, kWaitLimitNs))
+          return false;
+        if (!mbar_wait_converged(own_bar(V_FULL + st), (t / kStages) & 1, abort_flag, p.status, kWaitLimitNs))
+          return false;
+        tc_fence_after();
+        const uint64_t ap = dp + ((pb * kPBytes) >> 4);
+        const uint64_t bv = dv + ((st * kVStage) >> 4);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_pair_elect(tmem + 128u * h, ap + kk * 2, bv + ((2 * h * kChunkV + kk * 2048) >> 4), kIdescPV,
+                           (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        commit_pair_mc_elect(own_bar(V_EMPTY + st), 0x3);
+        commit_pair_mc_elect(own_bar(O_DONE + pb), 0x3);
         return true;
       };
       if (ok) ok = issue_s(0);
       if (ok && n > 1) ok = issue_s(1);
       for (int t = 0; ok && t < n; ++t) {
-        const int st = t & 1;
-        bool w = mbar_wait(own_bar(P_READY), t & 1, abort_flag, p.status, kWaitLimitNs);
-        if (w) w = mbar_wait(own_bar(V_FULL + st), (t >> 1) & 1, abort_flag, p.status, kWaitLimitNs);
-        if (!__all_sync(0xffffffffu, w)) break;
-        if (lane == 0) {
-          tc_fence_after();
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = desc_sw128(sa + kPOff + kk * 32, 16, 1024);
-              const uint64_t bd =
-                  desc_sw128(sa + kVOff + st * kVStage + 2 * h * kChunkV + kk * 2048, kChunkV, 1024);
-              mma_pair(tmem + 128u * h, ad, bd, kIdescPV, (t > 0 || kk > 0) ? 1u : 0u);
-            }
-          }
-          commit_pair_mc(own_bar(V_EMPTY + st), 0x3);
-          commit_pair_mc(own_bar(O_DONE), 0x3);
-        }
-        __syncwarp();
-        if (t + 2 < n) ok = issue_s(t + 2);
+        ok = issue_pv(t);
+        if (ok && t + 2 < n) ok = issue_s(t + 2);
       }
       // every issued MMA has completed before TMEM is released
-      if (lane == 0) commit_pair_mc(own_bar(DRAIN), 0x1);
-      __syncwarp();
+      commit_pair_mc_elect(own_bar(DRAIN), 0x1);
       int dummy = 0;
-      mbar_wait(own_bar(DRAIN), 0, &dummy, p.status, kWaitLimitNs);
+      mbar_wait_converged(own_bar(DRAIN), 0, &dummy, p.status, kWaitLimitNs);
     }
   } else {
     // ====================== softmax / correction / epilogue ======================
@@ -330,12 +357,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         l += p0 + p1;
         pk[j >> 1] = pack_bf16(p0, p1);
       }
-      if (t > 0) {
-        w = mbar_wait(own_bar(O_DONE), (t - 1) & 1, abort_flag, p.status, kWaitLimitNs);
+      // P buffer sb was last read by PV(t-2)
+      if (t >= 2) {
+        w = mbar_wait(own_bar(O_DONE + sb), ((t - 2) >> 1) & 1, abort_flag, p.status, kWaitLimitNs);
+        if (group_any(!w)) { alive = false; break; }
+      }
+      // O may only be rescaled once PV(t-1) has finished accumulating into it
+      const bool any_resc = group_any(resc);
+      if (any_resc && t >= 1) {
+        w = mbar_wait(own_bar(O_DONE + (sb ^ 1)), ((t - 1) >> 1) & 1, abort_flag, p.status, kWaitLimitNs);
         if (group_any(!w)) { alive = false; break; }
         tc_fence_after();
       }
-      if (__any_sync(0xffffffffu, resc)) {
+      if (any_resc) {
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           uint32_t ov[32];
@@ -348,7 +382,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_wait_st();
       }
       // P row m, tokens 32*half .. +31: four 16-byte chunks of the 128-byte row
-      uint8_t* prow = sm + kPOff + m * 128;
+      uint8_t* prow = sm + kPOff + sb * kPBytes + m * 128;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int q = 4 * half + k;
@@ -358,10 +392,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(1, 128);
-      if (lt == 0) mbar_arrive_cluster(lead_bar(P_READY));
+      if (lt == 0) mbar_arrive_remote(lead_bar(P_READY + sb));
     }
     if (alive && n > 0) {
-      bool w = mbar_wait(own_bar(O_DONE), (n - 1) & 1, abort_flag, p.status, kWaitLimitNs);
+      bool w = mbar_wait(own_bar(O_DONE + ((n - 1) & 1)), ((n - 1) >> 1) & 1, abort_flag, p.status,
+                         kWaitLimitNs);
       if (group_any(!w)) alive = false;
       tc_fence_after();
     }
@@ -471,6 +506,7 @@ cudaError_t launch_decode_tc(const mla_decode_args_t* a, int splits, cudaStream_
       !encode_2d(&tm_kv, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 64))
     return cudaErrorInvalidValue;
   TcParams p;
+  p.kv = static_cast<const uint8_t*>(a->kv_cache);
   p.block_table = a->block_table;
   p.seq_lens = a->seq_lens;
   p.o_lat = static_cast<__nv_bfloat16*>(a->o_lat);

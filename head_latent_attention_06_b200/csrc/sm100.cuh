@@ -42,32 +42,54 @@ MLA_DEVI void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.clus
 MLA_DEVI void mbar_arrive_cluster(uint32_t addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
 }
+// Arrive (count 1) on a barrier of this or the peer CTA with the default
+// release semantics at CTA scope.
+MLA_DEVI void mbar_arrive_remote(uint32_t addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+MLA_DEVI void mbar_arrive_expect_tx_local(uint32_t addr, uint32_t tx) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(addr), "r"(tx) : "memory");
+}
 MLA_DEVI void mbar_arrive_expect_tx_cluster(uint32_t addr, uint32_t tx) {
   asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(addr),
                "r"(tx)
                : "memory");
 }
+// try_wait with acquire at CTA scope (TMA bytes and tcgen05 commits) or at
+// cluster scope (arrivals of the peer CTA's threads after their own writes).
+template <bool kCluster = false>
 MLA_DEVI bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(addr), "r"(parity)
-      : "memory");
+  if (kCluster) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity)
+        : "memory");
+  }
   return ok != 0;
 }
 
 // Waits for the phase with the given parity.  Bounded: gives up after
 // `limit_ns` of wall time or as soon as *abort is set, records
 // MLA_ERR_DEVICE_TIMEOUT in `status` when it times out, and returns false.
+template <bool kCluster = false>
 MLA_DEVI bool mbar_wait(uint32_t addr, uint32_t parity, volatile int* abort, uint32_t* status,
                         uint64_t limit_ns) {
-  if (mbar_try_wait(addr, parity)) return true;
+  if (mbar_try_wait<kCluster>(addr, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(addr, parity)) return true;
+    if (mbar_try_wait<kCluster>(addr, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort) return false;
       if (globaltimer() - t0 > limit_ns) {
@@ -75,6 +97,40 @@ MLA_DEVI bool mbar_wait(uint32_t addr, uint32_t parity, volatile int* abort, uin
         set_status(status, MLA_ERR_DEVICE_TIMEOUT);
         return false;
       }
+    }
+  }
+}
+
+// Warp-level form: lane 0 waits, the result is broadcast to the warp.
+template <bool kCluster = false>
+MLA_DEVI bool mbar_wait_warp(uint32_t addr, uint32_t parity, volatile int* abort, uint32_t* status,
+                             uint64_t limit_ns) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait<kCluster>(addr, parity, abort, status, limit_ns) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Converged-warp form: every lane polls, the loop exits uniformly.  Bounded
+// like mbar_wait.
+template <bool kCluster = false>
+MLA_DEVI bool mbar_wait_converged(uint32_t addr, uint32_t parity, volatile int* abort, uint32_t* status,
+                                  uint64_t limit_ns) {
+  if (__all_sync(0xffffffffu, mbar_try_wait<kCluster>(addr, parity))) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (__all_sync(0xffffffffu, mbar_try_wait<kCluster>(addr, parity))) return true;
+    if ((it & 255u) == 0) {
+      int stop = 0;
+      if ((threadIdx.x & 31) == 0) {
+        if (*abort) {
+          stop = 1;
+        } else if (globaltimer() - t0 > limit_ns) {
+          *abort = 1;
+          set_status(status, MLA_ERR_DEVICE_TIMEOUT);
+          stop = 1;
+        }
+      }
+      if (__shfl_sync(0xffffffffu, stop, 0)) return false;
     }
   }
 }
@@ -89,6 +145,34 @@ MLA_DEVI void tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t mbar_clu
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(tmap), "r"(mbar_cluster), "r"(x), "r"(y)
       : "memory");
+}
+
+// Same, executed by a converged warp: one elected lane issues.
+MLA_DEVI void tma_load_2d_pair_elect(uint32_t dst, const void* tmap, uint32_t mbar_cluster, int32_t x,
+                                     int32_t y) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 rx;\n\t"
+      "elect.sync rx|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];\n\t}" ::"r"(dst),
+      "l"(tmap), "r"(mbar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+// Arrive with an expected byte count on a barrier of this CTA (CTA-scope
+// release: the bytes themselves are counted by the TMA engine).
+MLA_DEVI void mbar_arrive_expect_tx_local_elect(uint32_t addr, uint32_t tx) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 rx;\n\t"
+      "elect.sync rx|e, 0xffffffff;\n\t"
+      "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(addr),
+      "r"(tx)
+      : "memory");
+}
+
+// Brings `bytes` (multiple of 16) of global memory at a 16-byte aligned address
+// into L2 without touching shared memory.
+MLA_DEVI void prefetch_l2_bulk(const void* gaddr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gaddr), "r"(bytes) : "memory");
 }
 
 MLA_DEVI void prefetch_tmap(const void* tmap) {
@@ -140,6 +224,27 @@ MLA_DEVI void mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Converged-warp forms of the two above: one elected lane issues.
+MLA_DEVI void mma_pair_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 rx;\n\t"
+      "elect.sync rx|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+MLA_DEVI void commit_pair_mc_elect(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 rx;\n\t"
+      "elect.sync rx|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;\n\t}" ::"r"(bar),
+      "h"(cta_mask)
       : "memory");
 }
 
