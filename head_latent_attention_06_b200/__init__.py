@@ -29,7 +29,7 @@ STATUS = {
 # Every symbol include/mla.h declares.
 EXPORTS = ("mla_absorb_q", "mla_decode_workspace_size", "mla_decode_num_splits",
            "mla_decode_paged", "mla_combine_splits", "mla_up_proj_v", "mla_get_status",
-           "mla_status_string")
+           "mla_status_string", "mla_decode_paged_noalloc")
 
 
 class MlaError(RuntimeError):
@@ -74,6 +74,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_decode_num_splits.argtypes = [pa, ctypes.POINTER(ctypes.c_int32)]
     lib.mla_decode_paged.argtypes = [pa, vp]
     lib.mla_combine_splits.argtypes = [pa, vp]
+    lib.mla_decode_paged_noalloc.argtypes = [pa, vp]
     lib.mla_get_status.argtypes = [vp, vp]
     lib.mla_status_string.argtypes = [ctypes.c_int]
     lib.mla_status_string.restype = ctypes.c_char_p
@@ -182,6 +183,12 @@ def mla_decode_paged(args: DecodeArgs, stream=None):
 
 def mla_combine_splits(args: DecodeArgs, stream=None):
     _check("mla_combine_splits", load().mla_combine_splits(ctypes.byref(args), _stream(stream)))
+
+
+def mla_decode_paged_noalloc(args: DecodeArgs, stream=None):
+    """Decode plus split merge with the library's built-in scratch (args.workspace is
+    ignored); for callers that cannot allocate device memory."""
+    _check("mla_decode_paged_noalloc", load().mla_decode_paged_noalloc(ctypes.byref(args), _stream(stream)))
 
 
 def mla_get_status(workspace, stream=None) -> int:

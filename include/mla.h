@@ -151,6 +151,25 @@ mla_status_t mla_combine_splits(const mla_decode_args_t* args, void* stream);
 mla_status_t mla_up_proj_v(const void* o_lat, const void* w_uv, void* out,
                            int32_t n_tok, int32_t H, int32_t d_v, int32_t d_c, void* stream);
 
+/*
+ * mla_decode_paged_noalloc — mla_decode_paged followed by mla_combine_splits,
+ * for callers that cannot allocate device memory (for example a plugin inside
+ * an engine that owns all device memory and forbids allocations after start-up,
+ * or a latency-critical path where an allocation could synchronise the device).
+ * The pages describe no such entry point; it is a deployment convenience.
+ * It ignores args->workspace and uses a scratch array built into the library
+ * instead: 16 MiB of device memory on every GPU that loads the library, held
+ * until the process exits.  A problem needing more scratch than that (see
+ * mla_decode_workspace_size) is rejected with MLA_ERR_WORKSPACE_TOO_SMALL
+ * before anything is enqueued.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress); make that first call before
+ * any stream capture.  Every call shares the array: calls that overlap on the
+ * GPU race, so order them on one stream or with events.  The call allocates
+ * nothing (it clears the array's status word with cudaMemsetAsync); device-side
+ * status words are not reported through this entry point.
+ */
+mla_status_t mla_decode_paged_noalloc(const mla_decode_args_t* args, void* stream);
+
 /* Waits for `stream`, returns the sticky device status word of `workspace`
  * (MLA_OK if no device-side problem was recorded) and clears it. */
 mla_status_t mla_get_status(void* workspace, void* stream);
