@@ -19,6 +19,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
                                                       int splits) {
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  pdl_trigger();
+  pdl_wait();
   if (row >= rows) return;
   const float* lp = lse_part + (size_t)row * splits;
   float m = -CUDART_INF_F;
@@ -68,11 +70,10 @@ cudaError_t launch_combine(const mla_decode_args_t* a, int splits, cudaStream_t 
   const int rows = n_tok * a->H;
   WorkspaceLayout wl = workspace_layout(n_tok, a->H, splits);
   const unsigned char* ws = static_cast<const unsigned char*>(a->workspace);
-  combine_kernel<<<(rows + 3) / 4, 128, 0, stream>>>(
-      reinterpret_cast<const float*>(ws + wl.o_part_off),
-      reinterpret_cast<const float*>(ws + wl.lse_part_off), static_cast<__nv_bfloat16*>(a->o_lat),
-      a->lse, rows, splits);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3((rows + 3) / 4), dim3(128), 0, stream,
+                    reinterpret_cast<const float*>(ws + wl.o_part_off),
+                    reinterpret_cast<const float*>(ws + wl.lse_part_off),
+                    static_cast<__nv_bfloat16*>(a->o_lat), a->lse, rows, splits);
 }
 
 }  // namespace mla

@@ -39,6 +39,31 @@ inline WorkspaceLayout workspace_layout(int n_tok, int H, int splits) {
   return w;
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialisation may start while the previous kernel of the stream still runs;
+// pdl_wait() blocks until that kernel has completed and its writes are visible,
+// so nothing the previous kernel writes may be read before it.  pdl_trigger()
+// lets the next kernel of the stream be scheduled early (a scheduling hint only).
+MLA_DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+MLA_DEVI void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launches `kern` on `stream` with programmatic stream serialisation allowed.
+template <typename Kern, typename... Args>
+inline cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 MLA_DEVI void set_status(uint32_t* status, uint32_t code) {
   if (status) atomicCAS(status, 0u, code);
 }

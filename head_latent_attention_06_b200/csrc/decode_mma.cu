@@ -75,6 +75,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_mma_kernel(DecodeParams p)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_rows = p.s_q * p.H;
   const int row0 = g * ROWS;
+  pdl_trigger();
+  pdl_wait();
 
   int L = p.seq_lens[b];
   if (L < 0 || L > p.max_pages * kPage) {
@@ -370,12 +372,12 @@ cudaError_t launch_decode_mma(const mla_decode_args_t* a, int splits, cudaStream
     e = cudaFuncSetAttribute(decode_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)Smem<true>::total);
     if (e != cudaSuccess) return e;
-    decode_mma_kernel<true><<<grid, NTHREADS, Smem<true>::total, stream>>>(p);
+    return launch_pdl(decode_mma_kernel<true>, grid, dim3(NTHREADS), Smem<true>::total, stream, p);
   } else {
     e = cudaFuncSetAttribute(decode_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)Smem<false>::total);
     if (e != cudaSuccess) return e;
-    decode_mma_kernel<false><<<grid, NTHREADS, Smem<false>::total, stream>>>(p);
+    return launch_pdl(decode_mma_kernel<false>, grid, dim3(NTHREADS), Smem<false>::total, stream, p);
   }
   return cudaGetLastError();
 }

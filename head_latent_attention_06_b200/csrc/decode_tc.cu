@@ -28,10 +28,12 @@
 // columns, each S buffer 32 columns (two buffers).  Lane l < 64 holds head row l
 // for the first half of every N tile, lane 64 + l the same row for the second.
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM allocator and (in
-// the even CTA) the single MMA issuer, warps 2..5 softmax / correction /
-// epilogue, one thread per TMEM lane.  The MMA order S(0), S(1), PV(0), S(2),
-// PV(1), ... lets S(t+2) run on the tensor pipe while the softmax of t+1 runs.
+// Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM allocator and (in
+// the even CTA) issuer of the score MMAs, warp 2 (even CTA) issuer of the P.V
+// MMAs, warp 3 idle, warps 4..11 softmax / correction / epilogue, two warps per
+// TMEM lane quadrant, each thread 16 scores of a row half per page.
+// Two S buffers let S(t+2) run on the tensor pipe while the softmax of t+1 runs;
+// each softmax warp signals its own P rows to the P.V issuer.
 // P is double-buffered in shared memory, so the softmax of t+1 never waits for
 // P.V of t.  The output rescale is lazy: the reference maximum moves only when
 // the tile maximum exceeds it by more than 2^8, so O in TMEM is rarely touched.
@@ -42,6 +44,8 @@
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
+#include <mutex>
+
 #include "sm100.cuh"
 
 namespace mla {
@@ -49,40 +53,56 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
 constexpr uint32_t kChunkQ = 64 * 128;              // 64 rows x 64 bf16
-constexpr uint32_t kQBytes = 9 * kChunkQ;           // 73728
+#ifndef MLA_TC_Q_TMEM_CHUNKS
+#define MLA_TC_Q_TMEM_CHUNKS 6
+#endif
+#ifndef MLA_TC_S_STAGES
+#define MLA_TC_S_STAGES 3
+#endif
+#ifndef MLA_TC_PREFETCH
+#define MLA_TC_PREFETCH 4
+#endif
+constexpr int kQTmemChunks = MLA_TC_Q_TMEM_CHUNKS;  // Q chunks 0..5 (latent 0..383) live in TMEM
+constexpr int kQSmemChunks = 9 - kQTmemChunks;      // chunks 6..8 (latent 384..511, q_pe) in smem
+constexpr uint32_t kQBytes = kQSmemChunks * kChunkQ;
 constexpr uint32_t kChunkS = 32 * 128;              // 32 tokens x 64 bf16
 constexpr uint32_t kSStage = 9 * kChunkS;           // 36864: the CTA's 32 tokens x 576
 constexpr uint32_t kChunkV = 64 * 128;              // 64 tokens x 64 bf16
 constexpr uint32_t kVStage = 4 * kChunkV;           // 32768: 64 tokens x the CTA's 4 latent chunks
-constexpr int kStages = 2;
+constexpr int kSStages = MLA_TC_S_STAGES;           // score-operand stages
+constexpr int kVStages = 2;                         // value-operand stages
 constexpr uint32_t kPBytes = 64 * 128;              // 64 rows x 64 tokens bf16
 constexpr uint32_t kQOff = 0;
 constexpr uint32_t kSOff = kQOff + kQBytes;
-constexpr uint32_t kVOff = kSOff + kStages * kSStage;
-constexpr uint32_t kPOff = kVOff + kStages * kVStage;  // two P buffers
+constexpr uint32_t kVOff = kSOff + kSStages * kSStage;
+constexpr uint32_t kPOff = kVOff + kVStages * kVStage;  // two P buffers
 constexpr uint32_t kBarOff = kPOff + 2 * kPBytes;
 // barrier indices
-constexpr int S_FULL = 0;                 // [kStages] in the even CTA: stage filled in both CTAs
-constexpr int S_EMPTY = S_FULL + kStages; // [kStages] in each CTA: stage consumed by the MMAs
-constexpr int V_FULL = S_EMPTY + kStages;
-constexpr int V_EMPTY = V_FULL + kStages;
-constexpr int Q_FULL = V_EMPTY + kStages;
-constexpr int S_READY = Q_FULL + 1;       // [2]
+constexpr int S_FULL = 0;                  // [kSStages] in the even CTA: stage filled in both CTAs
+constexpr int S_EMPTY = S_FULL + kSStages; // [kSStages] in each CTA: stage consumed by the MMAs
+constexpr int V_FULL = S_EMPTY + kSStages; // [kVStages]
+constexpr int V_EMPTY = V_FULL + kVStages;
+constexpr int Q_FULL = V_EMPTY + kVStages; // smem part of Q landed (TMA bytes)
+constexpr int Q_TMEM = Q_FULL + 1;         // TMEM part of Q written by the softmax warps
+constexpr int S_READY = Q_TMEM + 1;        // [2]
 constexpr int P_READY = S_READY + 2;      // [2] in the even CTA
 constexpr int O_DONE = P_READY + 2;       // [2]
-constexpr int DRAIN = O_DONE + 2;
-constexpr int NBARS = DRAIN + 1;
-constexpr int kPrefetchTiles = 4;                    // L2 prefetch distance of the cache stream
+constexpr int DRAIN = O_DONE + 2;        // [2] one per MMA-issuing warp
+constexpr int NBARS = DRAIN + 2;
+constexpr int kSoftmaxWarps = 8;          // warps 4..11: two per TMEM lane quadrant
+constexpr int kPrefetchTiles = MLA_TC_PREFETCH;      // L2 prefetch distance of the cache stream
 constexpr uint32_t kMiscOff = kBarOff + 8 * NBARS;
-constexpr uint32_t kXmaxOff = kMiscOff + 16;         // float [2][128]
-constexpr uint32_t kXlOff = kXmaxOff + 2 * 128 * 4;  // float [128]
-constexpr uint32_t kSmemUsed = kXlOff + 128 * 4;
+constexpr uint32_t kXmaxOff = kMiscOff + 16;         // float [2 tiles][2 column halves][128 lanes]
+constexpr uint32_t kXlOff = kXmaxOff + 4 * 128 * 4;  // float [2][128]
+constexpr uint32_t kSmemUsed = kXlOff + 2 * 128 * 4;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;    // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 256;                     // S buffers at columns 256, 288
+constexpr uint32_t kTmemQ = 320;                     // Q chunks 0..5: columns 320..511 (2 bf16 each)
+static_assert(kTmemQ + kQTmemChunks * 32 <= kTmemCols, "TMEM budget");
 constexpr uint64_t kWaitLimitNs = 2000000000ull;     // 2 s
 constexpr float kRescaleThreshold = 8.0f;            // log2 units
 
@@ -90,6 +110,7 @@ constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
 
 struct TcParams {
+  const __nv_bfloat16* q_lat;
   const uint8_t* kv;
   const int32_t* block_table;
   const int32_t* seq_lens;
@@ -102,17 +123,11 @@ struct TcParams {
   float scale_log2;
 };
 
-MLA_DEVI bool group_any(bool pred) {  // OR over the 128 softmax threads (named barrier 2)
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 2, 128, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred)
-      : "memory");
-  return r != 0;
+// 2^x with the hardware approximation (MUFU), flushing subnormal results to 0.
+MLA_DEVI float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -152,19 +167,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     if (bad_len && r == 0 && g == 0 && split == 0) set_status(p.status, MLA_ERR_BAD_SEQ_LEN);
     *abort_flag = 0;
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kSStages; ++i) {
       mbar_init(own_bar(S_FULL + i), 1);
       mbar_init(own_bar(S_EMPTY + i), 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
       mbar_init(own_bar(V_FULL + i), 1);
       mbar_init(own_bar(V_EMPTY + i), 1);
     }
+    mbar_init(own_bar(Q_TMEM), 2 * kSoftmaxWarps);
     mbar_init(own_bar(Q_FULL), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(own_bar(S_READY + i), 1);
-      mbar_init(own_bar(P_READY + i), 2);
+      mbar_init(own_bar(P_READY + i), 2 * kSoftmaxWarps);
       mbar_init(own_bar(O_DONE + i), 1);
     }
     mbar_init(own_bar(DRAIN), 1);
+    mbar_init(own_bar(DRAIN + 1), 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -176,6 +195,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_wait();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_trigger();
 
   if (warp == 0) {
     // =========================== TMA producer ===========================
@@ -188,11 +208,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_qpe);
         prefetch_tmap(&tm_ks);
         prefetch_tmap(&tm_kv);
-        const int qrow = (b * p.s_q + g) * p.H + 64 * (int)r;
-        const uint32_t qb = lead_bar(Q_FULL);
-        if (r == 0) mbar_arrive_expect_tx_local(own_bar(Q_FULL), 2 * kQBytes);
-        for (int c = 0; c < 8; ++c) tma_load_2d_pair(sa + kQOff + c * kChunkQ, &tm_q, qb, 64 * c, qrow);
-        tma_load_2d_pair(sa + kQOff + 8 * kChunkQ, &tm_qpe, qb, 0, qrow);
       }
       // physical pages, fetched 32 at a time by the whole warp
       int blk_s = -1, pg_s = 0, blk_v = -1, pg_v = 0, blk_p = -1, pg_p = 0;
@@ -216,8 +231,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       };
       for (int u = 0; u < n && u < kPrefetchTiles; ++u) prefetch(u);
       auto load_s = [&](int u) -> bool {
-        const int st = u % kStages;
-        const uint32_t ph = ((u / kStages) & 1) ^ 1;
+        const int st = u % kSStages;
+        const uint32_t ph = ((u / kSStages) & 1) ^ 1;
         if (!mbar_wait_converged(own_bar(S_EMPTY + st), ph, abort_flag, p.status, kWaitLimitNs)) return false;
         const int pg = page_of(u, blk_s, pg_s);
         const uint32_t fb = lead_bar(S_FULL + st);
@@ -229,8 +244,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         return true;
       };
       auto load_v = [&](int u) -> bool {
-        const int st = u % kStages;
-        const uint32_t ph = ((u / kStages) & 1) ^ 1;
+        const int st = u % kVStages;
+        const uint32_t ph = ((u / kVStages) & 1) ^ 1;
         if (!mbar_wait_converged(own_bar(V_EMPTY + st), ph, abort_flag, p.status, kWaitLimitNs)) return false;
         const int pg = page_of(u, blk_v, pg_v);
         const uint32_t fb = lead_bar(V_FULL + st);
@@ -242,183 +257,243 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         return true;
       };
+      // The cache, block table and lengths are not written by the kernel this one
+      // may overlap with (the query absorption); q_lat is, so Q waits for it.
       bool ok = load_s(0);
+      pdl_wait();
+      if (lane == 0) {
+        const int qrow = (b * p.s_q + g) * p.H + 64 * (int)r;
+        const uint32_t qb = lead_bar(Q_FULL);
+        if (r == 0) mbar_arrive_expect_tx_local(own_bar(Q_FULL), 2 * kQBytes);
+        for (int c = kQTmemChunks; c < 8; ++c)
+          tma_load_2d_pair(sa + kQOff + (c - kQTmemChunks) * kChunkQ, &tm_q, qb, 64 * c, qrow);
+        tma_load_2d_pair(sa + kQOff + (8 - kQTmemChunks) * kChunkQ, &tm_qpe, qb, 0, qrow);
+      }
+      __syncwarp();
       for (int u = 0; ok && u < n; ++u) {
         if (u + 1 < n) ok = load_s(u + 1);
         if (ok) ok = load_v(u);
       }
     }
-  } else if (warp == 1) {
-    // =========================== MMA issuer (even CTA) ===========================
+  } else if (warp == 1 || warp == 2) {
+    // ============ MMA issuers (even CTA): warp 1 scores, warp 2 P.V ============
+    // The two streams touch disjoint TMEM (S buffers / O) and shared memory
+    // (Q and the S ring / P and the V ring), so they are issued independently.
     if (r == 0 && n > 0) {
-      bool ok = mbar_wait_converged(own_bar(Q_FULL), 0, abort_flag, p.status, kWaitLimitNs);
       const uint64_t dq = desc_sw128(sa + kQOff, 16, 1024);
       const uint64_t ds = desc_sw128(sa + kSOff, 16, 1024);
       const uint64_t dv = desc_sw128(sa + kVOff, kChunkV, 1024);
       const uint64_t dp = desc_sw128(sa + kPOff, 16, 1024);
-      auto issue_s = [&](int u) -> bool {
-        const int st = u % kStages, sb = u & 1;
-        if (!mbar_wait_converged(own_bar(S_FULL + st), (u / kStages) & 1, abort_flag, p.status, kWaitLimitNs))
-          return false;
-        tc_fence_after();
-        const uint32_t d = tmem + kTmemS + 32u * sb;
-        const uint64_t bs0 = ds + ((st * kSStage) >> 4);
+      bool ok = true;
+      if (warp == 1) {
+        ok = mbar_wait_converged(own_bar(Q_FULL), 0, abort_flag, p.status, kWaitLimitNs) &&
+             mbar_wait_converged(own_bar(Q_TMEM), 0, abort_flag, p.status, kWaitLimitNs);
+        for (int u = 0; ok && u < n; ++u) {
+          const int st = u % kSStages, sb = u & 1;
+          // S buffer sb was last read by the softmax of tile u-2
+          if (u >= 2 && !mbar_wait_converged(own_bar(P_READY + sb), ((u - 2) >> 1) & 1, abort_flag, p.status,
+                                             kWaitLimitNs))
+            break;
+          if (!mbar_wait_converged(own_bar(S_FULL + st), (u / kSStages) & 1, abort_flag, p.status, kWaitLimitNs))
+            break;
+          tc_fence_after();
+          const uint32_t d = tmem + kTmemS + 32u * sb;
+          const uint64_t bs0 = ds + ((st * kSStage) >> 4);
+          // K chunks 0..5: A (Q) from TMEM, only B is read from shared memory
 #pragma unroll
-        for (int c = 0; c < 9; ++c) {
-          const uint64_t aq = dq + ((c * kChunkQ) >> 4), bs = bs0 + ((c * kChunkS) >> 4);
-          mma_pair_elect(d, aq, bs, kIdescS, c != 0);
-          mma_pair_elect(d, aq + 2, bs + 2, kIdescS, 1);
-          mma_pair_elect(d, aq + 4, bs + 4, kIdescS, 1);
-          mma_pair_elect(d, aq + 6, bs + 6, kIdescS, 1);
+          for (int c = 0; c < kQTmemChunks; ++c) {
+            const uint32_t aq = tmem + kTmemQ + 32u * c;
+            const uint64_t bs = bs0 + ((c * kChunkS) >> 4);
+            mma_pair_ts_elect(d, aq, bs, kIdescS, c != 0);
+            mma_pair_ts_elect(d, aq + 8, bs + 2, kIdescS, 1);
+            mma_pair_ts_elect(d, aq + 16, bs + 4, kIdescS, 1);
+            mma_pair_ts_elect(d, aq + 24, bs + 6, kIdescS, 1);
+          }
+#pragma unroll
+          for (int c = kQTmemChunks; c < 9; ++c) {
+            const uint64_t aq = dq + (((c - kQTmemChunks) * kChunkQ) >> 4), bs = bs0 + ((c * kChunkS) >> 4);
+            mma_pair_elect(d, aq, bs, kIdescS, c != 0);
+            mma_pair_elect(d, aq + 2, bs + 2, kIdescS, 1);
+            mma_pair_elect(d, aq + 4, bs + 4, kIdescS, 1);
+            mma_pair_elect(d, aq + 6, bs + 6, kIdescS, 1);
+          }
+          commit_pair_mc_elect(own_bar(S_EMPTY + st), 0x3);
+          commit_pair_mc_elect(own_bar(S_READY + sb), 0x3);
         }
-        commit_pair_mc_elect(own_bar(S_EMPTY + st), 0x3);
-        commit_pair_mc_elect(own_bar(S_READY + sb), 0x3);
-        return true;
-      };
-      auto issue_pv = [&](int t) -> bool {
-        const int pb = t & 1, st = t % kStages;
-        if (!mbar_wait_converged(own_bar(P_READY + pb), (t >> 1) & 1, abort_flag, p.status, kWaitLimitNs))
-          return false;
-        if (!mbar_wait_converged(own_bar(V_FULL + st), (t / kStages) & 1, abort_flag, p.status, kWaitLimitNs))
-          return false;
-        tc_fence_after();
-        const uint64_t ap = dp + ((pb * kPBytes) >> 4);
-        const uint64_t bv = dv + ((st * kVStage) >> 4);
+      } else {
+        for (int t = 0; t < n; ++t) {
+          const int pb = t & 1, st = t % kVStages;
+          if (!mbar_wait_converged(own_bar(P_READY + pb), (t >> 1) & 1, abort_flag, p.status, kWaitLimitNs))
+            break;
+          if (!mbar_wait_converged(own_bar(V_FULL + st), (t / kVStages) & 1, abort_flag, p.status, kWaitLimitNs))
+            break;
+          tc_fence_after();
+          const uint64_t ap = dp + ((pb * kPBytes) >> 4);
+          const uint64_t bv = dv + ((st * kVStage) >> 4);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+          for (int h = 0; h < 2; ++h) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_pair_elect(tmem + 128u * h, ap + kk * 2, bv + ((2 * h * kChunkV + kk * 2048) >> 4), kIdescPV,
-                           (t > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_pair_elect(tmem + 128u * h, ap + kk * 2, bv + ((2 * h * kChunkV + kk * 2048) >> 4), kIdescPV,
+                             (t > 0 || kk > 0) ? 1u : 0u);
+          }
+          commit_pair_mc_elect(own_bar(V_EMPTY + st), 0x3);
+          commit_pair_mc_elect(own_bar(O_DONE + pb), 0x3);
         }
-        commit_pair_mc_elect(own_bar(V_EMPTY + st), 0x3);
-        commit_pair_mc_elect(own_bar(O_DONE + pb), 0x3);
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      if (ok && n > 1) ok = issue_s(1);
-      for (int t = 0; ok && t < n; ++t) {
-        ok = issue_pv(t);
-        if (ok && t + 2 < n) ok = issue_s(t + 2);
       }
-      // every issued MMA has completed before TMEM is released
-      commit_pair_mc_elect(own_bar(DRAIN), 0x1);
+      // every MMA this warp issued has completed before TMEM is released
+      const int db = DRAIN + (warp == 2 ? 1 : 0);
+      commit_pair_mc_elect(own_bar(db), 0x1);
       int dummy = 0;
-      mbar_wait_converged(own_bar(DRAIN), 0, &dummy, p.status, kWaitLimitNs);
+      mbar_wait_converged(own_bar(db), 0, &dummy, p.status, kWaitLimitNs);
     }
-  } else {
+  } else if (warp >= 4) {
     // ====================== softmax / correction / epilogue ======================
+    // Thread = (TMEM lane lt, column half ch).  Lane lt holds head row m = lt % 64
+    // for tokens 32*half .. 32*half+31 of the page (half = lt / 64); the two warps
+    // of a lane quadrant take 16 of those scores each, and half of the row's O
+    // columns each.  A row's four threads (lt, lt ^ 64, both ch) agree on the
+    // reference maximum through shared memory.
     const int wq = warp & 3;                 // TMEM lane quadrant of this warp
-    const int lt = wq * 32 + lane;           // TMEM lane = thread's row slot
-    const int m = lt & 63, half = lt >> 6;   // head row in this CTA, token / column half
+    const int ch = (warp - 4) >> 2;          // column half
+    const int lt = wq * 32 + lane;
+    const int m = lt & 63, half = lt >> 6;
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
+    const uint32_t grp_bar = 3 + (wq & 1);   // the 4 warps of quadrants {q, q^2}
+    // Q row m, latent columns 0 .. 64*kQTmemChunks-1, into this lane's TMEM columns
+    // (A operand of the score MMA: each 32-bit column holds two consecutive bf16;
+    // lanes l and 64 + l both hold row l, the duplicated layout of the paired MMA)
+    pdl_wait();
+    if (n > 0) {
+      const uint4* qsrc =
+          reinterpret_cast<const uint4*>(p.q_lat + (((size_t)b * p.s_q + g) * p.H + 64 * r + m) * kDc);
+      constexpr int kPerWarp = (kQTmemChunks + 1) / 2;
+#pragma unroll 1
+      for (int c = ch * kPerWarp; c < kQTmemChunks && c < (ch + 1) * kPerWarp; ++c) {
+        uint32_t qv[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint4 v = __ldg(qsrc + c * 8 + k);
+          qv[4 * k] = v.x;
+          qv[4 * k + 1] = v.y;
+          qv[4 * k + 2] = v.z;
+          qv[4 * k + 3] = v.w;
+        }
+        tmem_st32(tl + kTmemQ + 32u * c, qv);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(lead_bar(Q_TMEM));
+    }
     float m_used = -CUDART_INF_F, l = 0.f;
-    bool alive = true;
     const int lim = min(vis, j_end);
+    // Control flow stays uniform even if a wait gives up (the kernel is then
+    // aborting and every later wait returns at once): no barrier is skipped.
     for (int t = 0; t < n; ++t) {
       const int sb = t & 1;
-      bool w = mbar_wait(own_bar(S_READY + sb), (t >> 1) & 1, abort_flag, p.status, kWaitLimitNs);
-      if (group_any(!w)) { alive = false; break; }
+      mbar_wait(own_bar(S_READY + sb), (t >> 1) & 1, abort_flag, p.status, kWaitLimitNs);
       tc_fence_after();
-      uint32_t sv[32];
-      tmem_ld32(tl + kTmemS + 32u * sb, sv);
+      uint32_t sv[16];
+      tmem_ld16(tl + kTmemS + 32u * sb + 16u * ch, sv);
       tmem_wait_ld();
-      const int j0 = (t0 + t) * kPage + 32 * half;
-      const int nv = max(0, min(32, lim - j0));
-      float s[32];
-      float lmax = -CUDART_INF_F;
+      const int j0 = (t0 + t) * kPage + 32 * half + 16 * ch;
+      const int nv = max(0, min(16, lim - j0));
+      float s[16];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        s[j] = j < nv ? __uint_as_float(sv[j]) * p.scale_log2 : -CUDART_INF_F;
-        lmax = fmaxf(lmax, s[j]);
-      }
-      xmax[sb * 128 + lt] = lmax;
-      named_bar_sync(1, 128);
-      const float tmax = fmaxf(lmax, xmax[sb * 128 + (lt ^ 64)]);
+      for (int j = 0; j < 16; ++j) s[j] = j < nv ? __uint_as_float(sv[j]) : -CUDART_INF_F;
+      float mx[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mx[k] = fmaxf(fmaxf(s[k], s[k + 4]), fmaxf(s[k + 8], s[k + 12]));
+      // the softmax scale is positive: scaling commutes with the maximum
+      const float lmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
+      float* xm = xmax + sb * 256;
+      xm[ch * 128 + lt] = lmax;
+      named_bar_sync(grp_bar, 128);
+      const float tmax = fmaxf(fmaxf(xm[lt], xm[lt ^ 64]), fmaxf(xm[128 + lt], xm[128 + (lt ^ 64)]));
       float alpha = 1.f;
       bool resc = false;
       if (tmax > -CUDART_INF_F) {
         if (m_used == -CUDART_INF_F) {
           m_used = tmax;                       // nothing accumulated yet: O and l are zero
         } else if (tmax > m_used + kRescaleThreshold) {
-          alpha = exp2f(m_used - tmax);
+          alpha = ex2_approx(m_used - tmax);
           m_used = tmax;
           resc = true;
           l *= alpha;
         }
       }
-      // reference point of the exponentials; a row with nothing visible yet keeps
-      // 0 so that no (-inf) - (-inf) appears
-      const float ref = m_used == -CUDART_INF_F ? 0.f : m_used;
-      uint32_t pk[16];
+      // p = 2^(s * scale_log2 - ref); a row with nothing visible yet keeps ref = 0
+      // so that no (-inf) - (-inf) appears
+      const float nref = m_used == -CUDART_INF_F ? 0.f : -m_used;
+      uint32_t pk[8];
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float p0 = exp2f(s[j] - ref), p1 = exp2f(s[j + 1] - ref);
-        l += p0 + p1;
+      for (int j = 0; j < 16; j += 2) {
+        const float p0 = ex2_approx(fmaf(s[j], p.scale_log2, nref));
+        const float p1 = ex2_approx(fmaf(s[j + 1], p.scale_log2, nref));
+        ls[(j >> 1) & 3] += p0 + p1;
         pk[j >> 1] = pack_bf16(p0, p1);
       }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       // P buffer sb was last read by PV(t-2)
-      if (t >= 2) {
-        w = mbar_wait(own_bar(O_DONE + sb), ((t - 2) >> 1) & 1, abort_flag, p.status, kWaitLimitNs);
-        if (group_any(!w)) { alive = false; break; }
-      }
-      // O may only be rescaled once PV(t-1) has finished accumulating into it
-      const bool any_resc = group_any(resc);
-      if (any_resc && t >= 1) {
-        w = mbar_wait(own_bar(O_DONE + (sb ^ 1)), ((t - 1) >> 1) & 1, abort_flag, p.status, kWaitLimitNs);
-        if (group_any(!w)) { alive = false; break; }
-        tc_fence_after();
-      }
-      if (any_resc) {
+      if (t >= 2) mbar_wait(own_bar(O_DONE + sb), ((t - 2) >> 1) & 1, abort_flag, p.status, kWaitLimitNs);
+      // this warp's O columns may only be rescaled once PV(t-1) has accumulated into them
+      if (__any_sync(0xffffffffu, resc)) {
+        if (t >= 1) {
+          mbar_wait(own_bar(O_DONE + (sb ^ 1)), ((t - 1) >> 1) & 1, abort_flag, p.status, kWaitLimitNs);
+          tc_fence_after();
+        }
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t ov[32];
-          tmem_ld32(tl + 32u * c, ov);
+          const uint32_t col = 128u * ch + 32u * c;
+          tmem_ld32(tl + col, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
-          tmem_st32(tl + 32u * c, ov);
+          tmem_st32(tl + col, ov);
         }
         tmem_wait_st();
       }
-      // P row m, tokens 32*half .. +31: four 16-byte chunks of the 128-byte row
+      // P row m, tokens 32*half + 16*ch .. +15: two 16-byte chunks of the 128-byte row
       uint8_t* prow = sm + kPOff + sb * kPBytes + m * 128;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int q = 4 * half + k;
+      for (int k = 0; k < 2; ++k) {
+        const int q = 4 * half + 2 * ch + k;
         *reinterpret_cast<uint4*>(prow + ((q ^ (m & 7)) << 4)) =
             make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      named_bar_sync(1, 128);
-      if (lt == 0) mbar_arrive_remote(lead_bar(P_READY + sb));
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(lead_bar(P_READY + sb));
     }
-    if (alive && n > 0) {
-      bool w = mbar_wait(own_bar(O_DONE + ((n - 1) & 1)), ((n - 1) >> 1) & 1, abort_flag, p.status,
-                         kWaitLimitNs);
-      if (group_any(!w)) alive = false;
+    if (n > 0) {
+      mbar_wait(own_bar(O_DONE + ((n - 1) & 1)), ((n - 1) >> 1) & 1, abort_flag, p.status, kWaitLimitNs);
       tc_fence_after();
     }
-    xl[lt] = l;
-    named_bar_sync(1, 128);
-    const float ltot = l + xl[lt ^ 64];
+    xl[ch * 128 + lt] = l;
+    named_bar_sync(1, 256);
+    const bool alive = *abort_flag == 0;
+    const float ltot = (xl[lt] + xl[lt ^ 64]) + (xl[128 + lt] + xl[128 + (lt ^ 64)]);
     const bool empty = !(ltot > 0.f) || !alive;
     const float inv = empty ? 0.f : 1.f / ltot;
     const float lse = empty ? -CUDART_INF_F : (m_used + log2f(ltot)) * 0.6931471805599453f;
     const size_t orow = ((size_t)b * p.s_q + g) * p.H + 64 * r + m;
     const bool read_o = alive && n > 0;
+    // TMEM columns 128*ch .. +127 of this lane: latent half*128 + 256*ch + 0..127
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < 4; ++c) {
       uint32_t ov[32];
       if (read_o) {
-        tmem_ld32(tl + 32u * c, ov);
+        tmem_ld32(tl + 128u * ch + 32u * c, ov);
         tmem_wait_ld();
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) ov[j] = 0u;
       }
-      const int col = (c < 4) ? half * 128 + 32 * c : 256 + half * 128 + 32 * (c - 4);
+      const int col = 256 * ch + half * 128 + 32 * c;
       if (p.splits == 1) {
         uint4* dst = reinterpret_cast<uint4*>(p.o_lat + orow * kDc + col);
 #pragma unroll
@@ -438,7 +513,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                __uint_as_float(ov[4 * k + 2]) * inv, __uint_as_float(ov[4 * k + 3]) * inv);
       }
     }
-    if (half == 0) {
+    if (half == 0 && ch == 0) {
       if (p.splits == 1) {
         if (p.lse) p.lse[orow] = lse;
       } else {
@@ -488,6 +563,40 @@ bool encode_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, ui
   return res == CUDA_SUCCESS;
 }
 
+
+// Encoded tensor maps, keyed by their parameters: a decode step re-encodes
+// nothing when its buffers and shapes repeat.
+struct MapKey {
+  const void* ptr;
+  uint64_t cols, rows, row_bytes;
+  uint32_t box_cols, box_rows;
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && cols == o.cols && rows == o.rows && row_bytes == o.row_bytes &&
+           box_cols == o.box_cols && box_rows == o.box_rows;
+  }
+};
+constexpr int kMapCache = 32;
+std::mutex g_map_mu;
+MapKey g_map_keys[kMapCache];
+CUtensorMap g_maps[kMapCache];
+int g_map_count = 0, g_map_next = 0;
+
+bool cached_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t row_bytes,
+                uint32_t box_cols, uint32_t box_rows) {
+  const MapKey k{ptr, cols, rows, row_bytes, box_cols, box_rows};
+  std::lock_guard<std::mutex> lock(g_map_mu);
+  for (int i = 0; i < g_map_count; ++i)
+    if (g_map_keys[i] == k) {
+      *m = g_maps[i];
+      return true;
+    }
+  if (!encode_2d(m, ptr, cols, rows, row_bytes, box_cols, box_rows)) return false;
+  const int slot = g_map_count < kMapCache ? g_map_count++ : (g_map_next++ % kMapCache);
+  g_map_keys[slot] = k;
+  g_maps[slot] = *m;
+  return true;
+}
+
 }  // namespace
 
 bool decode_tc_supported(const mla_decode_args_t* a) {
@@ -500,12 +609,13 @@ cudaError_t launch_decode_tc(const mla_decode_args_t* a, int splits, cudaStream_
   CUtensorMap tm_q, tm_qpe, tm_ks, tm_kv;
   const uint64_t rows_q = (uint64_t)a->B * a->s_q * a->H;
   const uint64_t rows_kv = (uint64_t)a->num_pages * kPage;
-  if (!encode_2d(&tm_q, a->q_lat, kDc, rows_q, kDc * 2, 64, 64) ||
-      !encode_2d(&tm_qpe, a->q_pe, kDr, rows_q, kDr * 2, 64, 64) ||
-      !encode_2d(&tm_ks, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 32) ||
-      !encode_2d(&tm_kv, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 64))
+  if (!cached_map(&tm_q, a->q_lat, kDc, rows_q, kDc * 2, 64, 64) ||
+      !cached_map(&tm_qpe, a->q_pe, kDr, rows_q, kDr * 2, 64, 64) ||
+      !cached_map(&tm_ks, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 32) ||
+      !cached_map(&tm_kv, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 64))
     return cudaErrorInvalidValue;
   TcParams p;
+  p.q_lat = static_cast<const __nv_bfloat16*>(a->q_lat);
   p.kv = static_cast<const uint8_t*>(a->kv_cache);
   p.block_table = a->block_table;
   p.seq_lens = a->seq_lens;
@@ -525,12 +635,17 @@ cudaError_t launch_decode_tc(const mla_decode_args_t* a, int splits, cudaStream_
   p.causal = a->causal;
   p.splits = splits;
   p.scale_log2 = a->softmax_scale * kLog2e;
-  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
-  if (e != cudaSuccess) return e;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
   dim3 grid(2 * splits, a->s_q, a->B);
-  decode_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_qpe, tm_ks, tm_kv, p);
-  return cudaGetLastError();
+  return launch_pdl(decode_tc_kernel, grid, dim3(kThreads), kSmemBytes, stream, tm_q, tm_qpe, tm_ks, tm_kv, p);
 }
 
 }  // namespace mla

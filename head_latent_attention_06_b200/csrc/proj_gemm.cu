@@ -36,6 +36,14 @@ __global__ void __launch_bounds__(128) proj_kernel(const __nv_bfloat16* __restri
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wm = warp >> 1, wn = warp & 1;  // warp tile: 32 tokens x 64 columns
   const __nv_bfloat16* Wh = W + (size_t)h * K * N;
+  pdl_trigger();
+  // The weight is never written by the kernel this one may overlap with: its rows
+  // for this CTA go to L2 before waiting for the activations.
+  if (tid < (W_KN ? K : TN)) {
+    const __nv_bfloat16* row = W_KN ? Wh + (size_t)tid * N + n0 : Wh + (size_t)(n0 + tid) * K;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(row) : "memory");
+  }
+  pdl_wait();
 
   auto load_chunk = [&](int kc, int buf) {
     const int k0 = kc * TK;
@@ -134,13 +142,17 @@ cudaError_t launch_proj(const void* X, const void* W, void* Y, int n_tok, int H,
   constexpr int WCH = W_KN ? TK * WKN : TN * WNK;
   const size_t smem = 2 * (TM * XS + WCH) * sizeof(__nv_bfloat16);
   auto kern = proj_kernel<K, N, W_KN>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
   dim3 grid(N / TN, (n_tok + TM - 1) / TM, H);
-  kern<<<grid, 128, smem, stream>>>(static_cast<const __nv_bfloat16*>(X),
-                                    static_cast<const __nv_bfloat16*>(W),
-                                    static_cast<__nv_bfloat16*>(Y), n_tok, H);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(128), smem, stream, static_cast<const __nv_bfloat16*>(X),
+                    static_cast<const __nv_bfloat16*>(W), static_cast<__nv_bfloat16*>(Y), n_tok, H);
 }
 
 }  // namespace
