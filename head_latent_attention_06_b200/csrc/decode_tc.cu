@@ -44,9 +44,8 @@
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
-#include <mutex>
-
 #include "sm100.cuh"
+#include "tma_host.cuh"
 
 namespace mla {
 namespace {
@@ -537,66 +536,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult q;
-    void* ptr = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-bool encode_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t row_bytes,
-               uint32_t box_cols, uint32_t box_rows) {
-  auto enc = get_encode();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult res = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return res == CUDA_SUCCESS;
-}
-
-
-// Encoded tensor maps, keyed by their parameters: a decode step re-encodes
-// nothing when its buffers and shapes repeat.
-struct MapKey {
-  const void* ptr;
-  uint64_t cols, rows, row_bytes;
-  uint32_t box_cols, box_rows;
-  bool operator==(const MapKey& o) const {
-    return ptr == o.ptr && cols == o.cols && rows == o.rows && row_bytes == o.row_bytes &&
-           box_cols == o.box_cols && box_rows == o.box_rows;
-  }
-};
-constexpr int kMapCache = 32;
-std::mutex g_map_mu;
-MapKey g_map_keys[kMapCache];
-CUtensorMap g_maps[kMapCache];
-int g_map_count = 0, g_map_next = 0;
-
-bool cached_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t row_bytes,
-                uint32_t box_cols, uint32_t box_rows) {
-  const MapKey k{ptr, cols, rows, row_bytes, box_cols, box_rows};
-  std::lock_guard<std::mutex> lock(g_map_mu);
-  for (int i = 0; i < g_map_count; ++i)
-    if (g_map_keys[i] == k) {
-      *m = g_maps[i];
-      return true;
-    }
-  if (!encode_2d(m, ptr, cols, rows, row_bytes, box_cols, box_rows)) return false;
-  const int slot = g_map_count < kMapCache ? g_map_count++ : (g_map_next++ % kMapCache);
-  g_map_keys[slot] = k;
-  g_maps[slot] = *m;
-  return true;
-}
-
 }  // namespace
 
 bool decode_tc_supported(const mla_decode_args_t* a) {
@@ -609,10 +548,10 @@ cudaError_t launch_decode_tc(const mla_decode_args_t* a, int splits, cudaStream_
   CUtensorMap tm_q, tm_qpe, tm_ks, tm_kv;
   const uint64_t rows_q = (uint64_t)a->B * a->s_q * a->H;
   const uint64_t rows_kv = (uint64_t)a->num_pages * kPage;
-  if (!cached_map(&tm_q, a->q_lat, kDc, rows_q, kDc * 2, 64, 64) ||
-      !cached_map(&tm_qpe, a->q_pe, kDr, rows_q, kDr * 2, 64, 64) ||
-      !cached_map(&tm_ks, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 32) ||
-      !cached_map(&tm_kv, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 64))
+  if (!tma_map_2d(&tm_q, a->q_lat, kDc, rows_q, kDc * 2, 64, 64) ||
+      !tma_map_2d(&tm_qpe, a->q_pe, kDr, rows_q, kDr * 2, 64, 64) ||
+      !tma_map_2d(&tm_ks, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 32) ||
+      !tma_map_2d(&tm_kv, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 64))
     return cudaErrorInvalidValue;
   TcParams p;
   p.q_lat = static_cast<const __nv_bfloat16*>(a->q_lat);
@@ -641,6 +580,8 @@ cudaError_t launch_decode_tc(const mla_decode_args_t* a, int splits, cudaStream_
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }

@@ -4,167 +4,213 @@
 // (weight absorption, nnets.ru article section "Суть MLA"; the up-projections
 // k = W_UK c, v = W_UV c of "MLA ... Explained", section "Architecture").
 //
-// Both are a batch of H small GEMMs out[t][n] = sum_k X[t][k] W(k, n) whose
-// weight (16.8 MB at H = 128) is read once per 64-token block; they are
-// HBM-bound on the weight.  One CTA computes a 64-token x 128-column tile of one
-// head, streaming K in 64-wide chunks through a cp.async double buffer, with
-// warp-level bf16 MMAs (fp32 accumulation).
-#include "common.cuh"
+// Both are a batch of H small GEMMs out[t][n] = sum_k X[t][k] W(k, n).  At decode
+// sizes (tens to hundreds of tokens) they are bound by reading the weight
+// (128 KB per head, 16.8 MB at H = 128).  One CTA owns one head and one block of
+// 64 tokens: TMA streams that head's whole weight and the block's activations,
+// K chunk by K chunk, into 128-byte-swizzled shared memory (bulk TMA requests keep
+// far more bytes in flight per SM than per-thread copies), and warp-level bf16
+// MMAs (fp32 accumulation) compute every output column.
+#include "sm100.cuh"
+#include "tma_host.cuh"
 
 namespace mla {
 namespace {
 
-constexpr int TM = 64, TN = 128, TK = 64;
-constexpr int XS = TK + 8;   // padded smem row (elements) of the X chunk
-constexpr int WKN = TN + 8;  // padded row of a [k][n] weight chunk
-constexpr int WNK = TK + 8;  // padded row of a [n][k] weight chunk
+using namespace sm100;
+
+constexpr int TM = 64;   // tokens per CTA
+constexpr int TK = 64;   // K per chunk: one 128-byte swizzled row per matrix row
+constexpr uint64_t kProjWaitNs = 2000000000ull;
+
+MLA_DEVI void tma_load_2d(uint32_t dst, const void* tmap, uint32_t mbar, int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(tmap), "r"(mbar), "r"(x), "r"(y)
+      : "memory");
+}
+MLA_DEVI void tma_load_3d(uint32_t dst, const void* tmap, uint32_t mbar, int32_t x, int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(tmap), "r"(mbar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// Address of the 16-byte unit holding columns c0 .. c0+7 of row r in a block of
+// 128-byte rows written by TMA with the 128-byte swizzle (block 1024-aligned).
+MLA_DEVI uint32_t sw128(uint32_t base, int r, int c0) {
+  return base + r * 128 + ((((c0 >> 3) ^ (r & 7)) & 7) << 4);
+}
 
 // W_KN: weight stored [K][N] per head (W_UK for absorption); otherwise [N][K]
-// (W_UV for the up-projection).
-template <int K, int N, bool W_KN>
-__global__ void __launch_bounds__(128) proj_kernel(const __nv_bfloat16* __restrict__ X,
-                                                   const __nv_bfloat16* __restrict__ W,
-                                                   __nv_bfloat16* __restrict__ Y, int n_tok,
-                                                   int H) {
-  constexpr int XCH = TM * XS;
-  constexpr int WCH = W_KN ? TK * WKN : TN * WNK;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // [2][TM][XS]
-  __nv_bfloat16* ws = xs + 2 * XCH;                                  // [2][WCH]
+// (W_UV for the up-projection).  Each warp owns N / NWARPS output columns of
+// all 64 tokens.
+template <int K, int N, bool W_KN, int NWARPS, int STAGES>
+struct ProjCfg {
+  static constexpr int NT = NWARPS * 32;
+  static constexpr int WN = N / NWARPS;                  // columns per warp
+  static constexpr uint32_t XBYTES = TM * 128;           // X chunk: 64 rows x 64 bf16
+  static constexpr uint32_t WBYTES = (uint32_t)N * 128;  // weight chunk: N x 64 (either layout)
+  static constexpr uint32_t STAGE = XBYTES + WBYTES;
+  static constexpr int NK = K / TK;
+  static constexpr size_t smem = (size_t)STAGES * STAGE + 1024 + 64;  // + alignment, barriers
+};
 
-  const int n0 = blockIdx.x * TN, t0 = blockIdx.y * TM, h = blockIdx.z;
+template <int K, int N, bool W_KN, int NWARPS, int STAGES>
+__global__ void __launch_bounds__(NWARPS * 32) proj_kernel(const __grid_constant__ CUtensorMap tm_x,
+                                                           const __grid_constant__ CUtensorMap tm_w,
+                                                           __nv_bfloat16* __restrict__ Y, int n_tok,
+                                                           int H) {
+  using C = ProjCfg<K, N, W_KN, NWARPS, STAGES>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sa = (raw + 1023u) & ~1023u;
+  const uint32_t bar0 = sa + STAGES * C::STAGE;
+
+  const int t0 = blockIdx.x * TM, h = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int wm = warp >> 1, wn = warp & 1;  // warp tile: 32 tokens x 64 columns
-  const __nv_bfloat16* Wh = W + (size_t)h * K * N;
   pdl_trigger();
-  // The weight is never written by the kernel this one may overlap with: its rows
-  // for this CTA go to L2 before waiting for the activations.
-  if (tid < (W_KN ? K : TN)) {
-    const __nv_bfloat16* row = W_KN ? Wh + (size_t)tid * N + n0 : Wh + (size_t)(n0 + tid) * K;
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(row) : "memory");
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) mbar_init(bar0 + 8 * s, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  // the weight is never written by the kernel this one may overlap with, the
+  // activations are: weight chunks are requested before waiting for it
+  auto load_w = [&](int kc, int s) {
+    const uint32_t dst = sa + s * C::STAGE + C::XBYTES, mb = bar0 + 8 * s;
+    if (W_KN) {
+      for (int g = 0; g < N / 64; ++g) tma_load_2d(dst + g * (TK * 128), &tm_w, mb, 64 * g, h * K + kc * TK);
+    } else {
+      tma_load_2d(dst, &tm_w, mb, kc * TK, h * N);
+    }
+  };
+  auto load_x = [&](int kc, int s) { tma_load_3d(sa + s * C::STAGE, &tm_x, bar0 + 8 * s, kc * TK, h, t0); };
+  if (tid == 0) {
+    for (int s = 0; s < STAGES && s < C::NK; ++s) {
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar0 + 8 * s),
+                   "r"(C::STAGE)
+                   : "memory");
+      load_w(s, s);
+    }
   }
   pdl_wait();
+  if (tid == 0)
+    for (int s = 0; s < STAGES && s < C::NK; ++s) load_x(s, s);
 
-  auto load_chunk = [&](int kc, int buf) {
-    const int k0 = kc * TK;
-    __nv_bfloat16* xb = xs + buf * XCH;
-    for (int v = tid; v < TM * (TK / 8); v += 128) {
-      int r = v / (TK / 8), c = (v % (TK / 8)) * 8;
-      int t = t0 + r;
-      if (t < n_tok) {
-        cp_async16(xb + r * XS + c, X + ((size_t)t * H + h) * K + k0 + c);
-      } else {
-        *reinterpret_cast<uint4*>(xb + r * XS + c) = make_uint4(0, 0, 0, 0);
-      }
-    }
-    __nv_bfloat16* wb = ws + buf * WCH;
-    if (W_KN) {
-      for (int v = tid; v < TK * (TN / 8); v += 128) {
-        int r = v / (TN / 8), c = (v % (TN / 8)) * 8;
-        cp_async16(wb + r * WKN + c, Wh + (size_t)(k0 + r) * N + n0 + c);
-      }
-    } else {
-      for (int v = tid; v < TN * (TK / 8); v += 128) {
-        int r = v / (TK / 8), c = (v % (TK / 8)) * 8;
-        cp_async16(wb + r * WNK + c, Wh + (size_t)(n0 + r) * K + k0 + c);
-      }
-    }
-    cp_async_commit();
-  };
-
-  float acc[2][8][4];
+  constexpr int NJ = C::WN / 8;  // n-tiles of 8 per warp
+  float acc[4][NJ][4];
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < NJ; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
 
-  constexpr int NK = K / TK;
-  load_chunk(0, 0);
-  for (int kc = 0; kc < NK; ++kc) {
-    if (kc + 1 < NK) {
-      load_chunk(kc + 1, (kc + 1) & 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const __nv_bfloat16* xb = xs + (kc & 1) * XCH;
-    const __nv_bfloat16* wb = ws + (kc & 1) * WCH;
+  const int n0 = warp * C::WN;
+  int no_abort = 0;
+#pragma unroll 1
+  for (int kc = 0; kc < C::NK; ++kc) {
+    const int s = kc % STAGES;
+    mbar_wait(bar0 + 8 * s, (kc / STAGES) & 1, &no_abort, nullptr, kProjWaitNs);
+    const uint32_t xb = sa + s * C::STAGE, wb = xb + C::XBYTES;
 #pragma unroll
     for (int ks = 0; ks < TK / 16; ++ks) {
-      uint32_t a[2][4];
+      uint32_t a[4][4];
 #pragma unroll
-      for (int mi = 0; mi < 2; ++mi)
-        ldmatrix_x4(a[mi][0], a[mi][1], a[mi][2], a[mi][3],
-                    xb + (wm * 32 + mi * 16 + (lane & 15)) * XS + ks * 16 + (lane >> 4) * 8);
+      for (int mi = 0; mi < 4; ++mi) {
+        const uint32_t ad = sw128(xb, mi * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8);
+        asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                     : "=r"(a[mi][0]), "=r"(a[mi][1]), "=r"(a[mi][2]), "=r"(a[mi][3])
+                     : "r"(ad));
+      }
 #pragma unroll
-      for (int np = 0; np < 4; ++np) {
+      for (int np = 0; np < NJ / 2; ++np) {
         uint32_t b0, b1, b2, b3;
         if (W_KN) {
-          ldmatrix_x4_trans(b0, b1, b2, b3,
-                            wb + (ks * 16 + (lane & 15)) * WKN + wn * 64 + np * 16 + (lane >> 4) * 8);
+          const int col = n0 + np * 16 + (lane >> 4) * 8;
+          const uint32_t ad = sw128(wb + (col >> 6) * (TK * 128), ks * 16 + (lane & 15), col & 63);
+          asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                       : "=r"(b0), "=r"(b1), "=r"(b2), "=r"(b3)
+                       : "r"(ad));
         } else {
-          ldmatrix_x4(b0, b1, b2, b3,
-                      wb + (wn * 64 + np * 16 + (lane & 7) + 8 * (lane >> 4)) * WNK + ks * 16 +
-                          8 * ((lane >> 3) & 1));
+          const uint32_t ad =
+              sw128(wb, n0 + np * 16 + (lane & 7) + 8 * (lane >> 4), ks * 16 + 8 * ((lane >> 3) & 1));
+          asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                       : "=r"(b0), "=r"(b1), "=r"(b2), "=r"(b3)
+                       : "r"(ad));
         }
 #pragma unroll
-        for (int mi = 0; mi < 2; ++mi) {
+        for (int mi = 0; mi < 4; ++mi) {
           mma_bf16_16816(acc[mi][2 * np], a[mi], b0, b1);
           mma_bf16_16816(acc[mi][2 * np + 1], a[mi], b2, b3);
         }
       }
     }
-    __syncthreads();
+    __syncthreads();  // everyone is done with stage s
+    const int nk = kc + STAGES;
+    if (tid == 0 && nk < C::NK) {
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar0 + 8 * s),
+                   "r"(C::STAGE)
+                   : "memory");
+      load_w(nk, s);
+      load_x(nk, s);
+    }
   }
 
 #pragma unroll
-  for (int mi = 0; mi < 2; ++mi) {
+  for (int mi = 0; mi < 4; ++mi) {
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      int t = t0 + wm * 32 + mi * 16 + (lane >> 2) + half * 8;
+    for (int hf = 0; hf < 2; ++hf) {
+      const int t = t0 + mi * 16 + (lane >> 2) + hf * 8;
       if (t >= n_tok) continue;
-      __nv_bfloat16* yrow = Y + ((size_t)t * H + h) * N + n0 + wn * 64 + 2 * (lane & 3);
+      __nv_bfloat16* yrow = Y + ((size_t)t * H + h) * N + n0 + 2 * (lane & 3);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        *reinterpret_cast<uint32_t*>(yrow + j * 8) =
-            pack_bf16(acc[mi][j][2 * half], acc[mi][j][2 * half + 1]);
-      }
+      for (int j = 0; j < NJ; ++j)
+        *reinterpret_cast<uint32_t*>(yrow + j * 8) = pack_bf16(acc[mi][j][2 * hf], acc[mi][j][2 * hf + 1]);
     }
   }
 }
 
-template <int K, int N, bool W_KN>
-cudaError_t launch_proj(const void* X, const void* W, void* Y, int n_tok, int H,
-                        cudaStream_t stream) {
-  constexpr int WCH = W_KN ? TK * WKN : TN * WNK;
-  const size_t smem = 2 * (TM * XS + WCH) * sizeof(__nv_bfloat16);
-  auto kern = proj_kernel<K, N, W_KN>;
+template <int K, int N, bool W_KN, int NWARPS, int STAGES>
+cudaError_t launch_proj(const void* X, const void* W, void* Y, int n_tok, int H, cudaStream_t stream) {
+  using C = ProjCfg<K, N, W_KN, NWARPS, STAGES>;
+  CUtensorMap tm_x, tm_w;
+  // X [n_tok][H][K]: dims (K, H, n_tok), boxes of 64 tokens x 1 head x 64 values
+  if (!tma_map_3d(&tm_x, X, K, H, n_tok, (uint64_t)K * 2, (uint64_t)H * K * 2, 64, 1, TM))
+    return cudaErrorInvalidValue;
+  const bool ok = W_KN ? tma_map_2d(&tm_w, W, N, (uint64_t)H * K, (uint64_t)N * 2, 64, TK)
+                       : tma_map_2d(&tm_w, W, K, (uint64_t)H * N, (uint64_t)K * 2, 64, N);
+  if (!ok) return cudaErrorInvalidValue;
+  auto kern = proj_kernel<K, N, W_KN, NWARPS, STAGES>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::smem);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  dim3 grid(N / TN, (n_tok + TM - 1) / TM, H);
-  return launch_pdl(kern, grid, dim3(128), smem, stream, static_cast<const __nv_bfloat16*>(X),
-                    static_cast<const __nv_bfloat16*>(W), static_cast<__nv_bfloat16*>(Y), n_tok, H);
+  dim3 grid((n_tok + TM - 1) / TM, H);
+  return launch_pdl(kern, grid, dim3(C::NT), C::smem, stream, tm_x, tm_w, static_cast<__nv_bfloat16*>(Y),
+                    n_tok, H);
 }
 
 }  // namespace
 
+// absorption: K = 128 (2 chunks, both in flight), N = 512, W_UK[h] is [K][N]; 8 warps x 64 columns
 cudaError_t launch_absorb_q(const void* q_nope, const void* w_uk, void* q_lat, int n_tok, int H,
                             cudaStream_t stream) {
-  return launch_proj<kDn, kDc, true>(q_nope, w_uk, q_lat, n_tok, H, stream);
+  return launch_proj<kDn, kDc, true, 8, 2>(q_nope, w_uk, q_lat, n_tok, H, stream);
 }
 
+// up-projection: K = 512 (8 chunks, 4 in flight), N = 128, W_UV[h] is [N][K]; 4 warps x 32 columns
 cudaError_t launch_up_proj_v(const void* o_lat, const void* w_uv, void* out, int n_tok, int H,
                              cudaStream_t stream) {
-  return launch_proj<kDc, kDv, false>(o_lat, w_uv, out, n_tok, H, stream);
+  return launch_proj<kDc, kDv, false, 4, 4>(o_lat, w_uv, out, n_tok, H, stream);
 }
 
 }  // namespace mla

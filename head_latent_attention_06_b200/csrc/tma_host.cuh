@@ -1,0 +1,20 @@
+// Host-side TMA tensor maps (bf16, 128-byte swizzle), cached by their parameters
+// so that a repeated call re-encodes nothing.
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+namespace mla {
+
+// 2-D map over `rows` rows of `cols` bf16 values, rows `row_bytes` apart; boxes of
+// box_rows x box_cols (box_cols * 2 <= 128).
+bool tma_map_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t row_bytes,
+                uint32_t box_cols, uint32_t box_rows);
+
+// 3-D map: dims (d0 values, d1, d2) with byte strides s1 (dim 1) and s2 (dim 2);
+// boxes of b2 x b1 x b0.
+bool tma_map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2);
+
+}  // namespace mla
