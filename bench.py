@@ -57,6 +57,11 @@ def shard_seed(base_seed: int, rank: int) -> int:
     return base_seed + 1000 * rank
 
 
+def whole_job_rate(world: int, bytes_per_rank: int, total_ms_max: float, steps: int) -> float:
+    """Bytes of all ranks per second over the slowest rank's device time (GB/s)."""
+    return world * bytes_per_rank * steps / (total_ms_max * 1e-3) / 1e9
+
+
 def reduce_max(x: float) -> float:
     import torch
     import torch.distributed as dist
@@ -294,7 +299,7 @@ def main(argv=None):
 
     peaks, peak_kind = load_peaks()
     hbm = float(peaks["hbm_gbs"])
-    value = world * cache_bytes / (ms_per_step * 1e-3) / 1e9
+    value = whole_job_rate(world, cache_bytes, total_ms, args.steps)
     dec_gbs = cache_bytes / (dec_avg_ms * 1e-3) / 1e9
     dec_tflops = flops / (dec_avg_ms * 1e-3) / 1e12
     t_mem = cache_bytes / (hbm * 1e9)
