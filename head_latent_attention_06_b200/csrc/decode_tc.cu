@@ -1,6 +1,8 @@
 // Paged latent-attention decode on the 5th-generation tensor cores (sm_100a):
 // tcgen05 MMAs over a CTA pair, accumulators in tensor memory (TMEM), cache
-// pages streamed by TMA.  This is the path for 128 heads and a bf16 cache.
+// pages streamed by TMA.  This is the path for a bf16 cache and up to 128 heads
+// (fewer heads pad the 128-row tile with zero rows: the step stays bound by the
+// cache stream, so the idle rows cost tensor work only).
 //
 // What it computes (absorbed MLA decode; nnets.ru article, sections "Суть MLA"
 // and "MLA и FlashAttention"; snowgate thread 35 on the 512 + 64 latent record):
@@ -261,12 +263,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool ok = load_s(0);
       pdl_wait();
       if (lane == 0) {
-        const int qrow = (b * p.s_q + g) * p.H + 64 * (int)r;
+        // 3-D maps (values, heads, query tokens): heads >= H come in as zeros
+        const int qtok = b * p.s_q + g, h0 = 64 * (int)r;
         const uint32_t qb = lead_bar(Q_FULL);
         if (r == 0) mbar_arrive_expect_tx_local(own_bar(Q_FULL), 2 * kQBytes);
         for (int c = kQTmemChunks; c < 8; ++c)
-          tma_load_2d_pair(sa + kQOff + (c - kQTmemChunks) * kChunkQ, &tm_q, qb, 64 * c, qrow);
-        tma_load_2d_pair(sa + kQOff + (8 - kQTmemChunks) * kChunkQ, &tm_qpe, qb, 0, qrow);
+          tma_load_3d_pair(sa + kQOff + (c - kQTmemChunks) * kChunkQ, &tm_q, qb, 64 * c, h0, qtok);
+        tma_load_3d_pair(sa + kQOff + (8 - kQTmemChunks) * kChunkQ, &tm_qpe, qb, 0, h0, qtok);
       }
       __syncwarp();
       for (int u = 0; ok && u < n; ++u) {
@@ -363,16 +366,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // (A operand of the score MMA: each 32-bit column holds two consecutive bf16;
     // lanes l and 64 + l both hold row l, the duplicated layout of the paired MMA)
     pdl_wait();
+    const int head = 64 * (int)r + m;        // rows beyond H pad the 128-row MMA tile
+    const bool row_ok = head < p.H;
     if (n > 0) {
       const uint4* qsrc =
-          reinterpret_cast<const uint4*>(p.q_lat + (((size_t)b * p.s_q + g) * p.H + 64 * r + m) * kDc);
+          reinterpret_cast<const uint4*>(p.q_lat + (((size_t)b * p.s_q + g) * p.H + (row_ok ? head : 0)) * kDc);
       constexpr int kPerWarp = (kQTmemChunks + 1) / 2;
 #pragma unroll 1
       for (int c = ch * kPerWarp; c < kQTmemChunks && c < (ch + 1) * kPerWarp; ++c) {
         uint32_t qv[32];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint4 v = __ldg(qsrc + c * 8 + k);
+          const uint4 v = row_ok ? __ldg(qsrc + c * 8 + k) : make_uint4(0u, 0u, 0u, 0u);
           qv[4 * k] = v.x;
           qv[4 * k + 1] = v.y;
           qv[4 * k + 2] = v.z;
@@ -479,7 +484,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const bool empty = !(ltot > 0.f) || !alive;
     const float inv = empty ? 0.f : 1.f / ltot;
     const float lse = empty ? -CUDART_INF_F : (m_used + log2f(ltot)) * 0.6931471805599453f;
-    const size_t orow = ((size_t)b * p.s_q + g) * p.H + 64 * r + m;
+    const size_t orow = ((size_t)b * p.s_q + g) * p.H + (row_ok ? head : 0);
     const bool read_o = alive && n > 0;
     // TMEM columns 128*ch .. +127 of this lane: latent half*128 + 256*ch + 0..127
 #pragma unroll 1
@@ -493,6 +498,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 32; ++j) ov[j] = 0u;
       }
       const int col = 256 * ch + half * 128 + 32 * c;
+      if (!row_ok) continue;
       if (p.splits == 1) {
         uint4* dst = reinterpret_cast<uint4*>(p.o_lat + orow * kDc + col);
 #pragma unroll
@@ -512,7 +518,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                __uint_as_float(ov[4 * k + 2]) * inv, __uint_as_float(ov[4 * k + 3]) * inv);
       }
     }
-    if (half == 0 && ch == 0) {
+    if (half == 0 && ch == 0 && row_ok) {
       if (p.splits == 1) {
         if (p.lse) p.lse[orow] = lse;
       } else {
@@ -539,17 +545,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }  // namespace
 
 bool decode_tc_supported(const mla_decode_args_t* a) {
-  return a->H == 128 && a->kv_dtype == MLA_KV_BF16;
+  // any head count up to 128 (rows beyond H pad the 128-row tile), bf16 cache
+  return a->H % 16 == 0 && a->H <= 128 && a->kv_dtype == MLA_KV_BF16;
 }
 
 int decode_tc_clusters_per_split(const mla_decode_args_t* a) { return a->B * a->s_q; }
 
 cudaError_t launch_decode_tc(const mla_decode_args_t* a, int splits, cudaStream_t stream) {
   CUtensorMap tm_q, tm_qpe, tm_ks, tm_kv;
-  const uint64_t rows_q = (uint64_t)a->B * a->s_q * a->H;
   const uint64_t rows_kv = (uint64_t)a->num_pages * kPage;
-  if (!tma_map_2d(&tm_q, a->q_lat, kDc, rows_q, kDc * 2, 64, 64) ||
-      !tma_map_2d(&tm_qpe, a->q_pe, kDr, rows_q, kDr * 2, 64, 64) ||
+  const int n_tok = a->B * a->s_q;
+  // query maps are 3-D (values, heads, tokens) so that a 64-head box past H reads zeros
+  if (!tma_map_3d(&tm_q, a->q_lat, kDc, a->H, n_tok, kDc * 2, (uint64_t)a->H * kDc * 2, 64, 64, 1) ||
+      !tma_map_3d(&tm_qpe, a->q_pe, kDr, a->H, n_tok, kDr * 2, (uint64_t)a->H * kDr * 2, 64, 64, 1) ||
       !tma_map_2d(&tm_ks, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 32) ||
       !tma_map_2d(&tm_kv, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 64))
     return cudaErrorInvalidValue;
@@ -560,7 +568,6 @@ cudaError_t launch_decode_tc(const mla_decode_args_t* a, int splits, cudaStream_
   p.seq_lens = a->seq_lens;
   p.o_lat = static_cast<__nv_bfloat16*>(a->o_lat);
   p.lse = a->lse;
-  const int n_tok = a->B * a->s_q;
   WorkspaceLayout wl = workspace_layout(n_tok, a->H, splits);
   unsigned char* ws = static_cast<unsigned char*>(a->workspace);
   p.status = reinterpret_cast<uint32_t*>(ws + wl.status_off);

@@ -147,6 +147,15 @@ MLA_DEVI void tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t mbar_clu
       : "memory");
 }
 
+MLA_DEVI void tma_load_3d_pair(uint32_t dst, const void* tmap, uint32_t mbar_cluster, int32_t x,
+                               int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(tmap), "r"(mbar_cluster), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 // Same, executed by a converged warp: one elected lane issues.
 MLA_DEVI void tma_load_2d_pair_elect(uint32_t dst, const void* tmap, uint32_t mbar_cluster, int32_t x,
                                      int32_t y) {

@@ -75,7 +75,7 @@ def test_workspace_size_is_host_only_and_grows_with_splits(lib):
 
 def test_auto_split_count(lib):
     # few sequences, long context: many splits; a batch that fills the GPU: one
-    assert mla.mla_decode_num_splits(_args(B=4, H=16, max_len=131072)) >= 32
+    assert mla.mla_decode_num_splits(_args(B=4, H=16, max_len=131072)) >= 16
     assert mla.mla_decode_num_splits(_args(B=4, H=128, max_len=131072)) >= 16
     assert mla.mla_decode_num_splits(_args(B=64, H=128, max_len=4096)) == 1
     assert mla.mla_decode_num_splits(_args(B=128, H=128, max_len=8192, s_q=2)) <= 2
