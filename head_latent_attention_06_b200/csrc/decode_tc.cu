@@ -40,10 +40,24 @@
 // P.V of t.  The output rescale is lazy: the reference maximum moves only when
 // the tile maximum exceeds it by more than 2^8, so O in TMEM is rarely touched.
 //
+// fp8 (e4m3) cache with a per-token scale: the MMAs run on f16 operands.  Every
+// e4m3 value is exactly an f16 value, so the cache needs only a format change:
+// the producer brings the raw bytes of a stage into the back half of its slot
+// (the CTA's 32 rows with one bulk copy; the value operand's 64 rows x 2 x 128
+// bytes with two TMA boxes), four converter warps (12..15) read the whole stage,
+// then write it back as f16 in the layout the TMA gives the bf16 cache, and mark
+// the slot full.  Q is rounded from bf16 to f16 once (exact inside f16's normal
+// range).  The token scales stay out of the operands: the softmax multiplies
+// the raw scores by them, and P by them before the P.V MMA, so that
+// O = sum_t p_t * scale_t * code_t.  Rows past the sequence end are written as
+// zeros in the value operand, so that whatever bytes they hold cannot reach O.
+//
 // Every mbarrier wait is bounded (MLA_ERR_DEVICE_TIMEOUT in the status word,
 // then an orderly exit that drains issued MMAs and frees TMEM).
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <math_constants.h>
 
 #include "sm100.cuh"
@@ -54,7 +68,10 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 384;
+constexpr int kThreadsBf16 = 384;            // warps 0..11
+constexpr int kConvWarps = 4;                // fp8: converter warps 12..15
+constexpr int kThreadsFp8 = kThreadsBf16 + 32 * kConvWarps;
+constexpr int kScRing = 8;                   // fp8: per-tile token scales (64 floats each)
 constexpr uint32_t kChunkQ = 64 * 128;              // 64 rows x 64 bf16
 #ifndef MLA_TC_Q_TMEM_CHUNKS
 #define MLA_TC_Q_TMEM_CHUNKS 6
@@ -79,7 +96,8 @@ constexpr uint32_t kQOff = 0;
 constexpr uint32_t kSOff = kQOff + kQBytes;
 constexpr uint32_t kVOff = kSOff + kSStages * kSStage;
 constexpr uint32_t kPOff = kVOff + kVStages * kVStage;  // two P buffers
-constexpr uint32_t kBarOff = kPOff + 2 * kPBytes;
+constexpr uint32_t kScOff = kPOff + 2 * kPBytes;      // fp8 token scales [kScRing][64]
+constexpr uint32_t kBarOff = kScOff + kScRing * 256;
 // barrier indices
 constexpr int S_FULL = 0;                  // [kSStages] in the even CTA: stage filled in both CTAs
 constexpr int S_EMPTY = S_FULL + kSStages; // [kSStages] in each CTA: stage consumed by the MMAs
@@ -91,7 +109,14 @@ constexpr int S_READY = Q_TMEM + 1;        // [2]
 constexpr int P_READY = S_READY + 2;      // [2] in the even CTA
 constexpr int O_DONE = P_READY + 2;       // [2]
 constexpr int DRAIN = O_DONE + 2;        // [2] one per MMA-issuing warp
-constexpr int NBARS = DRAIN + 2;
+constexpr int RAW_S = DRAIN + 2;          // [kSStages] fp8: raw bytes of a score stage landed
+constexpr int RAW_V = RAW_S + kSStages;   // [kVStages] fp8: raw bytes of a value stage landed
+constexpr int SC_FULL = RAW_V + kVStages; // [kScRing]  fp8: token scales of a tile landed
+constexpr int NBARS = SC_FULL + kScRing;
+// A scale entry is reloaded for tile u + kScRing only after the score stage of
+// tile u + kScRing - kSStages was consumed, which needed the softmax of tile
+// u + kScRing - kSStages - 2 to be done; the softmax of tile u must be among them.
+static_assert(kScRing >= kSStages + 2 + 1, "scale ring too short");
 constexpr int kSoftmaxWarps = 8;          // warps 4..11: two per TMEM lane quadrant
 constexpr int kPrefetchTiles = MLA_TC_PREFETCH;      // L2 prefetch distance of the cache stream
 constexpr uint32_t kMiscOff = kBarOff + 8 * NBARS;
@@ -107,12 +132,16 @@ static_assert(kTmemQ + kQTmemChunks * 32 <= kTmemCols, "TMEM budget");
 constexpr uint64_t kWaitLimitNs = 2000000000ull;     // 2 s
 constexpr float kRescaleThreshold = 8.0f;            // log2 units
 
-constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, false, false);
-constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
+template <bool FP8>
+constexpr uint32_t idesc_s() { return FP8 ? idesc_f16_f32(128, 64, false, false) : idesc_bf16_f32(128, 64, false, false); }
+template <bool FP8>
+constexpr uint32_t idesc_pv() { return FP8 ? idesc_f16_f32(128, 256, false, true) : idesc_bf16_f32(128, 256, false, true); }
 
 struct TcParams {
   const __nv_bfloat16* q_lat;
+  const __nv_bfloat16* q_pe;
   const uint8_t* kv;
+  const float* kv_scale;  // fp8: [num_pages][64]
   const int32_t* block_table;
   const int32_t* seq_lens;
   __nv_bfloat16* o_lat;
@@ -131,7 +160,34 @@ MLA_DEVI float ex2_approx(float x) {
   return y;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+// bf16 pair -> f16 pair (round to nearest even; exact inside f16's normal range)
+MLA_DEVI uint32_t bf16x2_to_f16x2(uint32_t x) {
+  const __half2 h = __floats2half2_rn(__uint_as_float(x << 16), __uint_as_float(x & 0xFFFF0000u));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+MLA_DEVI uint32_t pack_f16(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// 16 e4m3 codes (16 bytes, lowest address first) -> 16 f16 values, exactly
+MLA_DEVI void e4m3x16_to_f16(const uint4 v, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] & 0xFFFFu), __NV_E4M3);
+    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] >> 16), __NV_E4M3);
+    o[2 * k] = (uint32_t)a.x | ((uint32_t)a.y << 16);
+    o[2 * k + 1] = (uint32_t)b.x | ((uint32_t)b.y << 16);
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+template <bool FP8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : kThreadsBf16, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qpe,
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_kv,
                      const TcParams p) {
@@ -168,14 +224,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     if (bad_len && r == 0 && g == 0 && split == 0) set_status(p.status, MLA_ERR_BAD_SEQ_LEN);
     *abort_flag = 0;
+    // bf16: a full score stage is the even CTA's expect_tx plus both CTAs' TMA
+    // bytes, a full value stage that and the odd CTA's arrival (a last, partial
+    // page instead takes one arrival per CTA after its tail rows are zeroed);
+    // fp8: the arrivals of both CTAs' converter warps
+    const uint32_t full_count = FP8 ? 2 * kConvWarps : 1;
     for (int i = 0; i < kSStages; ++i) {
-      mbar_init(own_bar(S_FULL + i), 1);
+      mbar_init(own_bar(S_FULL + i), full_count);
       mbar_init(own_bar(S_EMPTY + i), 1);
+      mbar_init(own_bar(RAW_S + i), 1);
     }
     for (int i = 0; i < kVStages; ++i) {
-      mbar_init(own_bar(V_FULL + i), 1);
+      mbar_init(own_bar(V_FULL + i), FP8 ? full_count : 2);
       mbar_init(own_bar(V_EMPTY + i), 1);
+      mbar_init(own_bar(RAW_V + i), 1);
     }
+    for (int i = 0; i < kScRing; ++i) mbar_init(own_bar(SC_FULL + i), 1);
     mbar_init(own_bar(Q_TMEM), 2 * kSoftmaxWarps);
     mbar_init(own_bar(Q_FULL), 1);
     for (int i = 0; i < 2; ++i) {
@@ -226,9 +290,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         return __shfl_sync(0xffffffffu, pg, u & 31);
       };
       // the CTA's half page (32 contiguous rows) of tile u, into L2 ahead of its TMA
+      constexpr int kElem = FP8 ? 1 : 2;  // bytes per cached value
       auto prefetch = [&](int u) {
         const int pg = page_of(u, blk_p, pg_p);
-        if (lane == 0) prefetch_l2_bulk(p.kv + ((size_t)pg * kPage + 32 * r) * kRow * 2, kSStage);
+        if (lane == 0) prefetch_l2_bulk(p.kv + ((size_t)pg * kPage + 32 * r) * kRow * kElem, 32 * kRow * kElem);
       };
       for (int u = 0; u < n && u < kPrefetchTiles; ++u) prefetch(u);
       auto load_s = [&](int u) -> bool {
@@ -236,11 +301,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t ph = ((u / kSStages) & 1) ^ 1;
         if (!mbar_wait_converged(own_bar(S_EMPTY + st), ph, abort_flag, p.status, kWaitLimitNs)) return false;
         const int pg = page_of(u, blk_s, pg_s);
-        const uint32_t fb = lead_bar(S_FULL + st);
-        if (r == 0) mbar_arrive_expect_tx_local_elect(own_bar(S_FULL + st), 2 * kSStage);
         const uint32_t dst = sa + kSOff + st * kSStage;
-        for (int c = 0; c < 9; ++c)
-          tma_load_2d_pair_elect(dst + c * kChunkS, &tm_ks, fb, 64 * c, pg * kPage + 32 * (int)r);
+        if constexpr (FP8) {
+          // raw e4m3 rows 32r .. 32r+31 of the page (contiguous) into the back half
+          // of the slot, and the page's 64 token scales
+          if (lane == 0) {
+            mbar_arrive_expect_tx_local(own_bar(RAW_S + st), kSStage / 2);
+            bulk_load_cta(dst + kSStage / 2, p.kv + ((size_t)pg * kPage + 32 * r) * kRow, kSStage / 2,
+                          own_bar(RAW_S + st));
+            const int e = u % kScRing;
+            mbar_arrive_expect_tx_local(own_bar(SC_FULL + e), 256);
+            bulk_load_cta(sa + kScOff + 256 * e, p.kv_scale + (size_t)pg * kPage, 256, own_bar(SC_FULL + e));
+          }
+          __syncwarp();
+        } else {
+          const uint32_t fb = lead_bar(S_FULL + st);
+          if (r == 0) mbar_arrive_expect_tx_local_elect(own_bar(S_FULL + st), 2 * kSStage);
+          for (int c = 0; c < 9; ++c)
+            tma_load_2d_pair_elect(dst + c * kChunkS, &tm_ks, fb, 64 * c, pg * kPage + 32 * (int)r);
+        }
         if (u + kPrefetchTiles < n) prefetch(u + kPrefetchTiles);
         return true;
       };
@@ -249,12 +328,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t ph = ((u / kVStages) & 1) ^ 1;
         if (!mbar_wait_converged(own_bar(V_EMPTY + st), ph, abort_flag, p.status, kWaitLimitNs)) return false;
         const int pg = page_of(u, blk_v, pg_v);
-        const uint32_t fb = lead_bar(V_FULL + st);
-        if (r == 0) mbar_arrive_expect_tx_local_elect(own_bar(V_FULL + st), 2 * kVStage);
         const uint32_t dst = sa + kVOff + st * kVStage;
-        for (int j = 0; j < 4; ++j) {
-          const int lc = 4 * (j >> 1) + 2 * (int)r + (j & 1);  // latent chunk: halves {2r, 2r+1}, {4+2r, 5+2r}
-          tma_load_2d_pair_elect(dst + j * kChunkV, &tm_kv, fb, 64 * lc, pg * kPage);
+        if constexpr (FP8) {
+          // raw bytes 128r .. +127 and 256+128r .. +127 of the page's 64 rows (the
+          // map views a row as 288 two-byte units) into the back half of the slot
+          if (lane == 0) {
+            mbar_arrive_expect_tx_local(own_bar(RAW_V + st), kVStage / 2);
+            for (int seg = 0; seg < 2; ++seg)
+              tma_load_2d_cta(dst + kVStage / 2 + seg * (kVStage / 4), &tm_kv, own_bar(RAW_V + st),
+                              64 * (int)r + 128 * seg, pg * kPage);
+          }
+          __syncwarp();
+        } else {
+          const int nvalid = j_end - (t0 + u) * kPage;  // cached rows of this page inside the sequence
+          if (nvalid >= kPage) {
+            const uint32_t fb = lead_bar(V_FULL + st);
+            if (r == 0) mbar_arrive_expect_tx_local_elect(own_bar(V_FULL + st), 2 * kVStage);
+            else if (lane == 0) mbar_arrive_remote_relaxed(fb);
+            for (int j = 0; j < 4; ++j) {
+              const int lc = 4 * (j >> 1) + 2 * (int)r + (j & 1);  // latent chunk: halves {2r, 2r+1}, {4+2r, 5+2r}
+              tma_load_2d_pair_elect(dst + j * kChunkV, &tm_kv, fb, 64 * lc, pg * kPage);
+            }
+          } else {
+            // The last page of the sequence: P is 0 past the end, but 0 * NaN is
+            // not, so whatever those rows hold is replaced by zeros before the MMA.
+            // The stage lands on this CTA's own barrier (once per work unit).
+            if (lane == 0) {
+              mbar_arrive_expect_tx_local(own_bar(RAW_V + st), kVStage);
+              for (int j = 0; j < 4; ++j) {
+                const int lc = 4 * (j >> 1) + 2 * (int)r + (j & 1);
+                tma_load_2d_cta(dst + j * kChunkV, &tm_kv, own_bar(RAW_V + st), 64 * lc, pg * kPage);
+              }
+            }
+            __syncwarp();
+            if (!mbar_wait_converged(own_bar(RAW_V + st), 0, abort_flag, p.status, kWaitLimitNs)) return false;
+            const int units = (kPage - nvalid) * 8;  // 16-byte units per chunk past the end
+            for (int q = lane; q < 4 * units; q += 32) {
+              const int j = q / units, rem = q - j * units;
+              *reinterpret_cast<uint4*>(sm + kVOff + st * kVStage + j * kChunkV + (nvalid + (rem >> 3)) * 128 +
+                                        (rem & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(lead_bar(V_FULL + st));
+          }
         }
         return true;
       };
@@ -262,7 +379,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // may overlap with (the query absorption); q_lat is, so Q waits for it.
       bool ok = load_s(0);
       pdl_wait();
-      if (lane == 0) {
+      if (!FP8 && lane == 0) {
         // 3-D maps (values, heads, query tokens): heads >= H come in as zeros
         const int qtok = b * p.s_q + g, h0 = 64 * (int)r;
         const uint32_t qb = lead_bar(Q_FULL);
@@ -288,7 +405,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint64_t dp = desc_sw128(sa + kPOff, 16, 1024);
       bool ok = true;
       if (warp == 1) {
-        ok = mbar_wait_converged(own_bar(Q_FULL), 0, abort_flag, p.status, kWaitLimitNs) &&
+        // fp8: the softmax warps write all of Q (TMEM and shared memory parts)
+        ok = (FP8 || mbar_wait_converged(own_bar(Q_FULL), 0, abort_flag, p.status, kWaitLimitNs)) &&
              mbar_wait_converged(own_bar(Q_TMEM), 0, abort_flag, p.status, kWaitLimitNs);
         for (int u = 0; ok && u < n; ++u) {
           const int st = u % kSStages, sb = u & 1;
@@ -306,18 +424,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kQTmemChunks; ++c) {
             const uint32_t aq = tmem + kTmemQ + 32u * c;
             const uint64_t bs = bs0 + ((c * kChunkS) >> 4);
-            mma_pair_ts_elect(d, aq, bs, kIdescS, c != 0);
-            mma_pair_ts_elect(d, aq + 8, bs + 2, kIdescS, 1);
-            mma_pair_ts_elect(d, aq + 16, bs + 4, kIdescS, 1);
-            mma_pair_ts_elect(d, aq + 24, bs + 6, kIdescS, 1);
+            mma_pair_ts_elect(d, aq, bs, idesc_s<FP8>(), c != 0);
+            mma_pair_ts_elect(d, aq + 8, bs + 2, idesc_s<FP8>(), 1);
+            mma_pair_ts_elect(d, aq + 16, bs + 4, idesc_s<FP8>(), 1);
+            mma_pair_ts_elect(d, aq + 24, bs + 6, idesc_s<FP8>(), 1);
           }
 #pragma unroll
           for (int c = kQTmemChunks; c < 9; ++c) {
             const uint64_t aq = dq + (((c - kQTmemChunks) * kChunkQ) >> 4), bs = bs0 + ((c * kChunkS) >> 4);
-            mma_pair_elect(d, aq, bs, kIdescS, c != 0);
-            mma_pair_elect(d, aq + 2, bs + 2, kIdescS, 1);
-            mma_pair_elect(d, aq + 4, bs + 4, kIdescS, 1);
-            mma_pair_elect(d, aq + 6, bs + 6, kIdescS, 1);
+            mma_pair_elect(d, aq, bs, idesc_s<FP8>(), c != 0);
+            mma_pair_elect(d, aq + 2, bs + 2, idesc_s<FP8>(), 1);
+            mma_pair_elect(d, aq + 4, bs + 4, idesc_s<FP8>(), 1);
+            mma_pair_elect(d, aq + 6, bs + 6, idesc_s<FP8>(), 1);
           }
           commit_pair_mc_elect(own_bar(S_EMPTY + st), 0x3);
           commit_pair_mc_elect(own_bar(S_READY + sb), 0x3);
@@ -336,7 +454,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int h = 0; h < 2; ++h) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_pair_elect(tmem + 128u * h, ap + kk * 2, bv + ((2 * h * kChunkV + kk * 2048) >> 4), kIdescPV,
+              mma_pair_elect(tmem + 128u * h, ap + kk * 2, bv + ((2 * h * kChunkV + kk * 2048) >> 4), idesc_pv<FP8>(),
                              (t > 0 || kk > 0) ? 1u : 0u);
           }
           commit_pair_mc_elect(own_bar(V_EMPTY + st), 0x3);
@@ -349,7 +467,84 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int dummy = 0;
       mbar_wait_converged(own_bar(db), 0, &dummy, p.status, kWaitLimitNs);
     }
-  } else if (warp >= 4) {
+  } else if (FP8 && warp >= 12) {
+    // ====================== fp8 -> f16 converters (fp8 only) ======================
+    // Same stage order as the producer: S(0), S(1), V(0), S(2), V(1), ...  Each
+    // stage is read whole into registers, the four warps meet, and the f16 values
+    // are written over the slot (the raw bytes sit in its back half).
+    const int ct = threadIdx.x - kThreadsBf16;  // 0 .. 127
+    auto convert_s = [&](int u) {
+      const int st = u % kSStages;
+      mbar_wait(own_bar(RAW_S + st), (u / kSStages) & 1, abort_flag, p.status, kWaitLimitNs);
+      const uint32_t slot = sa + kSOff + st * kSStage;
+      const uint32_t raw = slot + kSStage / 2;  // 32 rows x 576 bytes
+      // rows i (even) and i + 1 share a quarter-warp, four 16-byte units each: the
+      // reads (576-byte row pitch) and the swizzled writes both hit 8 distinct bank groups
+      const int i = 2 * (ct >> 3) + ((ct >> 2) & 1), w = 2 * (ct & 3);
+      uint4 v[9];
+#pragma unroll
+      for (int c = 0; c < 9; ++c)
+        v[c] = lds128(raw + i * kRow + 16 * (4 * c + (ct & 3)));
+      named_bar_sync(5, 32 * kConvWarps);
+#pragma unroll
+      for (int c = 0; c < 9; ++c) {
+        // values 64c + 16(ct&3) .. +15 of row i: f16 units w, w + 1 of chunk c
+        uint4 lo, hi;
+        e4m3x16_to_f16(v[c], lo, hi);
+        const uint32_t row = slot + c * kChunkS + i * 128;
+        sts128(row + ((w ^ (i & 7)) << 4), lo);
+        sts128(row + (((w + 1) ^ (i & 7)) << 4), hi);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(lead_bar(S_FULL + st));
+    };
+    auto convert_v = [&](int u) {
+      const int st = u % kVStages;
+      mbar_wait(own_bar(RAW_V + st), (u / kVStages) & 1, abort_flag, p.status, kWaitLimitNs);
+      const uint32_t slot = sa + kVOff + st * kVStage;
+      const uint32_t raw = slot + kVStage / 2;  // [2 segments][64 rows][128 bytes], 128-byte swizzle
+      const int nvalid = j_end - (t0 + u) * kPage;  // rows at or past it are zeroed
+      // item = (segment, row pair, flip); a quarter-warp takes rows i, i + 1 and
+      // units e ^ 4flip: conflict-free reads and writes
+      auto coords = [&](int k, int& seg, int& i, int& uu) {
+        const int item = 16 * k + (ct >> 3);
+        seg = item >> 6;
+        i = 2 * ((item >> 1) & 31) + ((ct >> 2) & 1);
+        uu = (ct & 7) ^ (4 * (item & 1));
+      };
+      uint4 v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        int seg, i, uu;
+        coords(k, seg, i, uu);
+        v[k] = lds128(raw + seg * (kVStage / 4) + i * 128 + ((uu ^ (i & 7)) << 4));
+      }
+      named_bar_sync(5, 32 * kConvWarps);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        int seg, i, uu;
+        coords(k, seg, i, uu);
+        uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
+        if (i < nvalid) e4m3x16_to_f16(v[k], lo, hi);
+        // values 16uu .. 16uu+15 of the segment: chunk 2seg + uu/4, f16 units 2(uu&3), +1
+        const uint32_t row = slot + (2 * seg + (uu >> 2)) * kChunkV + i * 128;
+        const int w = 2 * (uu & 3);
+        sts128(row + ((w ^ (i & 7)) << 4), lo);
+        sts128(row + (((w + 1) ^ (i & 7)) << 4), hi);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(lead_bar(V_FULL + st));
+    };
+    if (n > 0) {
+      convert_s(0);
+      for (int u = 0; u < n; ++u) {
+        if (u + 1 < n) convert_s(u + 1);
+        convert_v(u);
+      }
+    }
+  } else if (warp >= 4 && warp < 12) {
     // ====================== softmax / correction / epilogue ======================
     // Thread = (TMEM lane lt, column half ch).  Lane lt holds head row m = lt % 64
     // for tokens 32*half .. 32*half+31 of the page (half = lt / 64); the two warps
@@ -378,12 +573,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint4 v = row_ok ? __ldg(qsrc + c * 8 + k) : make_uint4(0u, 0u, 0u, 0u);
-          qv[4 * k] = v.x;
-          qv[4 * k + 1] = v.y;
-          qv[4 * k + 2] = v.z;
-          qv[4 * k + 3] = v.w;
+          qv[4 * k] = FP8 ? bf16x2_to_f16x2(v.x) : v.x;
+          qv[4 * k + 1] = FP8 ? bf16x2_to_f16x2(v.y) : v.y;
+          qv[4 * k + 2] = FP8 ? bf16x2_to_f16x2(v.z) : v.z;
+          qv[4 * k + 3] = FP8 ? bf16x2_to_f16x2(v.w) : v.w;
         }
         tmem_st32(tl + kTmemQ + 32u * c, qv);
+      }
+      if constexpr (FP8) {
+        // the shared-memory chunks of Q as f16 (128-byte swizzled rows, the layout
+        // TMA gives the bf16 path); the row's four threads take six 16-byte units each
+        static_assert(kQSmemChunks * 8 % 4 == 0, "Q units per thread");
+        constexpr int kUnits = kQSmemChunks * 8 / 4;
+        const size_t qr = ((size_t)b * p.s_q + g) * p.H + (row_ok ? head : 0);
+        const int qi = 2 * half + ch;
+#pragma unroll
+        for (int k = 0; k < kUnits; ++k) {
+          const int gu = qi * kUnits + k, cs = gu >> 3, w = gu & 7, c = kQTmemChunks + cs;
+          const uint4* src = c < 8 ? reinterpret_cast<const uint4*>(p.q_lat + qr * kDc + 64 * c + 8 * w)
+                                   : reinterpret_cast<const uint4*>(p.q_pe + qr * kDr + 8 * w);
+          uint4 v = row_ok ? __ldg(src) : make_uint4(0u, 0u, 0u, 0u);
+          v = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
+          *reinterpret_cast<uint4*>(sm + kQOff + cs * kChunkQ + m * 128 + ((w ^ (m & 7)) << 4)) = v;
+        }
+        fence_proxy_async_smem();
       }
       tmem_wait_st();
       tc_fence_before();
@@ -403,14 +616,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tmem_wait_ld();
       const int j0 = (t0 + t) * kPage + 32 * half + 16 * ch;
       const int nv = max(0, min(16, lim - j0));
+      // fp8: token scales of these 16 columns (0 where masked, so that nothing a
+      // masked row holds reaches P)
+      float sc[16];
+      if constexpr (FP8) {
+        mbar_wait(own_bar(SC_FULL + t % kScRing), (t / kScRing) & 1, abort_flag, p.status, kWaitLimitNs);
+        const float4* sp = reinterpret_cast<const float4*>(sm + kScOff + 256 * (t % kScRing)) + 8 * half + 4 * ch;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float4 f = sp[k];
+          sc[4 * k] = 4 * k < nv ? f.x : 0.f;
+          sc[4 * k + 1] = 4 * k + 1 < nv ? f.y : 0.f;
+          sc[4 * k + 2] = 4 * k + 2 < nv ? f.z : 0.f;
+          sc[4 * k + 3] = 4 * k + 3 < nv ? f.w : 0.f;
+        }
+      }
       float s[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) s[j] = j < nv ? __uint_as_float(sv[j]) : -CUDART_INF_F;
+      for (int j = 0; j < 16; ++j)
+        s[j] = j < nv ? (FP8 ? __uint_as_float(sv[j]) * sc[j] : __uint_as_float(sv[j])) : -CUDART_INF_F;
       float mx[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) mx[k] = fmaxf(fmaxf(s[k], s[k + 4]), fmaxf(s[k + 8], s[k + 12]));
       // the softmax scale is positive: scaling commutes with the maximum
-      const float lmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
+      float lmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
+      if constexpr (FP8) {
+        // the reference of O (and l) bounds x_t + log2(scale_t) rather than x_t, so
+        // that every P entry p_t * scale_t stays at or below 2^8 whatever the scales
+        float scm = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) scm = fmaxf(scm, sc[j]);
+        if (nv > 0) lmax += __log2f(fmaxf(scm, 0x1p-64f));
+      }
       float* xm = xmax + sb * 256;
       xm[ch * 128 + lt] = lmax;
       named_bar_sync(grp_bar, 128);
@@ -437,7 +674,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const float p0 = ex2_approx(fmaf(s[j], p.scale_log2, nref));
         const float p1 = ex2_approx(fmaf(s[j + 1], p.scale_log2, nref));
         ls[(j >> 1) & 3] += p0 + p1;
-        pk[j >> 1] = pack_bf16(p0, p1);
+        // fp8: the P.V operand carries the token scale (the cache operand is the raw code)
+        pk[j >> 1] = FP8 ? pack_f16(p0 * sc[j], p1 * sc[j + 1]) : pack_bf16(p0, p1);
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       // P buffer sb was last read by PV(t-2)
@@ -542,28 +780,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-}  // namespace
-
-bool decode_tc_supported(const mla_decode_args_t* a) {
-  // any head count up to 128 (rows beyond H pad the 128-row tile), bf16 cache
-  return a->H % 16 == 0 && a->H <= 128 && a->kv_dtype == MLA_KV_BF16;
-}
-
-int decode_tc_clusters_per_split(const mla_decode_args_t* a) { return a->B * a->s_q; }
-
-cudaError_t launch_decode_tc(const mla_decode_args_t* a, int splits, cudaStream_t stream) {
+template <bool FP8>
+cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t stream) {
   CUtensorMap tm_q, tm_qpe, tm_ks, tm_kv;
   const uint64_t rows_kv = (uint64_t)a->num_pages * kPage;
   const int n_tok = a->B * a->s_q;
   // query maps are 3-D (values, heads, tokens) so that a 64-head box past H reads zeros
   if (!tma_map_3d(&tm_q, a->q_lat, kDc, a->H, n_tok, kDc * 2, (uint64_t)a->H * kDc * 2, 64, 64, 1) ||
-      !tma_map_3d(&tm_qpe, a->q_pe, kDr, a->H, n_tok, kDr * 2, (uint64_t)a->H * kDr * 2, 64, 64, 1) ||
-      !tma_map_2d(&tm_ks, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 32) ||
-      !tma_map_2d(&tm_kv, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 64))
+      !tma_map_3d(&tm_qpe, a->q_pe, kDr, a->H, n_tok, kDr * 2, (uint64_t)a->H * kDr * 2, 64, 64, 1))
     return cudaErrorInvalidValue;
+  if (FP8) {
+    // the e4m3 rows (576 bytes) viewed as 288 two-byte units: boxes of 128 bytes x 64 rows
+    if (!tma_map_2d(&tm_kv, a->kv_cache, kRow / 2, rows_kv, kRow, 64, 64)) return cudaErrorInvalidValue;
+    tm_ks = tm_kv;  // unused: the score operand's raw rows come by a plain bulk copy
+  } else if (!tma_map_2d(&tm_ks, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 32) ||
+             !tma_map_2d(&tm_kv, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 64)) {
+    return cudaErrorInvalidValue;
+  }
   TcParams p;
   p.q_lat = static_cast<const __nv_bfloat16*>(a->q_lat);
+  p.q_pe = static_cast<const __nv_bfloat16*>(a->q_pe);
   p.kv = static_cast<const uint8_t*>(a->kv_cache);
+  p.kv_scale = a->kv_scale;
   p.block_table = a->block_table;
   p.seq_lens = a->seq_lens;
   p.o_lat = static_cast<__nv_bfloat16*>(a->o_lat);
@@ -581,19 +819,36 @@ cudaError_t launch_decode_tc(const mla_decode_args_t* a, int splits, cudaStream_
   p.causal = a->causal;
   p.splits = splits;
   p.scale_log2 = a->softmax_scale * kLog2e;
+  auto kern = decode_tc_kernel<FP8>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   dim3 grid(2 * splits, a->s_q, a->B);
-  return launch_pdl(decode_tc_kernel, grid, dim3(kThreads), kSmemBytes, stream, tm_q, tm_qpe, tm_ks, tm_kv, p);
+  return launch_pdl(kern, grid, dim3(FP8 ? kThreadsFp8 : kThreadsBf16), kSmemBytes, stream, tm_q, tm_qpe, tm_ks,
+                    tm_kv, p);
+}
+
+}  // namespace
+
+bool decode_tc_supported(const mla_decode_args_t* a) {
+  // any head count up to 128 (rows beyond H pad the 128-row tile); a bf16 cache,
+  // or an e4m3 cache whose scale array starts on 16 bytes (bulk copies)
+  if (a->H % 16 != 0 || a->H > 128) return false;
+  if (a->kv_dtype == MLA_KV_BF16) return true;
+  return a->kv_dtype == MLA_KV_FP8_E4M3 && (reinterpret_cast<uintptr_t>(a->kv_scale) & 15u) == 0;
+}
+
+int decode_tc_clusters_per_split(const mla_decode_args_t* a) { return a->B * a->s_q; }
+
+cudaError_t launch_decode_tc(const mla_decode_args_t* a, int splits, cudaStream_t stream) {
+  return a->kv_dtype == MLA_KV_FP8_E4M3 ? launch_tc<true>(a, splits, stream) : launch_tc<false>(a, splits, stream);
 }
 
 }  // namespace mla

@@ -47,6 +47,11 @@ MLA_DEVI void mbar_arrive_cluster(uint32_t addr) {
 MLA_DEVI void mbar_arrive_remote(uint32_t addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
 }
+// Arrive on a barrier of either CTA of the pair with no ordering of this thread's
+// memory operations (for arrivals that only count).
+MLA_DEVI void mbar_arrive_remote_relaxed(uint32_t addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
 MLA_DEVI void mbar_arrive_expect_tx_local(uint32_t addr, uint32_t tx) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(addr), "r"(tx) : "memory");
 }
@@ -178,6 +183,25 @@ MLA_DEVI void mbar_arrive_expect_tx_local_elect(uint32_t addr, uint32_t tx) {
       : "memory");
 }
 
+// 2-D tile load into this CTA's shared memory, completion counted on a barrier
+// of this CTA.
+MLA_DEVI void tma_load_2d_cta(uint32_t dst, const void* tmap, uint32_t mbar, int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(tmap), "r"(mbar), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Contiguous copy of `bytes` (multiple of 16; both addresses 16-byte aligned)
+// from global to this CTA's shared memory, completion counted on `mbar`.
+MLA_DEVI void bulk_load_cta(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(mbar)
+      : "memory");
+}
+
 // Brings `bytes` (multiple of 16) of global memory at a 16-byte aligned address
 // into L2 without touching shared memory.
 MLA_DEVI void prefetch_l2_bulk(const void* gaddr, uint32_t bytes) {
@@ -186,6 +210,17 @@ MLA_DEVI void prefetch_l2_bulk(const void* gaddr, uint32_t bytes) {
 
 MLA_DEVI void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
+// 16-byte shared-memory accesses at 32-bit shared addresses
+MLA_DEVI uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+MLA_DEVI void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
 }
 
 MLA_DEVI void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -207,6 +242,12 @@ MLA_DEVI uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
          ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Same for f16 A and B (format fields 0).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // ---------------------------------------------------------------- tcgen05

@@ -55,6 +55,8 @@ SMALL = [
     ("bf16", 16, 1, False, [300, 5000], 0),
     ("bf16", 64, 2, True, [100, 129], 2),
     ("fp8", 32, 1, False, [1000, 31], 0),
+    ("fp8", 16, 1, False, [300, 5000], 0),
+    ("fp8", 128, 1, False, [1, 63, 64, 65, 200, 1000], 3),
     ("bf16", 48, 1, False, [95], 0),
 ]
 
@@ -111,6 +113,62 @@ def test_page_permutation_is_bit_exact(cuda_lib, kv, H):
     assert not torch.equal(a.block_table, b.block_table)
     oa, ob = _run(cuda_lib, a).out, _run(cuda_lib, b).out
     assert torch.equal(oa, ob)
+
+
+def _poison_page_tails(w):
+    """Fill the cache rows past each sequence's end (and, fp8, their scales) with NaN."""
+    for b, L in enumerate(w.lens):
+        if L % 64 == 0:
+            continue
+        pg = int(w.block_table[b, L // 64])
+        if w.spec.kv_dtype == "fp8":
+            w.kv_cache[pg, L % 64:] = torch.full((64 - L % 64, 576), float("nan")).to(w.kv_cache.dtype)
+            w.kv_scale[pg, L % 64:] = float("nan")
+        else:
+            w.kv_cache[pg, L % 64:] = float("nan")
+
+
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+@pytest.mark.parametrize("H", [128, 32])
+def test_bytes_past_the_sequence_end_never_reach_the_output(cuda_lib, kv, H):
+    """Rows of a last page past the length are not part of the sequence: NaN there changes nothing."""
+    w = make_workload(_spec(kv, H, 2, [70, 1000, 129], causal=True))
+    clean = _run(cuda_lib, w, 2)
+    o_clean, lse_clean = clean.out.clone(), clean.lse.clone()
+    _poison_page_tails(w)
+    for splits in (1, 2):
+        st = _run(cuda_lib, w, splits)
+        assert torch.isfinite(st.out).all() and torch.isfinite(st.lse).all()
+        ma, rl = errors(to_np(st.out), to_np(o_clean))
+        assert ma <= 1e-2 and rl <= 5e-3, (ma, rl)
+
+
+@pytest.mark.parametrize("factor", [2.0 ** -14, 1.0, 2.0 ** 8])
+def test_fp8_scale_magnitudes(cuda_lib, factor):
+    """Token scales far from 1 (values near f16's smallest normals, or scores 256x
+    larger): the decode kernel alone, given a q_lat that the oracle also uses (the
+    oracle's fp64 absorption rounded to bf16, the boundary's type), tracks the
+    oracle relative to the value magnitude.  The absorption's own bf16 rounding is
+    left out because its score error grows with the score magnitude."""
+    from head_latent_attention_06_b200.step import step_from_workload
+    w = make_workload(_spec("fp8", 128, 1, [700, 64, 3]))
+    w.kv_scale.mul_(factor)
+    inp = oracle.from_workload(w)
+    q_lat = torch.from_numpy(om.absorb_q(inp.q_nope, inp.w_uk)).to(torch.bfloat16)
+    st = step_from_workload(w)
+    st.q_lat.copy_(q_lat.to(st.q_lat.device))
+    st.attend()
+    torch.cuda.synchronize()
+    assert cuda_lib.mla_get_status(st.workspace) == 0
+    qb = q_lat.double().numpy()
+    o_lat, lse = to_np(st.o_lat), to_np(st.lse)
+    amax, rl2 = TOL["fp8"]
+    for b in range(w.B):
+        C = inp.rows(b, inp.visible(b, 0))
+        ref_o, ref_lse = om.latent_attention(qb[b, 0], inp.q_pe[b, 0], C, inp.softmax_scale)
+        ma, rl = errors(o_lat[b, 0] / factor, ref_o / factor)
+        assert ma <= amax and rl <= rl2, (b, ma, rl)
+        assert np.abs(lse[b, 0] - ref_lse).max() <= amax
 
 
 def test_projections_against_oracle(cuda_lib):
