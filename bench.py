@@ -10,9 +10,10 @@ Under torchrun every rank runs its own batch (different seed, same shape): the
 sequences are independent, so ranks exchange nothing on the data path and the
 line reports weak scaling, timed on the device as the max over ranks.
 
-Timing: W untimed warm-up steps, then K steps; each step is bracketed by CUDA
-events on the launching stream and L2 is flushed (a 256 MB write) between steps,
-outside the events.  ``value`` is cache GB/s of the whole step (all ranks);
+Timing: the step is captured once in a CUDA graph (absorb, decode, combine,
+up-projection); W untimed warm-up replays, then K replays, each bracketed by
+CUDA events on the launching stream, with L2 flushed (a 256 MB write) before
+each, outside the events.  The parts are then timed the same way one by one.  ``value`` is cache GB/s of the whole step (all ranks);
 ``roofline`` is the decode kernel's own cache bytes over its event-timed
 duration against the measured HBM copy bandwidth.
 """
@@ -236,35 +237,48 @@ def main(argv=None):
     cache_bytes = w.cache_bytes()
     flops = step_flops(w.lens, w.H, w.s_q)
 
-    def timed_step(ev):
+    # The step and its parts are replayed from CUDA graphs: one host call issues
+    # all launches of a part, so the device never waits on the host and the
+    # events measure device time only.
+    g_step = st.capture()
+    g_absorb = st.capture(st.absorb)
+    g_decode = st.capture(lambda: mla.mla_decode_paged(st.args))
+    g_tail = st.capture(lambda: (mla.mla_combine_splits(st.args), st.up_project()))
+
+    def timed(graph, ev):
+        flush.zero_()
         ev[0].record(stream)
-        st.absorb()
+        graph.replay()
         ev[1].record(stream)
-        mla.mla_decode_paged(st.args)
-        ev[2].record(stream)
-        mla.mla_combine_splits(st.args)
-        st.up_project()
-        ev[3].record(stream)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
-        st.run()
+        g_step.replay()
     torch.cuda.synchronize()
     assert mla.mla_get_status(st.workspace) == 0
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    def new_events():
+        return [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+
+    evs, ev_abs, ev_dec, ev_tail = new_events(), new_events(), new_events(), new_events()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         for k in range(args.steps):
-            flush.zero_()
-            timed_step(evs[k])
+            timed(g_step, evs[k])
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    # the parts one by one (each after an L2 flush), for the kernel rooflines
+    for k in range(args.steps):
+        timed(g_absorb, ev_abs[k])
+        timed(g_decode, ev_dec[k])
+        timed(g_tail, ev_tail[k])
+    torch.cuda.synchronize()
+    assert mla.mla_get_status(st.workspace) == 0
+    ms = lambda ev: [e[0].elapsed_time(e[1]) for e in ev]
+    step_ms, dec_ms, absorb_ms, tail_ms = ms(evs), ms(ev_dec), ms(ev_abs), ms(ev_tail)
     total_ms = reduce_max(sum(step_ms))
     dec_avg_ms = reduce_max(sum(dec_ms) / len(dec_ms))
     ms_per_step = total_ms / args.steps
@@ -290,7 +304,7 @@ def main(argv=None):
         st.q_pe.copy_(h_q_pe, non_blocking=True)
         d_bt.copy_(h_bt, non_blocking=True)
         d_len.copy_(h_len, non_blocking=True)
-        st.run()
+        g_step.replay()
         h_out.copy_(st.out, non_blocking=True)
         if e1 is not None:
             e1.record(stream)
@@ -316,6 +330,8 @@ def main(argv=None):
         "tflops": round(world * (flops + proj_flops(w.n_tok, w.H)) / (ms_per_step * 1e-3) / 1e12, 2),
         "tokens_per_s": round(world * w.n_tok / (ms_per_step * 1e-3), 1),
         "decode_us": round(dec_avg_ms * 1e3, 2),
+        "absorb_us": round(1e3 * sum(absorb_ms) / len(absorb_ms), 2),
+        "combine_up_proj_us": round(1e3 * sum(tail_ms) / len(tail_ms), 2),
         "roofline": {
             "bound": "hbm", "achieved": round(dec_gbs, 1), "peak": hbm, "unit": "GB/s",
             "frac": round(dec_gbs / hbm, 4), "traffic": None,

@@ -34,8 +34,10 @@
 // the even CTA) issuer of the score MMAs, warp 2 (even CTA) issuer of the P.V
 // MMAs, warp 3 idle, warps 4..11 softmax / correction / epilogue, two warps per
 // TMEM lane quadrant, each thread 16 scores of a row half per page.
-// Two S buffers let S(t+2) run on the tensor pipe while the softmax of t+1 runs;
-// each softmax warp signals its own P rows to the P.V issuer.
+// Two S buffers: each softmax warp releases its S buffer as soon as its scores
+// are in registers, so S(t+2) is issued while the softmax of t is still running
+// and the tensor pipe does not wait on it; each softmax warp signals its own P
+// rows to the P.V issuer.
 // P is double-buffered in shared memory, so the softmax of t+1 never waits for
 // P.V of t.  The output rescale is lazy: the reference maximum moves only when
 // the tile maximum exceeds it by more than 2^8, so O in TMEM is rarely touched.
@@ -109,14 +111,17 @@ constexpr int S_READY = Q_TMEM + 1;        // [2]
 constexpr int P_READY = S_READY + 2;      // [2] in the even CTA
 constexpr int O_DONE = P_READY + 2;       // [2]
 constexpr int DRAIN = O_DONE + 2;        // [2] one per MMA-issuing warp
-constexpr int RAW_S = DRAIN + 2;          // [kSStages] fp8: raw bytes of a score stage landed
+constexpr int S_FREE = DRAIN + 2;         // [2] in the even CTA: the softmax has read S buffer sb
+constexpr int RAW_S = S_FREE + 2;         // [kSStages] fp8: raw bytes of a score stage landed
 constexpr int RAW_V = RAW_S + kSStages;   // [kVStages] fp8: raw bytes of a value stage landed
 constexpr int SC_FULL = RAW_V + kVStages; // [kScRing]  fp8: token scales of a tile landed
 constexpr int NBARS = SC_FULL + kScRing;
 // A scale entry is reloaded for tile u + kScRing only after the score stage of
-// tile u + kScRing - kSStages was consumed, which needed the softmax of tile
-// u + kScRing - kSStages - 2 to be done; the softmax of tile u must be among them.
-static_assert(kScRing >= kSStages + 2 + 1, "scale ring too short");
+// tile u + kScRing - kSStages was consumed; that score MMA waited for every
+// softmax warp to release the S buffer of tile u + kScRing - kSStages - 2, which
+// each does only after finishing tile u + kScRing - kSStages - 3.  Tile u must
+// be among the finished ones.
+static_assert(kScRing >= kSStages + 3, "scale ring too short");
 constexpr int kSoftmaxWarps = 8;          // warps 4..11: two per TMEM lane quadrant
 constexpr int kPrefetchTiles = MLA_TC_PREFETCH;      // L2 prefetch distance of the cache stream
 constexpr uint32_t kMiscOff = kBarOff + 8 * NBARS;
@@ -245,6 +250,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
     for (int i = 0; i < 2; ++i) {
       mbar_init(own_bar(S_READY + i), 1);
       mbar_init(own_bar(P_READY + i), 2 * kSoftmaxWarps);
+      mbar_init(own_bar(S_FREE + i), 2 * kSoftmaxWarps);
       mbar_init(own_bar(O_DONE + i), 1);
     }
     mbar_init(own_bar(DRAIN), 1);
@@ -315,10 +321,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
           }
           __syncwarp();
         } else {
+          // one box: (64 values, 32 rows, 9 chunks) lands chunk-major, 9 x 4 KB
           const uint32_t fb = lead_bar(S_FULL + st);
           if (r == 0) mbar_arrive_expect_tx_local_elect(own_bar(S_FULL + st), 2 * kSStage);
-          for (int c = 0; c < 9; ++c)
-            tma_load_2d_pair_elect(dst + c * kChunkS, &tm_ks, fb, 64 * c, pg * kPage + 32 * (int)r);
+          tma_load_3d_pair_elect(dst, &tm_ks, fb, 0, pg * kPage + 32 * (int)r, 0);
         }
         if (u + kPrefetchTiles < n) prefetch(u + kPrefetchTiles);
         return true;
@@ -334,31 +340,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
           // map views a row as 288 two-byte units) into the back half of the slot
           if (lane == 0) {
             mbar_arrive_expect_tx_local(own_bar(RAW_V + st), kVStage / 2);
-            for (int seg = 0; seg < 2; ++seg)
-              tma_load_2d_cta(dst + kVStage / 2 + seg * (kVStage / 4), &tm_kv, own_bar(RAW_V + st),
-                              64 * (int)r + 128 * seg, pg * kPage);
+            tma_load_3d_cta(dst + kVStage / 2, &tm_kv, own_bar(RAW_V + st), 64 * (int)r, pg * kPage, 0);
           }
           __syncwarp();
         } else {
           const int nvalid = j_end - (t0 + u) * kPage;  // cached rows of this page inside the sequence
           if (nvalid >= kPage) {
+            // one box: (64 values, 64 rows, chunks 2r and 2r+1, groups 0 and 1): latent
+            // chunks {2r, 2r+1, 4+2r, 5+2r} of the page, 4 x 8 KB
             const uint32_t fb = lead_bar(V_FULL + st);
             if (r == 0) mbar_arrive_expect_tx_local_elect(own_bar(V_FULL + st), 2 * kVStage);
             else if (lane == 0) mbar_arrive_remote_relaxed(fb);
-            for (int j = 0; j < 4; ++j) {
-              const int lc = 4 * (j >> 1) + 2 * (int)r + (j & 1);  // latent chunk: halves {2r, 2r+1}, {4+2r, 5+2r}
-              tma_load_2d_pair_elect(dst + j * kChunkV, &tm_kv, fb, 64 * lc, pg * kPage);
-            }
+            tma_load_4d_pair_elect(dst, &tm_kv, fb, 0, pg * kPage, 2 * (int)r, 0);
           } else {
             // The last page of the sequence: P is 0 past the end, but 0 * NaN is
             // not, so whatever those rows hold is replaced by zeros before the MMA.
             // The stage lands on this CTA's own barrier (once per work unit).
             if (lane == 0) {
               mbar_arrive_expect_tx_local(own_bar(RAW_V + st), kVStage);
-              for (int j = 0; j < 4; ++j) {
-                const int lc = 4 * (j >> 1) + 2 * (int)r + (j & 1);
-                tma_load_2d_cta(dst + j * kChunkV, &tm_kv, own_bar(RAW_V + st), 64 * lc, pg * kPage);
-              }
+              tma_load_4d_cta(dst, &tm_kv, own_bar(RAW_V + st), 0, pg * kPage, 2 * (int)r, 0);
             }
             __syncwarp();
             if (!mbar_wait_converged(own_bar(RAW_V + st), 0, abort_flag, p.status, kWaitLimitNs)) return false;
@@ -410,8 +410,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
              mbar_wait_converged(own_bar(Q_TMEM), 0, abort_flag, p.status, kWaitLimitNs);
         for (int u = 0; ok && u < n; ++u) {
           const int st = u % kSStages, sb = u & 1;
-          // S buffer sb was last read by the softmax of tile u-2
-          if (u >= 2 && !mbar_wait_converged(own_bar(P_READY + sb), ((u - 2) >> 1) & 1, abort_flag, p.status,
+          // S buffer sb was last read by the softmax of tile u-2 (released as soon as
+          // its scores are in registers)
+          if (u >= 2 && !mbar_wait_converged(own_bar(S_FREE + sb), ((u - 2) >> 1) & 1, abort_flag, p.status,
                                              kWaitLimitNs))
             break;
           if (!mbar_wait_converged(own_bar(S_FULL + st), (u / kSStages) & 1, abort_flag, p.status, kWaitLimitNs))
@@ -614,6 +615,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
       uint32_t sv[16];
       tmem_ld16(tl + kTmemS + 32u * sb + 16u * ch, sv);
       tmem_wait_ld();
+      // the scores are in registers: S buffer sb may take S(t+2)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(lead_bar(S_FREE + sb));
       const int j0 = (t0 + t) * kPage + 32 * half + 16 * ch;
       const int nv = max(0, min(16, lim - j0));
       // fp8: token scales of these 16 columns (0 where masked, so that nothing a
@@ -790,12 +795,23 @@ cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t strea
       !tma_map_3d(&tm_qpe, a->q_pe, kDr, a->H, n_tok, kDr * 2, (uint64_t)a->H * kDr * 2, 64, 64, 1))
     return cudaErrorInvalidValue;
   if (FP8) {
-    // the e4m3 rows (576 bytes) viewed as 288 two-byte units: boxes of 128 bytes x 64 rows
-    if (!tma_map_2d(&tm_kv, a->kv_cache, kRow / 2, rows_kv, kRow, 64, 64)) return cudaErrorInvalidValue;
+    // the e4m3 rows (576 bytes) viewed as two-byte units: (128 units, rows, 2
+    // segments 256 bytes apart); a box of 64 units at unit 64r brings the bytes
+    // 128r .. 128r+127 and 256+128r .. 256+128r+127 of each row
+    const uint64_t dims[3] = {128, rows_kv, 2}, strides[2] = {kRow, 256};
+    const uint32_t box[3] = {64, 64, 2};
+    if (!tma_map_nd(&tm_kv, a->kv_cache, 3, dims, strides, box)) return cudaErrorInvalidValue;
     tm_ks = tm_kv;  // unused: the score operand's raw rows come by a plain bulk copy
-  } else if (!tma_map_2d(&tm_ks, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 32) ||
-             !tma_map_2d(&tm_kv, a->kv_cache, kRow, rows_kv, kRow * 2, 64, 64)) {
-    return cudaErrorInvalidValue;
+  } else {
+    // score operand: (64 values, rows, 9 chunks 128 bytes apart), one box per stage;
+    // value operand: (64 values, rows, 4 chunks 128 bytes apart, 2 groups 512 bytes
+    // apart), one box of 2 x 2 chunks per stage
+    const uint64_t dks[3] = {64, rows_kv, 9}, sks[2] = {kRow * 2, 128};
+    const uint32_t bks[3] = {64, 32, 9};
+    const uint64_t dkv[4] = {64, rows_kv, 4, 2}, skv[3] = {kRow * 2, 128, 512};
+    const uint32_t bkv[4] = {64, 64, 2, 2};
+    if (!tma_map_nd(&tm_ks, a->kv_cache, 3, dks, sks, bks) || !tma_map_nd(&tm_kv, a->kv_cache, 4, dkv, skv, bkv))
+      return cudaErrorInvalidValue;
   }
   TcParams p;
   p.q_lat = static_cast<const __nv_bfloat16*>(a->q_lat);

@@ -172,6 +172,26 @@ MLA_DEVI void tma_load_2d_pair_elect(uint32_t dst, const void* tmap, uint32_t mb
       "l"(tmap), "r"(mbar_cluster), "r"(x), "r"(y)
       : "memory");
 }
+MLA_DEVI void tma_load_3d_pair_elect(uint32_t dst, const void* tmap, uint32_t mbar_cluster, int32_t x,
+                                     int32_t y, int32_t z) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 rx;\n\t"
+      "elect.sync rx|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];\n\t}" ::"r"(dst),
+      "l"(tmap), "r"(mbar_cluster), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+MLA_DEVI void tma_load_4d_pair_elect(uint32_t dst, const void* tmap, uint32_t mbar_cluster, int32_t x,
+                                     int32_t y, int32_t z, int32_t w) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 rx;\n\t"
+      "elect.sync rx|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];\n\t}" ::"r"(dst),
+      "l"(tmap), "r"(mbar_cluster), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
 // Arrive with an expected byte count on a barrier of this CTA (CTA-scope
 // release: the bytes themselves are counted by the TMA engine).
 MLA_DEVI void mbar_arrive_expect_tx_local_elect(uint32_t addr, uint32_t tx) {
@@ -190,6 +210,22 @@ MLA_DEVI void tma_load_2d_cta(uint32_t dst, const void* tmap, uint32_t mbar, int
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(tmap), "r"(mbar), "r"(x), "r"(y)
+      : "memory");
+}
+
+MLA_DEVI void tma_load_3d_cta(uint32_t dst, const void* tmap, uint32_t mbar, int32_t x, int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(tmap), "r"(mbar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+MLA_DEVI void tma_load_4d_cta(uint32_t dst, const void* tmap, uint32_t mbar, int32_t x, int32_t y, int32_t z,
+                              int32_t w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(tmap), "r"(mbar), "r"(x), "r"(y), "r"(z), "r"(w)
       : "memory");
 }
 

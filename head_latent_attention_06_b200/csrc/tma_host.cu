@@ -25,13 +25,15 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 struct MapKey {
   const void* ptr;
   uint32_t rank;
-  uint64_t dims[3], strides[2];
-  uint32_t box[3];
+  uint64_t dims[5], strides[4];
+  uint32_t box[5];
   bool operator==(const MapKey& o) const {
     if (ptr != o.ptr || rank != o.rank) return false;
-    for (int i = 0; i < 3; ++i)
+    for (int i = 0; i < 5; ++i)
       if (dims[i] != o.dims[i] || box[i] != o.box[i]) return false;
-    return strides[0] == o.strides[0] && strides[1] == o.strides[1];
+    for (int i = 0; i < 4; ++i)
+      if (strides[i] != o.strides[i]) return false;
+    return true;
   }
 };
 
@@ -52,10 +54,14 @@ bool encode(CUtensorMap* m, const MapKey& k) {
   }
   auto enc = get_encode();
   if (!enc) return false;
-  cuuint64_t dims[3] = {k.dims[0], k.dims[1], k.dims[2]};
-  cuuint64_t strides[2] = {k.strides[0], k.strides[1]};
-  cuuint32_t box[3] = {k.box[0], k.box[1], k.box[2]};
-  cuuint32_t estr[3] = {1, 1, 1};
+  cuuint64_t dims[5], strides[4];
+  cuuint32_t box[5], estr[5];
+  for (int i = 0; i < 5; ++i) {
+    dims[i] = k.dims[i];
+    box[i] = k.box[i];
+    estr[i] = 1;
+  }
+  for (int i = 0; i < 4; ++i) strides[i] = k.strides[i];
   CUresult res = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k.rank, const_cast<void*>(k.ptr), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -71,13 +77,25 @@ bool encode(CUtensorMap* m, const MapKey& k) {
 
 bool tma_map_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t row_bytes,
                 uint32_t box_cols, uint32_t box_rows) {
-  MapKey k{ptr, 2, {cols, rows, 1}, {row_bytes, 0}, {box_cols, box_rows, 1}};
+  MapKey k{ptr, 2, {cols, rows, 1, 1, 1}, {row_bytes, 0, 0, 0}, {box_cols, box_rows, 1, 1, 1}};
   return encode(m, k);
 }
 
 bool tma_map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
                 uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
-  MapKey k{ptr, 3, {d0, d1, d2}, {s1, s2}, {b0, b1, b2}};
+  MapKey k{ptr, 3, {d0, d1, d2, 1, 1}, {s1, s2, 0, 0}, {b0, b1, b2, 1, 1}};
+  return encode(m, k);
+}
+
+bool tma_map_nd(CUtensorMap* m, const void* ptr, uint32_t rank, const uint64_t* dims, const uint64_t* strides,
+                const uint32_t* box) {
+  if (rank < 1 || rank > 5) return false;
+  MapKey k{ptr, rank, {1, 1, 1, 1, 1}, {0, 0, 0, 0}, {1, 1, 1, 1, 1}};
+  for (uint32_t i = 0; i < rank; ++i) {
+    k.dims[i] = dims[i];
+    k.box[i] = box[i];
+    if (i > 0) k.strides[i - 1] = strides[i - 1];
+  }
   return encode(m, k);
 }
 

@@ -17,4 +17,12 @@ bool tma_map_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, u
 bool tma_map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
                 uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2);
 
+// Map of rank 1..5: dims[i] values along dimension i (dimension 0 contiguous),
+// strides[i] the byte stride of dimension i + 1 (any order, multiples of 16),
+// boxes of box[i] values.  The box lands in shared memory with dimension 0
+// fastest, so a stride smaller than the row pitch can order several chunks of a
+// row one after another.
+bool tma_map_nd(CUtensorMap* m, const void* ptr, uint32_t rank, const uint64_t* dims, const uint64_t* strides,
+                const uint32_t* box);
+
 }  // namespace mla

@@ -54,6 +54,19 @@ class DecodeStep:
         self.up_project(stream)
         return self.out
 
+    def capture(self, fn=None):
+        """Records ``fn`` (default: the whole step) into a CUDA graph and returns
+        it; ``graph.replay()`` then issues all of its launches with one host call.
+        The step allocates nothing, so the graph stays valid while the buffers
+        (and the arguments captured in it) are unchanged."""
+        fn = fn or self.run
+        fn()                       # first call outside capture: one-time host setup
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        return g
+
 
 def step_from_workload(w, device="cuda", num_splits=0):
     """Copy a ``mla_inputs.Workload`` to the device and build its ``DecodeStep``."""
