@@ -12,8 +12,9 @@ line reports weak scaling, timed on the device as the max over ranks.
 
 Timing: the step is captured once in a CUDA graph (absorb, decode, combine,
 up-projection); W untimed warm-up replays, then K replays, each bracketed by
-CUDA events on the launching stream, with L2 flushed (a 256 MB write) before
-each, outside the events.  The parts are then timed the same way one by one.  ``value`` is cache GB/s of the whole step (all ranks);
+CUDA events on the launching stream, with L2 flushed (a 256 MB write, then
+a 256 MB read that leaves no dirty line behind) before each, outside the events.  The parts are then timed the same way one by one.
+``value`` is cache GB/s of the whole step (all ranks);
 ``roofline`` is the decode kernel's own cache bytes over its event-timed
 duration against the measured HBM copy bandwidth.
 """
@@ -191,7 +192,7 @@ def _config_dict(name, w, splits=None):
     s = preset(name)
     d = {"workload": f"{name}: {s.note}", "B": s.B, "H": s.H, "s_q": s.s_q,
          "kv_cache": s.kv_dtype, "page_size": 64, "d_c": 512, "d_r": 64,
-         "causal": s.causal, "l2": "flushed between timed steps (256 MB write)"}
+         "causal": s.causal, "l2": "flushed between timed steps (256 MB write, then 256 MB read)"}
     if w is not None:
         d["cached_tokens"] = sum(w.lens)
     if splits is not None:
@@ -233,7 +234,16 @@ def main(argv=None):
     st = step_from_workload(w, num_splits=args.splits)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    # L2 flush: write a 256 MB buffer (twice the 126 MB L2), then read another
+    # one.  The write evicts everything the step left in L2; the read then
+    # replaces the written (dirty) lines with clean ones, so that the timed step
+    # does not pay for writing back the flush buffer itself.
+    flush_w = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    flush_r = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+
+    def flush_l2():
+        flush_w.zero_()
+        torch.sum(flush_r)
     cache_bytes = w.cache_bytes()
     flops = step_flops(w.lens, w.H, w.s_q)
 
@@ -246,13 +256,13 @@ def main(argv=None):
     g_tail = st.capture(lambda: (mla.mla_combine_splits(st.args), st.up_project()))
 
     def timed(graph, ev):
-        flush.zero_()
+        flush_l2()
         ev[0].record(stream)
         graph.replay()
         ev[1].record(stream)
 
     for _ in range(max(3, args.warmup)):
-        flush.zero_()
+        flush_l2()
         g_step.replay()
     torch.cuda.synchronize()
     assert mla.mla_get_status(st.workspace) == 0
@@ -296,7 +306,7 @@ def main(argv=None):
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     for k in range(args.steps + 2):
-        flush.zero_()
+        flush_l2()
         e0, e1 = e2e_ev[k - 2] if k >= 2 else (None, None)
         if e0 is not None:
             e0.record(stream)
