@@ -31,9 +31,10 @@
 // for the first half of every N tile, lane 64 + l the same row for the second.
 //
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM allocator and (in
-// the even CTA) issuer of the score MMAs, warp 2 (even CTA) issuer of the P.V
-// MMAs, warp 3 idle, warps 4..11 softmax / correction / epilogue, two warps per
-// TMEM lane quadrant, each thread 16 scores of a row half per page.
+// the even CTA) issuer of the score MMAs (bf16: of even pages, warp 3 of odd
+// ones), warp 2 (even CTA) issuer of the P.V MMAs, warps 4..11 softmax /
+// correction / epilogue, two warps per TMEM lane quadrant, each thread 16
+// scores of a row half per page.
 // Two S buffers: each softmax warp releases its S buffer as soon as its scores
 // are in registers, so S(t+2) is issued while the softmax of t is still running
 // and the tensor pipe does not wait on it; each softmax warp signals its own P
@@ -110,8 +111,8 @@ constexpr int Q_TMEM = Q_FULL + 1;         // TMEM part of Q written by the soft
 constexpr int S_READY = Q_TMEM + 1;        // [2]
 constexpr int P_READY = S_READY + 2;      // [2] in the even CTA
 constexpr int O_DONE = P_READY + 2;       // [2]
-constexpr int DRAIN = O_DONE + 2;        // [2] one per MMA-issuing warp
-constexpr int S_FREE = DRAIN + 2;         // [2] in the even CTA: the softmax has read S buffer sb
+constexpr int DRAIN = O_DONE + 2;        // [3] one per MMA-issuing warp
+constexpr int S_FREE = DRAIN + 3;         // [2] in the even CTA: the softmax has read S buffer sb
 constexpr int RAW_S = S_FREE + 2;         // [kSStages] fp8: raw bytes of a score stage landed
 constexpr int RAW_V = RAW_S + kSStages;   // [kVStages] fp8: raw bytes of a value stage landed
 constexpr int SC_FULL = RAW_V + kVStages; // [kScRing]  fp8: token scales of a tile landed
@@ -253,8 +254,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
       mbar_init(own_bar(S_FREE + i), 2 * kSoftmaxWarps);
       mbar_init(own_bar(O_DONE + i), 1);
     }
-    mbar_init(own_bar(DRAIN), 1);
-    mbar_init(own_bar(DRAIN + 1), 1);
+    for (int i = 0; i < 3; ++i) mbar_init(own_bar(DRAIN + i), 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -394,8 +394,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
         if (ok) ok = load_v(u);
       }
     }
-  } else if (warp == 1 || warp == 2) {
-    // ============ MMA issuers (even CTA): warp 1 scores, warp 2 P.V ============
+  } else if (warp == 1 || warp == 2 || (!FP8 && warp == 3)) {
+    // ==== MMA issuers (even CTA): warp 1 (bf16: and 3) scores, warp 2 P.V ====
     // The two streams touch disjoint TMEM (S buffers / O) and shared memory
     // (Q and the S ring / P and the V ring), so they are issued independently.
     if (r == 0 && n > 0) {
@@ -404,11 +404,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
       const uint64_t dv = desc_sw128(sa + kVOff, kChunkV, 1024);
       const uint64_t dp = desc_sw128(sa + kPOff, 16, 1024);
       bool ok = true;
-      if (warp == 1) {
+      if (warp != 2) {
         // fp8: the softmax warps write all of Q (TMEM and shared memory parts)
         ok = (FP8 || mbar_wait_converged(own_bar(Q_FULL), 0, abort_flag, p.status, kWaitLimitNs)) &&
              mbar_wait_converged(own_bar(Q_TMEM), 0, abort_flag, p.status, kWaitLimitNs);
-        for (int u = 0; ok && u < n; ++u) {
+        // bf16: warp 1 issues the even pages, warp 3 the odd ones.  Issuing 36 MMAs
+        // takes the issue slots of the warp's SM sub-partition, whose softmax warps
+        // then fall behind; two issuers halve that.  Each page's waits (S buffer
+        // free, then stage full) imply that the stage's previous phase has
+        // completed, so that parity waits stay exact with two issuers.  (fp8: the
+        // converter warp on warp 3's sub-partition needs those slots; warp 1 alone.)
+        constexpr int kStep = FP8 ? 1 : 2;
+        for (int u = warp == 3 ? 1 : 0; ok && u < n; u += kStep) {
           const int st = u % kSStages, sb = u & 1;
           // S buffer sb was last read by the softmax of tile u-2 (released as soon as
           // its scores are in registers)
@@ -463,7 +470,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
         }
       }
       // every MMA this warp issued has completed before TMEM is released
-      const int db = DRAIN + (warp == 2 ? 1 : 0);
+      const int db = DRAIN + warp - 1;
       commit_pair_mc_elect(own_bar(db), 0x1);
       int dummy = 0;
       mbar_wait_converged(own_bar(db), 0, &dummy, p.status, kWaitLimitNs);
@@ -567,19 +574,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
     if (n > 0) {
       const uint4* qsrc =
           reinterpret_cast<const uint4*>(p.q_lat + (((size_t)b * p.s_q + g) * p.H + (row_ok ? head : 0)) * kDc);
-      constexpr int kPerWarp = (kQTmemChunks + 1) / 2;
+      // the thread's chunks ch*kPerWarp .. in batches whose loads are all issued
+      // before the first TMEM store, so that the batch costs one memory latency
+      static_assert(kQTmemChunks % 2 == 0, "Q chunks split evenly between the column halves");
+      constexpr int kPerWarp = kQTmemChunks / 2;
+      constexpr int kBatch = FP8 ? 1 : kPerWarp;  // fp8 threads have fewer registers to spare
 #pragma unroll 1
-      for (int c = ch * kPerWarp; c < kQTmemChunks && c < (ch + 1) * kPerWarp; ++c) {
-        uint32_t qv[32];
+      for (int c0 = ch * kPerWarp; c0 < (ch + 1) * kPerWarp; c0 += kBatch) {
+        uint32_t qv[kBatch][32];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint4 v = row_ok ? __ldg(qsrc + c * 8 + k) : make_uint4(0u, 0u, 0u, 0u);
-          qv[4 * k] = FP8 ? bf16x2_to_f16x2(v.x) : v.x;
-          qv[4 * k + 1] = FP8 ? bf16x2_to_f16x2(v.y) : v.y;
-          qv[4 * k + 2] = FP8 ? bf16x2_to_f16x2(v.z) : v.z;
-          qv[4 * k + 3] = FP8 ? bf16x2_to_f16x2(v.w) : v.w;
-        }
-        tmem_st32(tl + kTmemQ + 32u * c, qv);
+        for (int i = 0; i < kBatch; ++i)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint4 v = row_ok ? __ldg(qsrc + (c0 + i) * 8 + k) : make_uint4(0u, 0u, 0u, 0u);
+            qv[i][4 * k] = FP8 ? bf16x2_to_f16x2(v.x) : v.x;
+            qv[i][4 * k + 1] = FP8 ? bf16x2_to_f16x2(v.y) : v.y;
+            qv[i][4 * k + 2] = FP8 ? bf16x2_to_f16x2(v.z) : v.z;
+            qv[i][4 * k + 3] = FP8 ? bf16x2_to_f16x2(v.w) : v.w;
+          }
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) tmem_st32(tl + kTmemQ + 32u * (c0 + i), qv[i]);
       }
       if constexpr (FP8) {
         // the shared-memory chunks of Q as f16 (128-byte swizzled rows, the layout
