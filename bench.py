@@ -37,6 +37,24 @@ METRIC = "MLA decode cache GB/s, TFLOP/s & % of B200 roofline; tokens/s per step
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes (read + write) of one decode launch from an ncu capture, recorded
+# with the sha256 prefix of the kernel source it was taken on: reported as the
+# roofline's ``traffic`` only while that source is unchanged.
+# (profiles/decode_tc_v3_bf16.md)
+MEASURED_TRAFFIC = {"v3": (311591424 + 4218368, "14a47a3b188a0421")}
+
+
+def decode_traffic(config: str):
+    import hashlib
+    entry = MEASURED_TRAFFIC.get(config)
+    if entry is None:
+        return None
+    src = os.path.join(ROOT, "head_latent_attention_06_b200", "csrc", "decode_tc.cu")
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    return entry[0] if digest == entry[1] else None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -344,7 +362,7 @@ def main(argv=None):
         "combine_up_proj_us": round(1e3 * sum(tail_ms) / len(tail_ms), 2),
         "roofline": {
             "bound": "hbm", "achieved": round(dec_gbs, 1), "peak": hbm, "unit": "GB/s",
-            "frac": round(dec_gbs / hbm, 4), "traffic": None,
+            "frac": round(dec_gbs / hbm, 4), "traffic": decode_traffic(args.config),
             "peak_kind": f"{peak_kind} HBM copy bandwidth",
             "kernel": "mla_decode_paged",
             "tensor": {"achieved_tflops": round(dec_tflops, 1),
