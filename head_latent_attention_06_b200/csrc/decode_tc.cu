@@ -83,7 +83,7 @@ constexpr uint32_t kChunkQ = 64 * 128;              // 64 rows x 64 bf16
 #define MLA_TC_S_STAGES 3
 #endif
 #ifndef MLA_TC_PREFETCH
-#define MLA_TC_PREFETCH 4
+#define MLA_TC_PREFETCH 2
 #endif
 constexpr int kQTmemChunks = MLA_TC_Q_TMEM_CHUNKS;  // Q chunks 0..5 (latent 0..383) live in TMEM
 constexpr int kQSmemChunks = 9 - kQTmemChunks;      // chunks 6..8 (latent 384..511, q_pe) in smem
@@ -116,7 +116,9 @@ constexpr int S_FREE = DRAIN + 3;         // [2] in the even CTA: the softmax ha
 constexpr int RAW_S = S_FREE + 2;         // [kSStages] fp8: raw bytes of a score stage landed
 constexpr int RAW_V = RAW_S + kSStages;   // [kVStages] fp8: raw bytes of a value stage landed
 constexpr int SC_FULL = RAW_V + kVStages; // [kScRing]  fp8: token scales of a tile landed
-constexpr int NBARS = SC_FULL + kScRing;
+constexpr int Q_STAGE = SC_FULL + kScRing; // bf16: Q chunks 0..5 landed in the value ring (this CTA)
+constexpr int Q_MOVED = Q_STAGE + 1;        // bf16: the softmax warps have moved them into TMEM
+constexpr int NBARS = Q_MOVED + 1;
 // A scale entry is reloaded for tile u + kScRing only after the score stage of
 // tile u + kScRing - kSStages was consumed; that score MMA waited for every
 // softmax warp to release the S buffer of tile u + kScRing - kSStages - 2, which
@@ -214,21 +216,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
   auto own_bar = [&](int i) -> uint32_t { return sa + kBarOff + 8u * i; };
   auto lead_bar = [&](int i) -> uint32_t { return mapa(sa + kBarOff + 8u * i, 0); };
 
-  // ---- the work unit: tiles [t0, t1) of sequence b, query g
-  int L = p.seq_lens[b];
-  const bool bad_len = L < 0 || L > p.max_pages * kPage;
-  if (bad_len) L = 0;
-  const int n_tiles = (L + kPage - 1) / kPage;
-  const int per = (n_tiles + p.splits - 1) / p.splits;
-  const int t0 = min(n_tiles, split * per);
-  const int t1 = min(n_tiles, t0 + per);
-  const int n = t1 - t0;
-  const int j_end = min(L, t1 * kPage);
-  const int vis = p.causal ? L - p.s_q + g + 1 : L;
+  // The length and (for the first split, which starts at page 0) the producer's
+  // first 32 block-table entries are requested here and used after the barrier
+  // set-up, TMEM allocation and cluster sync, so that their latencies overlap.
+  const int L_in = p.seq_lens[b];
   const int32_t* bt = p.block_table + (size_t)b * p.max_pages;
+  int bt_first = 0;
+  if (warp == 0 && split == 0 && lane < p.max_pages) bt_first = __ldg(bt + lane);
 
   if (threadIdx.x == 0) {
-    if (bad_len && r == 0 && g == 0 && split == 0) set_status(p.status, MLA_ERR_BAD_SEQ_LEN);
     *abort_flag = 0;
     // bf16: a full score stage is the even CTA's expect_tx plus both CTAs' TMA
     // bytes, a full value stage that and the odd CTA's arrival (a last, partial
@@ -248,6 +244,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
     for (int i = 0; i < kScRing; ++i) mbar_init(own_bar(SC_FULL + i), 1);
     mbar_init(own_bar(Q_TMEM), 2 * kSoftmaxWarps);
     mbar_init(own_bar(Q_FULL), 1);
+    mbar_init(own_bar(Q_STAGE), 1);
+    mbar_init(own_bar(Q_MOVED), kSoftmaxWarps);
     for (int i = 0; i < 2; ++i) {
       mbar_init(own_bar(S_READY + i), 1);
       mbar_init(own_bar(P_READY + i), 2 * kSoftmaxWarps);
@@ -268,25 +266,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
   const uint32_t tmem = *tmem_slot;
   pdl_trigger();
 
+  // ---- the work unit: tiles [t0, t1) of sequence b, query g
+  const bool bad_len = L_in < 0 || L_in > p.max_pages * kPage;
+  const int L = bad_len ? 0 : L_in;
+  if (bad_len && threadIdx.x == 0 && r == 0 && g == 0 && split == 0) set_status(p.status, MLA_ERR_BAD_SEQ_LEN);
+  const int n_tiles = (L + kPage - 1) / kPage;
+  const int per = (n_tiles + p.splits - 1) / p.splits;
+  const int t0 = min(n_tiles, split * per);
+  const int t1 = min(n_tiles, t0 + per);
+  const int n = t1 - t0;
+  const int j_end = min(L, t1 * kPage);
+  const int vis = p.causal ? L - p.s_q + g + 1 : L;
+
   if (warp == 0) {
     // =========================== TMA producer ===========================
     // Ring order = MMA order: S(0), S(1), V(0), S(2), V(1), ... where S(u) is the
     // CTA's 32 tokens x 576 of page u (9 slots) and V(u) the page's 64 tokens x
     // the CTA's latent columns of both P.V halves (8 slots of 16 tokens x 128).
     if (n > 0) {
-      if (lane == 0) {
-        prefetch_tmap(&tm_q);
-        prefetch_tmap(&tm_qpe);
-        prefetch_tmap(&tm_ks);
-        prefetch_tmap(&tm_kv);
-      }
       // physical pages, fetched 32 at a time by the whole warp
       int blk_s = -1, pg_s = 0, blk_v = -1, pg_v = 0, blk_p = -1, pg_p = 0;
       auto page_of = [&](int u, int& blk, int& pg) -> int {
         if ((u >> 5) != blk) {
           blk = u >> 5;
           const int idx = t0 + (blk << 5) + lane;
-          int v = idx < t1 ? bt[idx] : 0;
+          int v = idx < t1 ? (blk == 0 && split == 0 ? bt_first : bt[idx]) : 0;
           if (v < 0 || v >= p.num_pages) {
             if (idx < t1) set_status(p.status, MLA_ERR_BAD_BLOCK_TABLE);
             v = 0;
@@ -301,7 +305,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
         const int pg = page_of(u, blk_p, pg_p);
         if (lane == 0) prefetch_l2_bulk(p.kv + ((size_t)pg * kPage + 32 * r) * kRow * kElem, 32 * kRow * kElem);
       };
-      for (int u = 0; u < n && u < kPrefetchTiles; ++u) prefetch(u);
       auto load_s = [&](int u) -> bool {
         const int st = u % kSStages;
         const uint32_t ph = ((u / kSStages) & 1) ^ 1;
@@ -377,20 +380,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
       };
       // The cache, block table and lengths are not written by the kernel this one
       // may overlap with (the query absorption); q_lat is, so Q waits for it.
+      // page 0's score stage first, then the L2 prefetch of the next pages and Q
       bool ok = load_s(0);
+      for (int u = 1; u < n && u < kPrefetchTiles; ++u) prefetch(u);
       pdl_wait();
       if (!FP8 && lane == 0) {
-        // 3-D maps (values, heads, query tokens): heads >= H come in as zeros
+        // 3-D maps (values, heads, query tokens): heads >= H come in as zeros.
+        // Chunks 6.. (the MMA's shared-memory A operand) into the Q region; chunks
+        // 0..5 (the TMEM part) staged in the value ring, which V(0) may only
+        // overwrite once the softmax warps have moved them into TMEM.
         const int qtok = b * p.s_q + g, h0 = 64 * (int)r;
         const uint32_t qb = lead_bar(Q_FULL);
         if (r == 0) mbar_arrive_expect_tx_local(own_bar(Q_FULL), 2 * kQBytes);
         for (int c = kQTmemChunks; c < 8; ++c)
           tma_load_3d_pair(sa + kQOff + (c - kQTmemChunks) * kChunkQ, &tm_q, qb, 64 * c, h0, qtok);
         tma_load_3d_pair(sa + kQOff + (8 - kQTmemChunks) * kChunkQ, &tm_qpe, qb, 0, h0, qtok);
+        mbar_arrive_expect_tx_local(own_bar(Q_STAGE), kQTmemChunks * kChunkQ);
+        for (int c = 0; c < kQTmemChunks; ++c)
+          tma_load_3d_cta(sa + kVOff + c * kChunkQ, &tm_q, own_bar(Q_STAGE), 64 * c, h0, qtok);
       }
       __syncwarp();
       for (int u = 0; ok && u < n; ++u) {
         if (u + 1 < n) ok = load_s(u + 1);
+        if (!FP8 && u == 0 && ok)
+          ok = mbar_wait_converged(own_bar(Q_MOVED), 0, abort_flag, p.status, kWaitLimitNs);
         if (ok) ok = load_v(u);
       }
     }
@@ -574,13 +587,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
     if (n > 0) {
       const uint4* qsrc =
           reinterpret_cast<const uint4*>(p.q_lat + (((size_t)b * p.s_q + g) * p.H + (row_ok ? head : 0)) * kDc);
-      // the thread's chunks ch*kPerWarp .. in batches whose loads are all issued
-      // before the first TMEM store, so that the batch costs one memory latency
       static_assert(kQTmemChunks % 2 == 0, "Q chunks split evenly between the column halves");
       constexpr int kPerWarp = kQTmemChunks / 2;
-      constexpr int kBatch = FP8 ? 1 : kPerWarp;  // fp8 threads have fewer registers to spare
+      if constexpr (!FP8) {
+        // bf16: the chunks were staged by TMA (128-byte swizzled rows of 64 heads);
+        // read this row's, store them into TMEM, then free the staging area
+        mbar_wait(own_bar(Q_STAGE), 0, abort_flag, p.status, kWaitLimitNs);
+#pragma unroll
+        for (int i = 0; i < kPerWarp; ++i) {
+          const int c = ch * kPerWarp + i;
+          uint32_t qv[32];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint4 v = lds128(sa + kVOff + c * kChunkQ + m * 128 + ((k ^ (m & 7)) << 4));
+            qv[4 * k] = v.x;
+            qv[4 * k + 1] = v.y;
+            qv[4 * k + 2] = v.z;
+            qv[4 * k + 3] = v.w;
+          }
+          tmem_st32(tl + kTmemQ + 32u * c, qv);
+        }
+      }
+      // fp8: from global memory, rounded to f16 on the way
+      constexpr int kBatch = 1;
 #pragma unroll 1
-      for (int c0 = ch * kPerWarp; c0 < (ch + 1) * kPerWarp; c0 += kBatch) {
+      for (int c0 = ch * kPerWarp; FP8 && c0 < (ch + 1) * kPerWarp; c0 += kBatch) {
         uint32_t qv[kBatch][32];
 #pragma unroll
         for (int i = 0; i < kBatch; ++i)
@@ -616,7 +647,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(lead_bar(Q_TMEM));
+      if (lane == 0) {
+        mbar_arrive_remote(lead_bar(Q_TMEM));
+        if (!FP8) mbar_arrive_remote(own_bar(Q_MOVED));
+      }
     }
     float m_used = -CUDART_INF_F, l = 0.f;
     const int lim = min(vis, j_end);
@@ -743,36 +777,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
     const float lse = empty ? -CUDART_INF_F : (m_used + log2f(ltot)) * 0.6931471805599453f;
     const size_t orow = ((size_t)b * p.s_q + g) * p.H + (row_ok ? head : 0);
     const bool read_o = alive && n > 0;
-    // TMEM columns 128*ch .. +127 of this lane: latent half*128 + 256*ch + 0..127
+    // TMEM columns 128*ch .. +127 of this lane: latent half*128 + 256*ch + 0..127,
+    // loaded kEpi x 32 columns at a time (one wait per group)
+    constexpr int kEpi = FP8 ? 1 : 2;  // fp8 threads have fewer registers to spare
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      uint32_t ov[32];
+    for (int c0 = 0; c0 < 4; c0 += kEpi) {
+      uint32_t ovs[kEpi][32];
       if (read_o) {
-        tmem_ld32(tl + 128u * ch + 32u * c, ov);
+#pragma unroll
+        for (int i = 0; i < kEpi; ++i) tmem_ld32(tl + 128u * ch + 32u * (c0 + i), ovs[i]);
         tmem_wait_ld();
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) ov[j] = 0u;
+        for (int i = 0; i < kEpi; ++i)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ovs[i][j] = 0u;
       }
-      const int col = 256 * ch + half * 128 + 32 * c;
-      if (!row_ok) continue;
-      if (p.splits == 1) {
-        uint4* dst = reinterpret_cast<uint4*>(p.o_lat + orow * kDc + col);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint4 v;
-          v.x = pack_bf16(__uint_as_float(ov[8 * k + 0]) * inv, __uint_as_float(ov[8 * k + 1]) * inv);
-          v.y = pack_bf16(__uint_as_float(ov[8 * k + 2]) * inv, __uint_as_float(ov[8 * k + 3]) * inv);
-          v.z = pack_bf16(__uint_as_float(ov[8 * k + 4]) * inv, __uint_as_float(ov[8 * k + 5]) * inv);
-          v.w = pack_bf16(__uint_as_float(ov[8 * k + 6]) * inv, __uint_as_float(ov[8 * k + 7]) * inv);
-          dst[k] = v;
+      for (int i = 0; i < kEpi; ++i) {
+        const uint32_t (&ov)[32] = ovs[i];
+        const int c = c0 + i;
+        const int col = 256 * ch + half * 128 + 32 * c;
+        if (!row_ok) continue;
+        if (p.splits == 1) {
+          uint4* dst = reinterpret_cast<uint4*>(p.o_lat + orow * kDc + col);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            uint4 v;
+            v.x = pack_bf16(__uint_as_float(ov[8 * k + 0]) * inv, __uint_as_float(ov[8 * k + 1]) * inv);
+            v.y = pack_bf16(__uint_as_float(ov[8 * k + 2]) * inv, __uint_as_float(ov[8 * k + 3]) * inv);
+            v.z = pack_bf16(__uint_as_float(ov[8 * k + 4]) * inv, __uint_as_float(ov[8 * k + 5]) * inv);
+            v.w = pack_bf16(__uint_as_float(ov[8 * k + 6]) * inv, __uint_as_float(ov[8 * k + 7]) * inv);
+            dst[k] = v;
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(p.o_part + (orow * p.splits + split) * kDc + col);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            dst[k] = make_float4(__uint_as_float(ov[4 * k]) * inv, __uint_as_float(ov[4 * k + 1]) * inv,
+                                 __uint_as_float(ov[4 * k + 2]) * inv, __uint_as_float(ov[4 * k + 3]) * inv);
         }
-      } else {
-        float4* dst = reinterpret_cast<float4*>(p.o_part + (orow * p.splits + split) * kDc + col);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          dst[k] = make_float4(__uint_as_float(ov[4 * k]) * inv, __uint_as_float(ov[4 * k + 1]) * inv,
-                               __uint_as_float(ov[4 * k + 2]) * inv, __uint_as_float(ov[4 * k + 3]) * inv);
       }
     }
     if (half == 0 && ch == 0 && row_ok) {
