@@ -198,7 +198,7 @@ template <bool FP8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : kThreadsBf16, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qpe,
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_kv,
-                     const TcParams p) {
+                     const __grid_constant__ CUtensorMap tm_o, const TcParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
@@ -329,7 +329,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
           if (r == 0) mbar_arrive_expect_tx_local_elect(own_bar(S_FULL + st), 2 * kSStage);
           tma_load_3d_pair_elect(dst, &tm_ks, fb, 0, pg * kPage + 32 * (int)r, 0);
         }
-        if (u + kPrefetchTiles < n) prefetch(u + kPrefetchTiles);
+        if (u > 0 && u + kPrefetchTiles < n) prefetch(u + kPrefetchTiles);
         return true;
       };
       auto load_v = [&](int u) -> bool {
@@ -380,9 +380,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
       };
       // The cache, block table and lengths are not written by the kernel this one
       // may overlap with (the query absorption); q_lat is, so Q waits for it.
-      // page 0's score stage first, then the L2 prefetch of the next pages and Q
+      // page 0's score stage and Q first: every CTA asks for its first bytes at
+      // the same moment, and these two gate the first score MMA; the L2
+      // prefetch of the next pages only after them
       bool ok = load_s(0);
-      for (int u = 1; u < n && u < kPrefetchTiles; ++u) prefetch(u);
       pdl_wait();
       if (!FP8 && lane == 0) {
         // 3-D maps (values, heads, query tokens): heads >= H come in as zeros.
@@ -400,6 +401,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
           tma_load_3d_cta(sa + kVOff + c * kChunkQ, &tm_q, own_bar(Q_STAGE), 64 * c, h0, qtok);
       }
       __syncwarp();
+      for (int u = 1; u < n && u <= kPrefetchTiles; ++u) prefetch(u);
       for (int u = 0; ok && u < n; ++u) {
         if (u + 1 < n) ok = load_s(u + 1);
         if (!FP8 && u == 0 && ok)
@@ -798,9 +800,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
         const uint32_t (&ov)[32] = ovs[i];
         const int c = c0 + i;
         const int col = 256 * ch + half * 128 + 32 * c;
-        if (!row_ok) continue;
-        if (p.splits == 1) {
-          uint4* dst = reinterpret_cast<uint4*>(p.o_lat + orow * kDc + col);
+          if (p.splits == 1) {
+          // bf16 row m, latent col .. col+31 into the staging area (the score ring,
+          // idle now): 64-column chunks of 64 rows x 128 bytes, 128-byte swizzled
+          const int chunk = col >> 6;
+          const uint32_t base = sa + kSOff + chunk * (64 * 128) + m * 128;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             uint4 v;
@@ -808,15 +812,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
             v.y = pack_bf16(__uint_as_float(ov[8 * k + 2]) * inv, __uint_as_float(ov[8 * k + 3]) * inv);
             v.z = pack_bf16(__uint_as_float(ov[8 * k + 4]) * inv, __uint_as_float(ov[8 * k + 5]) * inv);
             v.w = pack_bf16(__uint_as_float(ov[8 * k + 6]) * inv, __uint_as_float(ov[8 * k + 7]) * inv);
-            dst[k] = v;
+            const int u = ((col & 63) >> 3) + k;
+            sts128(base + ((u ^ (m & 7)) << 4), v);
           }
         } else {
+          if (!row_ok) continue;
           float4* dst = reinterpret_cast<float4*>(p.o_part + (orow * p.splits + split) * kDc + col);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             dst[k] = make_float4(__uint_as_float(ov[4 * k]) * inv, __uint_as_float(ov[4 * k + 1]) * inv,
                                  __uint_as_float(ov[4 * k + 2]) * inv, __uint_as_float(ov[4 * k + 3]) * inv);
         }
+      }
+    }
+    if (p.splits == 1) {
+      // one thread stores the 8 chunks of this CTA's 64 rows (rows past H are
+      // outside the map and not written)
+      fence_proxy_async_smem();
+      named_bar_sync(1, 256);
+      if (warp == 4 && lane == 0) {
+        const int qtok = b * p.s_q + g;
+        for (int c = 0; c < 8; ++c) tma_store_3d(&tm_o, sa + kSOff + c * (64 * 128), 64 * c, 64 * (int)r, qtok);
+        bulk_commit_group();
+        bulk_wait_all();
       }
     }
     if (half == 0 && ch == 0 && row_ok) {
@@ -845,12 +863,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
 // ---------------------------------------------------------------- host side
 template <bool FP8>
 cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t stream) {
-  CUtensorMap tm_q, tm_qpe, tm_ks, tm_kv;
+  CUtensorMap tm_q, tm_qpe, tm_ks, tm_kv, tm_o;  // tm_o: o_lat, the single-split result
   const uint64_t rows_kv = (uint64_t)a->num_pages * kPage;
   const int n_tok = a->B * a->s_q;
   // query maps are 3-D (values, heads, tokens) so that a 64-head box past H reads zeros
   if (!tma_map_3d(&tm_q, a->q_lat, kDc, a->H, n_tok, kDc * 2, (uint64_t)a->H * kDc * 2, 64, 64, 1) ||
-      !tma_map_3d(&tm_qpe, a->q_pe, kDr, a->H, n_tok, kDr * 2, (uint64_t)a->H * kDr * 2, 64, 64, 1))
+      !tma_map_3d(&tm_qpe, a->q_pe, kDr, a->H, n_tok, kDr * 2, (uint64_t)a->H * kDr * 2, 64, 64, 1) ||
+      !tma_map_3d(&tm_o, a->o_lat, kDc, a->H, n_tok, kDc * 2, (uint64_t)a->H * kDc * 2, 64, 64, 1))
     return cudaErrorInvalidValue;
   if (FP8) {
     // the e4m3 rows (576 bytes) viewed as two-byte units: (128 units, rows, 2
@@ -906,7 +925,7 @@ cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t strea
   }
   dim3 grid(2 * splits, a->s_q, a->B);
   return launch_pdl(kern, grid, dim3(FP8 ? kThreadsFp8 : kThreadsBf16), kSmemBytes, stream, tm_q, tm_qpe, tm_ks,
-                    tm_kv, p);
+                    tm_kv, tm_o, p);
 }
 
 }  // namespace

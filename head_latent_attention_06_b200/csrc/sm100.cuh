@@ -229,6 +229,17 @@ MLA_DEVI void tma_load_4d_cta(uint32_t dst, const void* tmap, uint32_t mbar, int
       : "memory");
 }
 
+// 3-D tile store from this CTA's shared memory to global memory (bulk group);
+// out-of-bounds parts of the box are not written.
+MLA_DEVI void tma_store_3d(const void* tmap, uint32_t src, int32_t x, int32_t y, int32_t z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(tmap),
+               "r"(src), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+MLA_DEVI void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until every bulk store this thread committed has completed.
+MLA_DEVI void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Contiguous copy of `bytes` (multiple of 16; both addresses 16-byte aligned)
 // from global to this CTA's shared memory, completion counted on `mbar`.
 MLA_DEVI void bulk_load_cta(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
