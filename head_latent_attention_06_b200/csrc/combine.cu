@@ -12,6 +12,7 @@
 namespace mla {
 namespace {
 
+template <int kBatch>
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ o_part,
                                                       const float* __restrict__ lse_part,
                                                       __nv_bfloat16* __restrict__ o_lat,
@@ -39,18 +40,30 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
 #pragma unroll
   for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
   const float* op = o_part + (size_t)row * splits * kDc;
-  for (int s = 0; s < splits; ++s) {
-    const float ls = lp[s];
-    if (ls == -CUDART_INF_F) continue;
-    const float w = __expf(ls - ref) * inv_z;
+  // splits in batches of kBatch whose loads are all in flight before the first
+  // use: one memory latency per batch rather than per split
+  for (int s0 = 0; s0 < splits; s0 += kBatch) {
+    float w[kBatch];
+    float4 v[kBatch][4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float4 v = *reinterpret_cast<const float4*>(op + (size_t)s * kDc + k * 128 + lane * 4);
-      acc[k].x += w * v.x;
-      acc[k].y += w * v.y;
-      acc[k].z += w * v.z;
-      acc[k].w += w * v.w;
+    for (int j = 0; j < kBatch; ++j) {
+      const int s = s0 + j;
+      const float ls = s < splits ? lp[s] : -CUDART_INF_F;
+      w[j] = ls == -CUDART_INF_F ? 0.f : __expf(ls - ref) * inv_z;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        v[j][k] = w[j] != 0.f ? *reinterpret_cast<const float4*>(op + (size_t)s * kDc + k * 128 + lane * 4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc[k].x += w[j] * v[j][k].x;
+        acc[k].y += w[j] * v[j][k].y;
+        acc[k].z += w[j] * v[j][k].z;
+        acc[k].w += w[j] * v[j][k].w;
+      }
   }
   __nv_bfloat16* dst = o_lat + (size_t)row * kDc;
 #pragma unroll
@@ -70,7 +83,9 @@ cudaError_t launch_combine(const mla_decode_args_t* a, int splits, cudaStream_t 
   const int rows = n_tok * a->H;
   WorkspaceLayout wl = workspace_layout(n_tok, a->H, splits);
   const unsigned char* ws = static_cast<const unsigned char*>(a->workspace);
-  return launch_pdl(combine_kernel, dim3((rows + 3) / 4), dim3(128), 0, stream,
+  // few splits: a small batch keeps the registers low and the warps many
+  auto kern = splits <= 2 ? combine_kernel<2> : combine_kernel<6>;
+  return launch_pdl(kern, dim3((rows + 3) / 4), dim3(128), 0, stream,
                     reinterpret_cast<const float*>(ws + wl.o_part_off),
                     reinterpret_cast<const float*>(ws + wl.lse_part_off),
                     static_cast<__nv_bfloat16*>(a->o_lat), a->lse, rows, splits);
