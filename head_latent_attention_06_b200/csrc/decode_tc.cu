@@ -45,11 +45,11 @@
 //
 // fp8 (e4m3) cache with a per-token scale: the MMAs run on f16 operands.  Every
 // e4m3 value is exactly an f16 value, so the cache needs only a format change:
-// the producer brings the raw bytes of a stage into the back half of its slot
-// (the CTA's 32 rows with one bulk copy; the value operand's 64 rows x 2 x 128
-// bytes with two TMA boxes), four converter warps (12..15) read the whole stage,
-// then write it back as f16 in the layout the TMA gives the bf16 cache, and mark
-// the slot full.  Q is rounded from bf16 to f16 once (exact inside f16's normal
+// the producer brings the raw bytes of the CTA's 32 score rows into the back half
+// of their stage slot (one bulk copy), four converter warps (12..15) read the
+// whole stage, then write it back as f16 in the layout the TMA gives the bf16
+// cache, and mark the slot full.  The value operand is assembled from both
+// CTAs' converted score stages by shared-memory bulk copies (see copy_v).  Q is rounded from bf16 to f16 once (exact inside f16's normal
 // range).  The token scales stay out of the operands: the softmax multiplies
 // the raw scores by them, and P by them before the P.V MMA, so that
 // O = sum_t p_t * scale_t * code_t.  Rows past the sequence end are written as
@@ -114,7 +114,8 @@ constexpr int O_DONE = P_READY + 2;       // [2]
 constexpr int DRAIN = O_DONE + 2;        // [3] one per MMA-issuing warp
 constexpr int S_FREE = DRAIN + 3;         // [2] in the even CTA: the softmax has read S buffer sb
 constexpr int RAW_S = S_FREE + 2;         // [kSStages] fp8: raw bytes of a score stage landed
-constexpr int RAW_V = RAW_S + kSStages;   // [kVStages] fp8: raw bytes of a value stage landed
+constexpr int RAW_V = RAW_S + kSStages;   // [kVStages] bf16: a last page's value stage landed here;
+                                          // fp8: both CTAs' copies into this CTA's value stage landed
 constexpr int SC_FULL = RAW_V + kVStages; // [kScRing]  fp8: token scales of a tile landed
 constexpr int Q_STAGE = SC_FULL + kScRing; // bf16: Q chunks 0..5 landed in the value ring (this CTA)
 constexpr int Q_MOVED = Q_STAGE + 1;        // bf16: the softmax warps have moved them into TMEM
@@ -233,11 +234,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
     const uint32_t full_count = FP8 ? 2 * kConvWarps : 1;
     for (int i = 0; i < kSStages; ++i) {
       mbar_init(own_bar(S_FULL + i), full_count);
-      mbar_init(own_bar(S_EMPTY + i), 1);
+      // fp8: a stage is free once its score MMAs are done and the value-operand
+      // copies have read it
+      mbar_init(own_bar(S_EMPTY + i), FP8 ? 2 : 1);
       mbar_init(own_bar(RAW_S + i), 1);
     }
     for (int i = 0; i < kVStages; ++i) {
-      mbar_init(own_bar(V_FULL + i), FP8 ? full_count : 2);
+      mbar_init(own_bar(V_FULL + i), 2);
       mbar_init(own_bar(V_EMPTY + i), 1);
       mbar_init(own_bar(RAW_V + i), 1);
     }
@@ -338,15 +341,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
         if (!mbar_wait_converged(own_bar(V_EMPTY + st), ph, abort_flag, p.status, kWaitLimitNs)) return false;
         const int pg = page_of(u, blk_v, pg_v);
         const uint32_t dst = sa + kVOff + st * kVStage;
-        if constexpr (FP8) {
-          // raw bytes 128r .. +127 and 256+128r .. +127 of the page's 64 rows (the
-          // map views a row as 288 two-byte units) into the back half of the slot
-          if (lane == 0) {
-            mbar_arrive_expect_tx_local(own_bar(RAW_V + st), kVStage / 2);
-            tma_load_3d_cta(dst + kVStage / 2, &tm_kv, own_bar(RAW_V + st), 64 * (int)r, pg * kPage, 0);
-          }
-          __syncwarp();
-        } else {
+        {  // bf16 only: the fp8 value operand is copied from the converted score stages
           const int nvalid = j_end - (t0 + u) * kPage;  // cached rows of this page inside the sequence
           if (nvalid >= kPage) {
             // one box: (64 values, 64 rows, chunks 2r and 2r+1, groups 0 and 1): latent
@@ -406,7 +401,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
         if (u + 1 < n) ok = load_s(u + 1);
         if (!FP8 && u == 0 && ok)
           ok = mbar_wait_converged(own_bar(Q_MOVED), 0, abort_flag, p.status, kWaitLimitNs);
-        if (ok) ok = load_v(u);
+        if (!FP8 && ok) ok = load_v(u);
       }
     }
   } else if (warp == 1 || warp == 2 || (!FP8 && warp == 3)) {
@@ -504,6 +499,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
       // rows i (even) and i + 1 share a quarter-warp, four 16-byte units each: the
       // reads (576-byte row pitch) and the swizzled writes both hit 8 distinct bank groups
       const int i = 2 * (ct >> 3) + ((ct >> 2) & 1), w = 2 * (ct & 3);
+      // rows past the sequence end become zeros: the value operand is copied from here
+      const bool live = 32 * (int)r + i < j_end - (t0 + u) * kPage;
       uint4 v[9];
 #pragma unroll
       for (int c = 0; c < 9; ++c)
@@ -512,61 +509,64 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
 #pragma unroll
       for (int c = 0; c < 9; ++c) {
         // values 64c + 16(ct&3) .. +15 of row i: f16 units w, w + 1 of chunk c
-        uint4 lo, hi;
-        e4m3x16_to_f16(v[c], lo, hi);
+        uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
+        if (live) e4m3x16_to_f16(v[c], lo, hi);
         const uint32_t row = slot + c * kChunkS + i * 128;
         sts128(row + ((w ^ (i & 7)) << 4), lo);
         sts128(row + (((w + 1) ^ (i & 7)) << 4), hi);
       }
       fence_proxy_async_smem();
+      named_bar_sync(5, 32 * kConvWarps);  // the whole stage is written before it is copied
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(lead_bar(S_FULL + st));
     };
-    auto convert_v = [&](int u) {
-      const int st = u % kVStages;
-      mbar_wait(own_bar(RAW_V + st), (u / kVStages) & 1, abort_flag, p.status, kWaitLimitNs);
-      const uint32_t slot = sa + kVOff + st * kVStage;
-      const uint32_t raw = slot + kVStage / 2;  // [2 segments][64 rows][128 bytes], 128-byte swizzle
-      const int nvalid = j_end - (t0 + u) * kPage;  // rows at or past it are zeroed
-      // item = (segment, row pair, flip); a quarter-warp takes rows i, i + 1 and
-      // units e ^ 4flip: conflict-free reads and writes
-      auto coords = [&](int k, int& seg, int& i, int& uu) {
-        const int item = 16 * k + (ct >> 3);
-        seg = item >> 6;
-        i = 2 * ((item >> 1) & 31) + ((ct >> 2) & 1);
-        uu = (ct & 7) ^ (4 * (item & 1));
-      };
-      uint4 v[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        int seg, i, uu;
-        coords(k, seg, i, uu);
-        v[k] = lds128(raw + seg * (kVStage / 4) + i * 128 + ((uu ^ (i & 7)) << 4));
+    // The value operand of page u: the converted latent chunks of this CTA's 32
+    // rows go to the CTA that holds their columns (chunks {2d, 2d+1, 4+2d, 5+2d}
+    // belong to CTA d), into rows 32r .. 32r+31 of its value stage: eight 4 KB
+    // bulk copies, four to this CTA and four to the peer, counted on the
+    // destination's RAW_V barrier.  The 128-byte swizzle depends on the row mod 8
+    // only, so a block copied 32 rows down keeps its layout.  Both CTAs' value
+    // slots are released by the same multicast commit, so waiting for our own is
+    // enough for both destinations.  A score stage may be refilled once its copies
+    // have read it: the arrival on S_EMPTY for page u is made when the copies of
+    // page u+1 are issued (or never, for pages with no later refill).
+    auto copy_v = [&](int u) {
+      if (ct != 0) return;
+      const int st = u % kVStages, ss = u % kSStages;
+      mbar_wait(own_bar(V_EMPTY + st), ((u / kVStages) & 1) ^ 1, abort_flag, p.status, kWaitLimitNs);
+#pragma unroll 1
+      for (int lc = 0; lc < 8; ++lc) {
+        const uint32_t d = (lc >> 1) & 1, j = 2 * (lc >> 2) + (lc & 1);
+        const uint32_t dst = sa + kVOff + st * kVStage + j * kChunkV + r * (32 * 128);
+        bulk_copy_s2s(mapa(dst, d), sa + kSOff + ss * kSStage + lc * kChunkS, kChunkS, mapa(own_bar(RAW_V + st), d));
       }
-      named_bar_sync(5, 32 * kConvWarps);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        int seg, i, uu;
-        coords(k, seg, i, uu);
-        uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-        if (i < nvalid) e4m3x16_to_f16(v[k], lo, hi);
-        // values 16uu .. 16uu+15 of the segment: chunk 2seg + uu/4, f16 units 2(uu&3), +1
-        const uint32_t row = slot + (2 * seg + (uu >> 2)) * kChunkV + i * 128;
-        const int w = 2 * (uu & 3);
-        sts128(row + ((w ^ (i & 7)) << 4), lo);
-        sts128(row + (((w + 1) ^ (i & 7)) << 4), hi);
+      bulk_commit_group();
+      if (u >= 1) {
+        bulk_wait_read<1>();  // page u-1's copies have read their stage
+        mbar_arrive_remote(own_bar(S_EMPTY + (u - 1) % kSStages));
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(lead_bar(V_FULL + st));
     };
     if (n > 0) {
       convert_s(0);
       for (int u = 0; u < n; ++u) {
         if (u + 1 < n) convert_s(u + 1);
-        convert_v(u);
+        copy_v(u);
+      }
+      if (ct == 0) bulk_wait_all();  // every copy has landed before shared memory is released
+    }
+  } else if (FP8 && warp == 3) {
+    // ============ fp8: value-stage relay (one thread) ============
+    // Posts the expected bytes of each value stage of this CTA (both CTAs' copies),
+    // waits for them, and arrives on the even CTA's V_FULL (count 2: one per CTA).
+    if (n > 0 && lane == 0) {
+      for (int u = 0; u < n; ++u) {
+        const int st = u % kVStages;
+        mbar_arrive_expect_tx_local(own_bar(RAW_V + st), kVStage);
+        if (!mbar_wait(own_bar(RAW_V + st), (u / kVStages) & 1, abort_flag, p.status, kWaitLimitNs)) break;
+        mbar_arrive_remote(lead_bar(V_FULL + st));
       }
     }
+    __syncwarp();
   } else if (warp >= 4 && warp < 12) {
     // ====================== softmax / correction / epilogue ======================
     // Thread = (TMEM lane lt, column half ch).  Lane lt holds head row m = lt % 64

@@ -229,6 +229,20 @@ MLA_DEVI void tma_load_4d_cta(uint32_t dst, const void* tmap, uint32_t mbar, int
       : "memory");
 }
 
+// Contiguous copy of `bytes` (multiple of 16) from this CTA's shared memory to
+// shared memory of either CTA of the cluster; completion (bytes) is counted on a
+// barrier in the destination CTA.  Committed with bulk_commit_group.
+MLA_DEVI void bulk_copy_s2s(uint32_t dst_cluster, uint32_t src, uint32_t bytes, uint32_t mbar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst_cluster),
+      "r"(src), "r"(bytes), "r"(mbar_cluster)
+      : "memory");
+}
+// Waits until at most N of this thread's committed bulk groups still read their source.
+template <int N>
+MLA_DEVI void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
+
 // 3-D tile store from this CTA's shared memory to global memory (bulk group);
 // out-of-bounds parts of the box are not written.
 MLA_DEVI void tma_store_3d(const void* tmap, uint32_t src, int32_t x, int32_t y, int32_t z) {
