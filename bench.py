@@ -41,7 +41,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # with the sha256 prefix of the kernel source it was taken on: reported as the
 # roofline's ``traffic`` only while that source is unchanged.
 # (profiles/decode_tc_v3_bf16.md)
-MEASURED_TRAFFIC = {"v3": (311513856 + 4139520, "86f8f7d81a0eb4b2")}
+MEASURED_TRAFFIC = {"v3": (311525632 + 5262080, "5a3679ac14259253")}
 
 
 def decode_traffic(config: str):

@@ -30,11 +30,12 @@
 // columns, each S buffer 32 columns (two buffers).  Lane l < 64 holds head row l
 // for the first half of every N tile, lane 64 + l the same row for the second.
 //
-// Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM allocator and (in
-// the even CTA) issuer of the score MMAs (bf16: of even pages, warp 3 of odd
-// ones), warp 2 (even CTA) issuer of the P.V MMAs, warps 4..11 softmax /
+// Warp roles (384 threads; fp8 512): warp 0 TMA producer, warp 1 TMEM allocator
+// and (in the even CTA) issuer of the score MMAs (bf16: of even pages, warp 3 of
+// odd ones), warp 2 (even CTA) issuer of the P.V MMAs, warps 4..11 softmax /
 // correction / epilogue, two warps per TMEM lane quadrant, each thread 16
-// scores of a row half per page.
+// scores of a row half per page; fp8: warps 12..15 convert, warp 3 relays the
+// value stages' completion.
 // Two S buffers: each softmax warp releases its S buffer as soon as its scores
 // are in registers, so S(t+2) is issued while the softmax of t is still running
 // and the tensor pipe does not wait on it; each softmax warp signals its own P
