@@ -102,7 +102,8 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        import tempfile
+        self.path = os.path.join(tempfile.gettempdir(), f"mla_bench_clocks_rank{index}.csv")
 
     def __enter__(self):
         try:

@@ -44,7 +44,7 @@ extern "C" {
 typedef enum {
   MLA_OK = 0,
   MLA_ERR_INVALID_VALUE = 1,        /* null pointer, negative or inconsistent size */
-  MLA_ERR_UNSUPPORTED = 2,          /* a dimension this build does not handle */
+  MLA_ERR_UNSUPPORTED = 2,          /* a dimension the library does not handle */
   MLA_ERR_MISALIGNED = 3,           /* a pointer is not 16-byte aligned */
   MLA_ERR_WORKSPACE_TOO_SMALL = 4,  /* workspace_bytes < mla_decode_workspace_size() */
   MLA_ERR_CUDA = 5,                 /* a CUDA runtime call or launch failed */

@@ -19,7 +19,7 @@ What it follows (page titles and sections of the pages this method comes from):
 * Standard softmax attention with a log-sum-exp output; split partials merge by
   the log-sum-exp identity (``combine_splits``).
 
-Readings taken where the pages are silent (each one is listed in the design doc):
+Readings taken where the pages are silent:
 RoPE is already applied to the cached ``k_pe`` and to ``q_pe`` (the kernel
 rotates nothing); the softmax scale is 1/sqrt(qk_nope + rope) = 1/sqrt(192);
 ``W_UK[h]`` and ``W_UV[h]`` are the per-head [128 x 512] slices; with causal
