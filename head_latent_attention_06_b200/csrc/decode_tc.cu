@@ -397,6 +397,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
           tma_load_3d_cta(sa + kVOff + c * kChunkQ, &tm_q, own_bar(Q_STAGE), 64 * c, h0, qtok);
       }
       __syncwarp();
+      // bf16: nothing else is requested until Q has landed: at start-up every CTA
+      // asks for its first bytes at once, and Q and page 0 gate the first MMA
+      if (!FP8 && ok) ok = mbar_wait_converged(own_bar(Q_STAGE), 0, abort_flag, p.status, kWaitLimitNs);
       for (int u = 1; u < n && u <= kPrefetchTiles; ++u) prefetch(u);
       for (int u = 0; ok && u < n; ++u) {
         if (u + 1 < n) ok = load_s(u + 1);
