@@ -55,6 +55,32 @@ def decode_traffic(config: str):
     return entry[0] if digest == entry[1] else None
 
 
+# Nominal B200 figures, the secondary denominators: HBM3e 7.7 TB/s (HGX), dense
+# bf16/f16 tensor 2.25 PFLOP/s.
+DATASHEET = {"hbm_gbs": 7700.0, "bf16_tflops": 2250.0}
+
+
+def datasheet_fracs(cache_bytes: float, flops: float, seconds: float) -> dict:
+    """The decode's fractions of the nominal figures (the measured peaks are the
+    primary denominators)."""
+    t_mem = cache_bytes / (DATASHEET["hbm_gbs"] * 1e9)
+    t_tc = flops / (DATASHEET["bf16_tflops"] * 1e12)
+    return {"hbm_gbs": DATASHEET["hbm_gbs"], "bf16_tflops": DATASHEET["bf16_tflops"],
+            "hbm_frac": round(t_mem / seconds, 4), "tensor_frac": round(t_tc / seconds, 4),
+            "binding_frac": round(max(t_mem, t_tc) / seconds, 4)}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown CPU"
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -177,7 +203,8 @@ def oracle_cpu_baseline(spec_name: str, budget_s: float = 12.0):
         pass
     gbs = done_tokens * row_bytes / dt / 1e9
     desc = (f"oracle decode_absorbed (fp64 numpy) on {done_b} of {w.B} sequences "
-            f"({done_tokens} cached tokens, all {w.H} heads, {w.s_q} queries) in {dt:.2f} s")
+            f"({done_tokens} cached tokens, all {w.H} heads, {w.s_q} queries) in {dt:.2f} s "
+            f"on {cpu_model()}")
     return gbs, desc, cores, dt
 
 
@@ -401,7 +428,9 @@ def main(argv=None):
                        "peak_tflops": float(peaks["bf16_tflops"]),
                        "frac": round(dec_tflops / float(peaks["bf16_tflops"]), 4)},
             "binding_roofline_frac": round(max(t_mem, t_tc) / (dec_avg_ms * 1e-3), 4),
+            "datasheet": datasheet_fracs(cache_bytes, flops, dec_avg_ms * 1e-3),
         },
+        "cached_tokens_per_s": round(world * sum(w.lens) / (dec_avg_ms * 1e-3), 1),
         "e2e": {"value": round(world * cache_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 5),
