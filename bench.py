@@ -208,6 +208,34 @@ def oracle_cpu_baseline(spec_name: str, budget_s: float = 12.0):
     return gbs, desc, cores, dt
 
 
+def oracle_nonabsorbed_sample(spec_name: str, budget_s: float = 3.0):
+    """Times the oracle's non-absorbed form (K and V formed per head, the
+    definition itself) on the heads of one query row that fit the budget, and
+    extrapolates to the whole workload by cached tokens x heads.  The
+    extrapolation is an estimate, labelled as such; the absorbed form above is
+    the measured baseline."""
+    from mla_inputs import make_workload, preset
+    import oracle
+    from oracle import mla_oracle as om
+    spec = preset(spec_name)
+    w = make_workload(spec)
+    inp = oracle.from_workload(w)
+    b, i = 0, w.s_q - 1
+    n = inp.visible(b, i)
+    heads, t0 = 0, time.perf_counter()
+    while heads < w.H and time.perf_counter() - t0 < budget_s:
+        om.decode_nonabsorbed(inp, rows=[(b, i)], heads=[heads])
+        heads += 1
+    dt = time.perf_counter() - t0
+    us_per_token_head = dt * 1e6 / max(1, heads * n)
+    work = sum(inp.visible(bb, ii) for bb in range(w.B) for ii in range(w.s_q)) * w.H
+    return {"us_per_token_head": round(us_per_token_head, 5),
+            "extrapolated_full_s": float(f"{us_per_token_head * work * 1e-6:.4g}"),
+            "sample": f"oracle decode_nonabsorbed (fp64 numpy), sequence 0 query {i} "
+                      f"({n} cached tokens), {heads} of {w.H} heads in {dt:.2f} s; "
+                      f"full-workload time extrapolated by cached tokens x heads"}
+
+
 def run_reference(args):
     """The oracle timed on the host cores as the reference arm (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
@@ -441,7 +469,8 @@ def main(argv=None):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, desc, cores, _ = oracle_cpu_baseline(args.config)
         line["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": cores,
-                                "kind": "oracle", "sample": desc}
+                                "kind": "oracle", "sample": desc,
+                                "nonabsorbed": oracle_nonabsorbed_sample(args.config)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

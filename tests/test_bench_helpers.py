@@ -31,3 +31,12 @@ def test_traffic_reported_only_for_the_profiled_source():
 
 def test_cpu_model_is_text():
     assert isinstance(bench.cpu_model(), str) and bench.cpu_model()
+
+
+def test_nonabsorbed_sample_extrapolates_by_tokens_and_heads():
+    r = bench.oracle_nonabsorbed_sample("tiny", budget_s=0.5)
+    assert r["us_per_token_head"] > 0
+    # tiny: one sequence of 256 cached tokens, 16 heads, one query
+    est = r["us_per_token_head"] * 256 * 16 * 1e-6
+    assert abs(r["extrapolated_full_s"] - est) <= 1e-3 * est + 1e-4
+    assert "extrapolated" in r["sample"]
