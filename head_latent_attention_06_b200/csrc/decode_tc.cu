@@ -1,8 +1,8 @@
 // Paged latent-attention decode on the 5th-generation tensor cores (sm_100a):
 // tcgen05 MMAs over a CTA pair, accumulators in tensor memory (TMEM), cache
-// pages streamed by TMA.  This is the path for a bf16 cache and up to 128 heads
-// (fewer heads pad the 128-row tile with zero rows: the step stays bound by the
-// cache stream, so the idle rows cost tensor work only).
+// pages streamed by TMA.  This is the path for a bf16 or e4m3 cache and 16 to 128
+// heads (fewer heads pad the 128-row tile with zero rows: the step stays bound by
+// the cache stream, so the idle rows cost tensor work only).
 //
 // What it computes (absorbed MLA decode; nnets.ru article, sections "Суть MLA"
 // and "MLA и FlashAttention"; snowgate thread 35 on the 512 + 64 latent record):
@@ -15,17 +15,20 @@
 // is the paired form (cta_group::2, M = 128): CTA r holds the Q rows of heads
 // 64r .. 64r+63 and receives their S and O rows in its TMEM.  Per 64-token page:
 //   S  (M=128, N=64,  K=576): B = the page's tokens; CTA r supplies its 32
-//        tokens x 576 (9 TMA boxes of 32 x 64).
+//        tokens x 576 (one 3-D TMA box: 64 values x 32 rows x 9 chunks).
 //   PV (M=128, N=256, K=64) twice (latent 0..255, 256..511): B = all 64 tokens x
-//        the CTA's 128-column half of each N tile (4 TMA boxes of 64 x 64, a
-//        second read of the page that hits L2).
+//        the CTA's 128-column half of each N tile (one 4-D TMA box of 4 chunks of
+//        64 x 64, a second read of the page that hits L2).
 // The cache streams through two rings, one for the score operand (S stages of
 // 36 KB) and one for the value operand (V stages of 32 KB), in the order the
 // MMAs consume them.  Only the even CTA posts the expected byte count of a stage
 // (both CTAs' bytes) on its own barrier; the odd CTA's TMA completes its bytes
-// there without arriving; each slot is released by the commit of the MMAs that read it, so
-// the producer refills it at once.  Each CTA also prefetches its half of the
-// page four tiles ahead into L2 with a bulk prefetch.
+// there without arriving; each slot is released by the commit of the MMAs that
+// read it, so the producer refills it at once.  Each CTA also prefetches its half
+// of the page two tiles ahead into L2 with a bulk prefetch.
+// Q: latent chunks 0..5 are the A operand from TMEM; they are staged by TMA in the
+// value ring (idle until page 0's value operand) and moved into TMEM by the
+// softmax warps; chunks 6..7 and q_pe stay in shared memory.
 // TMEM per CTA (2x2 datapath layout of the paired M = 128 MMA): O takes 256
 // columns, each S buffer 32 columns (two buffers).  Lane l < 64 holds head row l
 // for the first half of every N tile, lane 64 + l the same row for the second.
@@ -50,8 +53,9 @@
 // of their stage slot (one bulk copy), four converter warps (12..15) read the
 // whole stage, then write it back as f16 in the layout the TMA gives the bf16
 // cache, and mark the slot full.  The value operand is assembled from both
-// CTAs' converted score stages by shared-memory bulk copies (see copy_v).  Q is rounded from bf16 to f16 once (exact inside f16's normal
-// range).  The token scales stay out of the operands: the softmax multiplies
+// CTAs' converted score stages by shared-memory bulk copies (see copy_v).  Q is
+// rounded from bf16 to f16 once (exact inside f16's normal range).  The token
+// scales stay out of the operands: the softmax multiplies
 // the raw scores by them, and P by them before the P.V MMA, so that
 // O = sum_t p_t * scale_t * code_t.  Rows past the sequence end are written as
 // zeros in the value operand, so that whatever bytes they hold cannot reach O.
@@ -63,6 +67,7 @@
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <math_constants.h>
+#include <string.h>
 
 #include "sm100.cuh"
 #include "tma_host.cuh"
@@ -285,8 +290,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
   if (warp == 0) {
     // =========================== TMA producer ===========================
     // Ring order = MMA order: S(0), S(1), V(0), S(2), V(1), ... where S(u) is the
-    // CTA's 32 tokens x 576 of page u (9 slots) and V(u) the page's 64 tokens x
-    // the CTA's latent columns of both P.V halves (8 slots of 16 tokens x 128).
+    // CTA's 32 tokens x 576 of page u (one 36 KB score stage) and V(u) the page's
+    // 64 tokens x the CTA's latent columns of both P.V halves (one 32 KB value
+    // stage).
     if (n > 0) {
       // physical pages, fetched 32 at a time by the whole warp
       int blk_s = -1, pg_s = 0, blk_v = -1, pg_v = 0, blk_p = -1, pg_p = 0;
@@ -804,7 +810,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
         const uint32_t (&ov)[32] = ovs[i];
         const int c = c0 + i;
         const int col = 256 * ch + half * 128 + 32 * c;
-          if (p.splits == 1) {
+        if (p.splits == 1) {
           // bf16 row m, latent col .. col+31 into the staging area (the score ring,
           // idle now): 64-column chunks of 64 rows x 128 bytes, 128-byte swizzled
           const int chunk = col >> 6;
@@ -876,13 +882,10 @@ cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t strea
       !tma_map_3d(&tm_o, a->o_lat, kDc, a->H, n_tok, kDc * 2, (uint64_t)a->H * kDc * 2, 64, 64, 1))
     return cudaErrorInvalidValue;
   if (FP8) {
-    // the e4m3 rows (576 bytes) viewed as two-byte units: (128 units, rows, 2
-    // segments 256 bytes apart); a box of 64 units at unit 64r brings the bytes
-    // 128r .. 128r+127 and 256+128r .. 256+128r+127 of each row
-    const uint64_t dims[3] = {128, rows_kv, 2}, strides[2] = {kRow, 256};
-    const uint32_t box[3] = {64, 64, 2};
-    if (!tma_map_nd(&tm_kv, a->kv_cache, 3, dims, strides, box)) return cudaErrorInvalidValue;
-    tm_ks = tm_kv;  // unused: the score operand's raw rows come by a plain bulk copy
+    // unused: the raw e4m3 rows come by plain bulk copies and the value operand is
+    // copied from the converted score stages
+    memset(&tm_ks, 0, sizeof(tm_ks));
+    tm_kv = tm_ks;
   } else {
     // score operand: (64 values, rows, 9 chunks 128 bytes apart), one box per stage;
     // value operand: (64 values, rows, 4 chunks 128 bytes apart, 2 groups 512 bytes

@@ -38,10 +38,6 @@ MLA_DEVI void mbar_init(uint32_t addr, uint32_t count) {
 }
 MLA_DEVI void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 
-// Arrive (count 1) on a barrier given by its shared::cluster address (own or peer CTA).
-MLA_DEVI void mbar_arrive_cluster(uint32_t addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
-}
 // Arrive (count 1) on a barrier of this or the peer CTA with the default
 // release semantics at CTA scope.
 MLA_DEVI void mbar_arrive_remote(uint32_t addr) {
@@ -54,11 +50,6 @@ MLA_DEVI void mbar_arrive_remote_relaxed(uint32_t addr) {
 }
 MLA_DEVI void mbar_arrive_expect_tx_local(uint32_t addr, uint32_t tx) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(addr), "r"(tx) : "memory");
-}
-MLA_DEVI void mbar_arrive_expect_tx_cluster(uint32_t addr, uint32_t tx) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(addr),
-               "r"(tx)
-               : "memory");
 }
 // try_wait with acquire at CTA scope (TMA bytes and tcgen05 commits) or at
 // cluster scope (arrivals of the peer CTA's threads after their own writes).
@@ -106,15 +97,6 @@ MLA_DEVI bool mbar_wait(uint32_t addr, uint32_t parity, volatile int* abort, uin
   }
 }
 
-// Warp-level form: lane 0 waits, the result is broadcast to the warp.
-template <bool kCluster = false>
-MLA_DEVI bool mbar_wait_warp(uint32_t addr, uint32_t parity, volatile int* abort, uint32_t* status,
-                             uint64_t limit_ns) {
-  int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait<kCluster>(addr, parity, abort, status, limit_ns) ? 1 : 0;
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
 // Converged-warp form: every lane polls, the loop exits uniformly.  Bounded
 // like mbar_wait.
 template <bool kCluster = false>
@@ -141,17 +123,9 @@ MLA_DEVI bool mbar_wait_converged(uint32_t addr, uint32_t parity, volatile int* 
 }
 
 // ---------------------------------------------------------------- TMA
-// 2-D tile load into this CTA's shared memory; completion (bytes) is counted on
-// the barrier at `mbar_cluster`, which may live in the peer CTA of the pair.
-MLA_DEVI void tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t mbar_cluster, int32_t x,
-                               int32_t y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(tmap), "r"(mbar_cluster), "r"(x), "r"(y)
-      : "memory");
-}
-
+// Tile load of the CTA pair (cta_group::2) into this CTA's shared memory;
+// completion (bytes) is counted on the barrier at `mbar_cluster`, which may live
+// in the peer CTA of the pair.  No multicast.
 MLA_DEVI void tma_load_3d_pair(uint32_t dst, const void* tmap, uint32_t mbar_cluster, int32_t x,
                                int32_t y, int32_t z) {
   asm volatile(
@@ -162,16 +136,6 @@ MLA_DEVI void tma_load_3d_pair(uint32_t dst, const void* tmap, uint32_t mbar_clu
 }
 
 // Same, executed by a converged warp: one elected lane issues.
-MLA_DEVI void tma_load_2d_pair_elect(uint32_t dst, const void* tmap, uint32_t mbar_cluster, int32_t x,
-                                     int32_t y) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t.reg .b32 rx;\n\t"
-      "elect.sync rx|e, 0xffffffff;\n\t"
-      "@e cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];\n\t}" ::"r"(dst),
-      "l"(tmap), "r"(mbar_cluster), "r"(x), "r"(y)
-      : "memory");
-}
 MLA_DEVI void tma_load_3d_pair_elect(uint32_t dst, const void* tmap, uint32_t mbar_cluster, int32_t x,
                                      int32_t y, int32_t z) {
   asm volatile(
@@ -203,16 +167,8 @@ MLA_DEVI void mbar_arrive_expect_tx_local_elect(uint32_t addr, uint32_t tx) {
       : "memory");
 }
 
-// 2-D tile load into this CTA's shared memory, completion counted on a barrier
-// of this CTA.
-MLA_DEVI void tma_load_2d_cta(uint32_t dst, const void* tmap, uint32_t mbar, int32_t x, int32_t y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(tmap), "r"(mbar), "r"(x), "r"(y)
-      : "memory");
-}
-
+// Tile loads into this CTA's shared memory, completion counted on a barrier of
+// this CTA.
 MLA_DEVI void tma_load_3d_cta(uint32_t dst, const void* tmap, uint32_t mbar, int32_t x, int32_t y, int32_t z) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
@@ -269,10 +225,6 @@ MLA_DEVI void prefetch_l2_bulk(const void* gaddr, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gaddr), "r"(bytes) : "memory");
 }
 
-MLA_DEVI void prefetch_tmap(const void* tmap) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
-}
-
 // 16-byte shared-memory accesses at 32-bit shared addresses
 MLA_DEVI uint4 lds128(uint32_t addr) {
   uint4 v;
@@ -327,18 +279,9 @@ MLA_DEVI void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
 MLA_DEVI void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 MLA_DEVI void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem] * B[smem], issued for the CTA pair by the even CTA.
-MLA_DEVI void mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Converged-warp forms of the two above: one elected lane issues.
+// D[tmem] (+)= A[smem] * B[smem] for the CTA pair, issued by the even CTA from a
+// converged warp (one elected lane issues).  The commits below use the
+// tcgen05.commit multicast form, which signals barriers (no data movement).
 MLA_DEVI void mma_pair_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                              uint32_t accumulate) {
   asm volatile(
@@ -360,22 +303,14 @@ MLA_DEVI void mma_pair_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Arrive once on the barrier at offset `bar` in every CTA of `cta_mask` when all
+// previously issued tcgen05 operations of this thread have completed.
 MLA_DEVI void commit_pair_mc_elect(uint32_t bar, uint16_t cta_mask) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t.reg .b32 rx;\n\t"
       "elect.sync rx|e, 0xffffffff;\n\t"
       "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
       " [%0], %1;\n\t}" ::"r"(bar),
-      "h"(cta_mask)
-      : "memory");
-}
-
-// Arrive once on the barrier at offset `bar` in every CTA of `cta_mask` when all
-// previously issued tcgen05 operations of this thread have completed.
-MLA_DEVI void commit_pair_mc(uint32_t bar, uint16_t cta_mask) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(bar),
       "h"(cta_mask)
       : "memory");
 }
