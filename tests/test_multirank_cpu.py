@@ -38,7 +38,7 @@ def _worker(rank, world, port, out):
 
 def test_two_ranks_shard_and_take_the_max():
     world, port = 2, _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
