@@ -29,7 +29,8 @@ STATUS = {
 # Every symbol include/mla.h declares.
 EXPORTS = ("mla_absorb_q", "mla_decode_workspace_size", "mla_decode_num_splits",
            "mla_decode_paged", "mla_combine_splits", "mla_up_proj_v", "mla_get_status",
-           "mla_status_string", "mla_decode_paged_noalloc")
+           "mla_status_string", "mla_decode_paged_noalloc", "mla_write_kv_workspace_size",
+           "mla_write_kv")
 
 
 class MlaError(RuntimeError):
@@ -55,6 +56,20 @@ class DecodeArgs(ctypes.Structure):
     ]
 
 
+class WriteKvArgs(ctypes.Structure):
+    """Mirror of ``mla_write_kv_args_t`` (field order and types must match)."""
+    _fields_ = [
+        ("h", ctypes.c_void_p), ("w_dkv", ctypes.c_void_p),
+        ("kv_cache", ctypes.c_void_p), ("kv_scale", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("B", ctypes.c_int32), ("s_q", ctypes.c_int32), ("d_h", ctypes.c_int32),
+        ("d_c", ctypes.c_int32), ("d_r", ctypes.c_int32), ("page_size", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
+        ("kv_dtype", ctypes.c_int32), ("rope_base", ctypes.c_float),
+    ]
+
+
 _lib: Optional[ctypes.CDLL] = None
 
 
@@ -75,6 +90,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_decode_paged.argtypes = [pa, vp]
     lib.mla_combine_splits.argtypes = [pa, vp]
     lib.mla_decode_paged_noalloc.argtypes = [pa, vp]
+    pw = ctypes.POINTER(WriteKvArgs)
+    lib.mla_write_kv_workspace_size.argtypes = [pw, ctypes.POINTER(ctypes.c_size_t)]
+    lib.mla_write_kv.argtypes = [pw, vp]
     lib.mla_get_status.argtypes = [vp, vp]
     lib.mla_status_string.argtypes = [ctypes.c_int]
     lib.mla_status_string.restype = ctypes.c_char_p
@@ -191,6 +209,40 @@ def mla_decode_paged_noalloc(args: DecodeArgs, stream=None):
     _check("mla_decode_paged_noalloc", load().mla_decode_paged_noalloc(ctypes.byref(args), _stream(stream)))
 
 
+def make_write_kv_args(*, h, w_dkv, kv_cache, kv_scale, block_table, seq_lens, workspace=None,
+                       rope_base=10000.0) -> WriteKvArgs:
+    """Fill a ``WriteKvArgs`` from device tensors.  Shapes: h [B][s_q][d_h] bf16,
+    w_dkv [576][d_h] bf16 (W_DKV rows, then W_KR rows), kv_cache [num_pages][64][576]
+    (bf16 or float8_e4m3fn), kv_scale [num_pages][64] fp32 or None,
+    block_table [B][max_pages] int32, seq_lens [B] int32."""
+    import torch
+    B, s_q, d_h = h.shape
+    a = WriteKvArgs()
+    a.h, a.w_dkv = _ptr(h), _ptr(w_dkv)
+    a.kv_cache, a.kv_scale = _ptr(kv_cache), _ptr(kv_scale)
+    a.block_table, a.seq_lens = _ptr(block_table), _ptr(seq_lens)
+    a.B, a.s_q, a.d_h = B, s_q, d_h
+    a.d_c, a.d_r, a.page_size = D_C, D_R, PAGE
+    a.num_pages = kv_cache.shape[0]
+    a.max_pages_per_seq = block_table.shape[1]
+    a.kv_dtype = KV_FP8_E4M3 if kv_cache.dtype == torch.float8_e4m3fn else KV_BF16
+    a.rope_base = float(rope_base)
+    if workspace is not None:
+        a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    return a
+
+
+def mla_write_kv_workspace_size(args: WriteKvArgs) -> int:
+    n = ctypes.c_size_t(0)
+    _check("mla_write_kv_workspace_size", load().mla_write_kv_workspace_size(ctypes.byref(args), ctypes.byref(n)))
+    return int(n.value)
+
+
+def mla_write_kv(args: WriteKvArgs, stream=None):
+    """Appends the new tokens' latent and RoPE key rows to the paged cache."""
+    _check("mla_write_kv", load().mla_write_kv(ctypes.byref(args), _stream(stream)))
+
+
 def mla_get_status(workspace, stream=None) -> int:
     """Waits for the stream and returns (and clears) the device status word."""
     return int(load().mla_get_status(_ptr(workspace), _stream(stream)))
@@ -200,10 +252,11 @@ def mla_status_string(code: int) -> str:
     return load().mla_status_string(int(code)).decode()
 
 
-def alloc_workspace(args: DecodeArgs, device="cuda"):
-    """A zeroed workspace tensor sized for ``args``; also stored into ``args``."""
+def alloc_workspace(args, device="cuda"):
+    """A zeroed workspace tensor sized for ``args`` (``DecodeArgs`` or
+    ``WriteKvArgs``); also stored into ``args``."""
     import torch
-    n = mla_decode_workspace_size(args)
+    n = mla_write_kv_workspace_size(args) if isinstance(args, WriteKvArgs) else mla_decode_workspace_size(args)
     ws = torch.zeros(n, dtype=torch.uint8, device=device)
     args.workspace, args.workspace_bytes = _ptr(ws), n
     return ws

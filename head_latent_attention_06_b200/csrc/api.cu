@@ -1,6 +1,7 @@
 // C ABI of the MLA decode library (declared in include/mla.h): host-side
 // argument validation, split selection, workspace sizing and kernel launches.
 // Nothing here allocates device memory or synchronises, except mla_get_status.
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -17,6 +18,8 @@ bool decode_tc_supported(const mla_decode_args_t*);
 int decode_tc_clusters_per_split(const mla_decode_args_t*);
 int decode_mma_tiles(int len);
 int decode_mma_ctas_per_split(int s_q, int H, int B);
+int write_kv_k_split(int n_tok, int d_h);
+cudaError_t launch_write_kv(const mla_write_kv_args_t*, cudaStream_t);
 }  // namespace mla
 
 using namespace mla;
@@ -96,6 +99,22 @@ int choose_splits(const mla_decode_args_t* a) {
   return s;
 }
 
+mla_status_t check_write_kv_shape(const mla_write_kv_args_t* a) {
+  if (!a) return MLA_ERR_INVALID_VALUE;
+  if (a->B < 0 || a->s_q <= 0 || a->d_h <= 0 || a->num_pages < 0 || a->max_pages_per_seq <= 0)
+    return MLA_ERR_INVALID_VALUE;
+  if ((int64_t)a->B * a->s_q > (1 << 24)) return MLA_ERR_INVALID_VALUE;
+  if (a->d_c != kDc || a->d_r != kDr || a->page_size != kPage || a->d_h % 64 != 0) return MLA_ERR_UNSUPPORTED;
+  if (a->kv_dtype != MLA_KV_BF16 && a->kv_dtype != MLA_KV_FP8_E4M3) return MLA_ERR_UNSUPPORTED;
+  if (!(a->rope_base > 0.f) || !isfinite(a->rope_base)) return MLA_ERR_INVALID_VALUE;
+  return MLA_OK;
+}
+
+size_t write_kv_workspace(const mla_write_kv_args_t* a) {
+  const int n_tok = a->B * a->s_q;
+  return align_up(256 + (size_t)write_kv_k_split(n_tok, a->d_h) * n_tok * kRow * sizeof(float), 256);
+}
+
 }  // namespace
 
 extern "C" {
@@ -167,6 +186,31 @@ mla_status_t mla_combine_splits(const mla_decode_args_t* a, void* stream) {
   st = check_decode_ptrs(a, splits);
   if (st != MLA_OK || a->B == 0 || splits == 1) return st;
   return from_cuda(launch_combine(a, splits, (cudaStream_t)stream));
+}
+
+mla_status_t mla_write_kv_workspace_size(const mla_write_kv_args_t* a, size_t* bytes) {
+  mla_status_t st = check_write_kv_shape(a);
+  if (st != MLA_OK) return st;
+  if (!bytes) return MLA_ERR_INVALID_VALUE;
+  *bytes = write_kv_workspace(a);
+  return MLA_OK;
+}
+
+mla_status_t mla_write_kv(const mla_write_kv_args_t* a, void* stream) {
+  mla_status_t st = check_write_kv_shape(a);
+  if (st != MLA_OK) return st;
+  if (!a->workspace) return MLA_ERR_INVALID_VALUE;
+  if (!aligned16(a->workspace)) return MLA_ERR_MISALIGNED;
+  if (a->workspace_bytes < write_kv_workspace(a)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (a->B == 0) return MLA_OK;
+  if (!a->h || !a->w_dkv || !a->kv_cache || !a->block_table || !a->seq_lens) return MLA_ERR_INVALID_VALUE;
+  if (a->kv_dtype == MLA_KV_FP8_E4M3 && !a->kv_scale) return MLA_ERR_INVALID_VALUE;
+  if (a->num_pages <= 0) return MLA_ERR_INVALID_VALUE;
+  if (!aligned16(a->h) || !aligned16(a->w_dkv) || !aligned16(a->kv_cache)) return MLA_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(a->block_table) & 3u) || (reinterpret_cast<uintptr_t>(a->seq_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(a->kv_scale) & 3u))
+    return MLA_ERR_MISALIGNED;
+  return from_cuda(launch_write_kv(a, (cudaStream_t)stream));
 }
 
 mla_status_t mla_get_status(void* workspace, void* stream) {

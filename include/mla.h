@@ -15,6 +15,8 @@
  *   mla_decode_paged   scores, online softmax, o_lat = P c   (split-KV partials)
  *   mla_combine_splits log-sum-exp merge of the partials     (no-op for 1 split)
  *   mla_up_proj_v      o = W_UV o_lat                         (per head)
+ * and mla_write_kv appends new tokens (latent, RoPE key, bf16 or e4m3) to the
+ * cache before the decode that reads them.
  *
  * Conventions for every entry point:
  *  - Pointers are DEVICE pointers unless a field says otherwise; the caller owns
@@ -46,7 +48,7 @@ typedef enum {
   MLA_ERR_INVALID_VALUE = 1,        /* null pointer, negative or inconsistent size */
   MLA_ERR_UNSUPPORTED = 2,          /* a dimension the library does not handle */
   MLA_ERR_MISALIGNED = 3,           /* a pointer is not 16-byte aligned */
-  MLA_ERR_WORKSPACE_TOO_SMALL = 4,  /* workspace_bytes < mla_decode_workspace_size() */
+  MLA_ERR_WORKSPACE_TOO_SMALL = 4,  /* workspace_bytes below the matching *_workspace_size() */
   MLA_ERR_CUDA = 5,                 /* a CUDA runtime call or launch failed */
   MLA_ERR_DEVICE_TIMEOUT = 6,       /* a bounded device wait ran out (device-side) */
   MLA_ERR_BAD_BLOCK_TABLE = 7,      /* a block-table entry outside [0, num_pages) (device-side) */
@@ -169,6 +171,58 @@ mla_status_t mla_up_proj_v(const void* o_lat, const void* w_uv, void* out,
  * status words are not reported through this entry point.
  */
 mla_status_t mla_decode_paged_noalloc(const mla_decode_args_t* args, void* stream);
+
+/*
+ * Arguments of mla_write_kv / mla_write_kv_workspace_size.
+ * Zero-initialise the struct, then fill every field.
+ */
+typedef struct {
+  const void* h;                  /* bf16 [n_tok][d_h]: hidden states of the new tokens,
+                                     n_tok = B * s_q, token t = b * s_q + i */
+  const void* w_dkv;              /* bf16 [d_c + d_r][d_h]: rows 0 .. d_c-1 are W_DKV, rows
+                                     d_c .. d_c+d_r-1 the RoPE key's projection W_KR */
+  void* kv_cache;                 /* [num_pages][page_size][d_c + d_r], bf16 or e4m3; only the
+                                     new tokens' rows are written */
+  float* kv_scale;                /* fp32 [num_pages][page_size]: e4m3 only, written at the new
+                                     rows; NULL for bf16 */
+  const int32_t* block_table;     /* int32 [B][max_pages_per_seq]: physical page of each
+                                     64-token logical page */
+  const int32_t* seq_lens;        /* int32 [B], device: lengths including the s_q new tokens */
+  void* workspace;                /* device scratch, >= mla_write_kv_workspace_size() bytes,
+                                     16-byte aligned; its first 16 bytes must be zero before the
+                                     first use (they hold the sticky status word) */
+  size_t workspace_bytes;
+  int32_t B, s_q;
+  int32_t d_h;                    /* hidden width, a positive multiple of 64 */
+  int32_t d_c, d_r, page_size;
+  int32_t num_pages;              /* physical pages in kv_cache */
+  int32_t max_pages_per_seq;      /* row length of block_table */
+  int32_t kv_dtype;               /* mla_kv_dtype_t */
+  float rope_base;                /* RoPE frequency base, e.g. 10000 */
+} mla_write_kv_args_t;
+
+/* Bytes of workspace mla_write_kv needs for these arguments (host only). */
+mla_status_t mla_write_kv_workspace_size(const mla_write_kv_args_t* args, size_t* bytes);
+
+/*
+ * mla_write_kv — appends the s_q new tokens of every sequence to the paged
+ * cache.  The latent is the down-projection c = W_DKV h ("MLA: Multi-Head Latent
+ * Attention — DeepSeek-AI Explained", section "Architecture"); beside it goes the
+ * decoupled RoPE key k_pe = RoPE(W_KR h, pos) of the 576-value record (snowgate
+ * thread 35).  RoPE turns value pair (2i, 2i+1) of the key by the angle
+ * pos * rope_base^(-2i/d_r).  New token i of sequence b sits at position
+ * pos = L_b - s_q + i: row pos % page_size of page block_table[b][pos / page_size].
+ * bf16 cache: each value rounded to nearest even.  e4m3 cache (ik_llama.cpp docs
+ * "FlashMLA", "KV cache with MLA": the latent cache may be quantised): one fp32
+ * scale per 576-value row, scale = amax / 448 (1 for an all-zero row), codes =
+ * the fp32 quotients value / scale rounded to nearest even, saturated at +-448.
+ * The projections accumulate in fp32.  No other cache row is touched.  A length
+ * below s_q or beyond the block table (MLA_ERR_BAD_SEQ_LEN) or a page id outside
+ * the cache (MLA_ERR_BAD_BLOCK_TABLE) is recorded in the workspace's status word
+ * and that token is skipped.  Order this call before the decode that reads the
+ * rows, on the same stream.
+ */
+mla_status_t mla_write_kv(const mla_write_kv_args_t* args, void* stream);
 
 /* Waits for `stream`, returns the sticky device status word of `workspace`
  * (MLA_OK if no device-side problem was recorded) and clears it. */

@@ -137,3 +137,67 @@ def test_projection_argument_checks(lib, fn):
 
 def test_get_status_rejects_null(lib):
     assert lib.mla_get_status(None, None) == INVALID
+
+
+# ---------------------------------------------------------------- cache write
+
+def _wargs(B=64, s_q=1, d_h=7168, **kw):
+    a = mla.WriteKvArgs()
+    fake = 0x10000
+    for f in ("h", "w_dkv", "kv_cache", "block_table", "seq_lens"):
+        setattr(a, f, fake)
+    a.B, a.s_q, a.d_h = B, s_q, d_h
+    a.d_c, a.d_r, a.page_size = 512, 64, 64
+    a.num_pages, a.max_pages_per_seq = 4096, 64
+    a.kv_dtype, a.rope_base = 0, 10000.0
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_write_kv_workspace_holds_the_split_partials(lib):
+    # 64 tokens: 9 column tiles of one token block, split 16 ways along d_h
+    assert mla.mla_write_kv_workspace_size(_wargs()) == 256 + 16 * 64 * 576 * 4
+    # 4096 tokens fill the GPU without a split
+    assert mla.mla_write_kv_workspace_size(_wargs(B=2048, s_q=2)) == 256 + 4096 * 576 * 4
+    # never more splits than 64-wide chunks of d_h
+    assert mla.mla_write_kv_workspace_size(_wargs(B=1, d_h=128)) == 256 + 2 * 576 * 4
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("d_c", 256, UNSUPPORTED), ("d_r", 32, UNSUPPORTED), ("page_size", 32, UNSUPPORTED),
+    ("d_h", 100, UNSUPPORTED), ("kv_dtype", 5, UNSUPPORTED), ("d_h", 0, INVALID),
+    ("s_q", 0, INVALID), ("B", -1, INVALID), ("max_pages_per_seq", 0, INVALID),
+    ("rope_base", 0.0, INVALID), ("rope_base", float("nan"), INVALID), ("rope_base", float("inf"), INVALID),
+])
+def test_write_kv_rejects_bad_shapes(lib, field, value, code):
+    a = _wargs(**{field: value})
+    a.workspace, a.workspace_bytes = 0x20000, 1 << 30
+    assert lib.mla_write_kv(ctypes.byref(a), None) == code
+    n = ctypes.c_size_t(0)
+    assert lib.mla_write_kv_workspace_size(ctypes.byref(a), ctypes.byref(n)) == code
+
+
+def test_write_kv_rejects_bad_pointers_and_workspace(lib):
+    a = _wargs()
+    assert lib.mla_write_kv(ctypes.byref(a), None) == INVALID               # no workspace
+    a.workspace, a.workspace_bytes = 0x20008, 1 << 30
+    assert lib.mla_write_kv(ctypes.byref(a), None) == MISALIGNED
+    a.workspace, a.workspace_bytes = 0x20000, 256
+    assert lib.mla_write_kv(ctypes.byref(a), None) == WS_SMALL
+    a.workspace_bytes = 1 << 30
+    a.h = None
+    assert lib.mla_write_kv(ctypes.byref(a), None) == INVALID
+    a.h = 0x10008
+    assert lib.mla_write_kv(ctypes.byref(a), None) == MISALIGNED
+    a.h = 0x10000
+    a.kv_dtype, a.kv_scale = 1, None                                        # e4m3 needs scales
+    assert lib.mla_write_kv(ctypes.byref(a), None) == INVALID
+    a.kv_scale = 0x30002
+    assert lib.mla_write_kv(ctypes.byref(a), None) == MISALIGNED
+
+
+def test_write_kv_with_empty_batch_enqueues_nothing(lib):
+    a = _wargs(B=0)
+    a.workspace, a.workspace_bytes = 0x20000, 256
+    assert lib.mla_write_kv(ctypes.byref(a), None) == OK
