@@ -119,6 +119,28 @@ def _check(fn, code):
         raise MlaError(fn, code)
 
 
+def _want(specs):
+    """Argument check of the tensor builders.  ``specs``: (tensor, name, dtype or
+    tuple of dtypes, shape or None, optional).  Every tensor's dtype, shape and
+    contiguity are checked first, then every tensor's device; the first problem
+    raises ValueError naming the field."""
+    for t, name, dtypes, shape, optional in specs:
+        if t is None:
+            if optional:
+                continue
+            raise ValueError(f"{name} is required")
+        dtypes = dtypes if isinstance(dtypes, tuple) else (dtypes,)
+        if t.dtype not in dtypes:
+            raise ValueError(f"{name}: dtype {t.dtype}, expected {' or '.join(str(d) for d in dtypes)}")
+        if shape is not None and tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    for t, name, _, _, _ in specs:
+        if t is not None and not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+
+
 def _dev(t, dtype, name):
     import torch
     if t is None:
@@ -162,8 +184,21 @@ def make_decode_args(*, q_lat, q_pe, kv_cache, kv_scale, block_table, seq_lens, 
     kv_scale [num_pages][64] fp32 or None, block_table [B][max_pages] int32,
     seq_lens [B] int32, o_lat like q_lat, lse [B][s_q][H] fp32 or None."""
     import torch
+    bf16, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    if q_lat.dim() != 4 or kv_cache.dim() != 3 or block_table.dim() != 2:
+        raise ValueError("q_lat must be [B][s_q][H][512], kv_cache [pages][64][576], block_table [B][pages]")
     B, s_q, H, _ = q_lat.shape
+    P = kv_cache.shape[0]
     fp8 = kv_cache.dtype == torch.float8_e4m3fn
+    _want([(q_lat, "q_lat", bf16, (B, s_q, H, D_C), False),
+           (q_pe, "q_pe", bf16, (B, s_q, H, D_R), False),
+           (kv_cache, "kv_cache", (bf16, torch.float8_e4m3fn), (P, PAGE, D_C + D_R), False),
+           (kv_scale, "kv_scale", f32, (P, PAGE), not fp8),
+           (block_table, "block_table", i32, (B, block_table.shape[1]), False),
+           (seq_lens, "seq_lens", i32, (B,), False),
+           (o_lat, "o_lat", bf16, (B, s_q, H, D_C), False),
+           (lse, "lse", f32, (B, s_q, H), True),
+           (workspace, "workspace", torch.uint8, None, True)])
     a = DecodeArgs()
     a.q_lat, a.q_pe = _ptr(q_lat), _ptr(q_pe)
     a.kv_cache, a.kv_scale = _ptr(kv_cache), _ptr(kv_scale)
@@ -216,7 +251,19 @@ def make_write_kv_args(*, h, w_dkv, kv_cache, kv_scale, block_table, seq_lens, w
     (bf16 or float8_e4m3fn), kv_scale [num_pages][64] fp32 or None,
     block_table [B][max_pages] int32, seq_lens [B] int32."""
     import torch
+    bf16, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    if h.dim() != 3 or kv_cache.dim() != 3 or block_table.dim() != 2:
+        raise ValueError("h must be [B][s_q][d_h], kv_cache [pages][64][576], block_table [B][pages]")
     B, s_q, d_h = h.shape
+    P = kv_cache.shape[0]
+    fp8 = kv_cache.dtype == torch.float8_e4m3fn
+    _want([(h, "h", bf16, (B, s_q, d_h), False),
+           (w_dkv, "w_dkv", bf16, (D_C + D_R, d_h), False),
+           (kv_cache, "kv_cache", (bf16, torch.float8_e4m3fn), (P, PAGE, D_C + D_R), False),
+           (kv_scale, "kv_scale", f32, (P, PAGE), not fp8),
+           (block_table, "block_table", i32, (B, block_table.shape[1]), False),
+           (seq_lens, "seq_lens", i32, (B,), False),
+           (workspace, "workspace", torch.uint8, None, True)])
     a = WriteKvArgs()
     a.h, a.w_dkv = _ptr(h), _ptr(w_dkv)
     a.kv_cache, a.kv_scale = _ptr(kv_cache), _ptr(kv_scale)

@@ -1,0 +1,84 @@
+"""Argument checks of the Python binding's tensor builders (CPU): dtype, shape,
+contiguity and device are checked before any pointer reaches the C ABI."""
+
+import pytest
+import torch
+
+import head_latent_attention_06_b200 as mla
+
+bf16, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+
+
+def _decode_tensors(B=2, s_q=1, H=16, P=8, fp8=False):
+    return dict(
+        q_lat=torch.zeros(B, s_q, H, 512, dtype=bf16), q_pe=torch.zeros(B, s_q, H, 64, dtype=bf16),
+        kv_cache=torch.zeros(P, 64, 576, dtype=torch.float8_e4m3fn if fp8 else bf16),
+        kv_scale=torch.ones(P, 64, dtype=f32) if fp8 else None,
+        block_table=torch.zeros(B, 4, dtype=i32), seq_lens=torch.ones(B, dtype=i32),
+        o_lat=torch.zeros(B, s_q, H, 512, dtype=bf16), lse=torch.zeros(B, s_q, H, dtype=f32))
+
+
+def _write_tensors(B=2, s_q=1, d_h=128, P=8, fp8=False):
+    return dict(
+        h=torch.zeros(B, s_q, d_h, dtype=bf16), w_dkv=torch.zeros(576, d_h, dtype=bf16),
+        kv_cache=torch.zeros(P, 64, 576, dtype=torch.float8_e4m3fn if fp8 else bf16),
+        kv_scale=torch.ones(P, 64, dtype=f32) if fp8 else None,
+        block_table=torch.zeros(B, 4, dtype=i32), seq_lens=torch.ones(B, dtype=i32))
+
+
+def test_decode_args_need_device_tensors():
+    with pytest.raises(ValueError, match="q_lat must be a CUDA tensor"):
+        mla.make_decode_args(**_decode_tensors(), softmax_scale=0.07)
+
+
+@pytest.mark.parametrize("field,bad,msg", [
+    ("q_lat", torch.zeros(2, 1, 16, 512, dtype=f32), "q_lat: dtype"),
+    ("q_pe", torch.zeros(2, 1, 16, 32, dtype=bf16), "q_pe: shape"),
+    ("kv_cache", torch.zeros(8, 32, 576, dtype=bf16), "kv_cache: shape"),
+    ("block_table", torch.zeros(2, 4, dtype=torch.int64), "block_table: dtype"),
+    ("seq_lens", torch.ones(3, dtype=i32), "seq_lens: shape"),
+    ("o_lat", torch.zeros(2, 1, 16, 512, dtype=torch.float16), "o_lat: dtype"),
+    ("lse", torch.zeros(2, 1, 8, dtype=f32), "lse: shape"),
+    ("q_pe", torch.zeros(2, 1, 64, 16, dtype=bf16).transpose(2, 3), "q_pe must be contiguous"),
+])
+def test_decode_args_reject_bad_tensors(field, bad, msg):
+    t = _decode_tensors()
+    t[field] = bad
+    with pytest.raises(ValueError, match=msg):
+        mla.make_decode_args(**t, softmax_scale=0.07)
+
+
+def test_decode_args_fp8_cache_needs_scales():
+    t = _decode_tensors(fp8=True)
+    t["kv_scale"] = None
+    with pytest.raises(ValueError, match="kv_scale is required"):
+        mla.make_decode_args(**t, softmax_scale=0.07)
+    t["kv_scale"] = torch.ones(8, 64, dtype=torch.float64)
+    with pytest.raises(ValueError, match="kv_scale: dtype"):
+        mla.make_decode_args(**t, softmax_scale=0.07)
+
+
+def test_write_kv_args_need_device_tensors():
+    with pytest.raises(ValueError, match="h must be a CUDA tensor"):
+        mla.make_write_kv_args(**_write_tensors())
+
+
+@pytest.mark.parametrize("field,bad,msg", [
+    ("h", torch.zeros(2, 1, 128, dtype=f32), "h: dtype"),
+    ("w_dkv", torch.zeros(512, 128, dtype=bf16), "w_dkv: shape"),
+    ("w_dkv", torch.zeros(576, 64, dtype=bf16), "w_dkv: shape"),
+    ("kv_cache", torch.zeros(8, 64, 512, dtype=bf16), "kv_cache: shape"),
+    ("seq_lens", torch.ones(2, dtype=torch.int64), "seq_lens: dtype"),
+])
+def test_write_kv_args_reject_bad_tensors(field, bad, msg):
+    t = _write_tensors()
+    t[field] = bad
+    with pytest.raises(ValueError, match=msg):
+        mla.make_write_kv_args(**t)
+
+
+def test_write_kv_args_fp8_cache_needs_scales():
+    t = _write_tensors(fp8=True)
+    t["kv_scale"] = None
+    with pytest.raises(ValueError, match="kv_scale is required"):
+        mla.make_write_kv_args(**t)
