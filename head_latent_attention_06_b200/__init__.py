@@ -141,13 +141,11 @@ def _want(specs):
             raise ValueError(f"{name} must be a CUDA tensor")
 
 
-def _dev(t, dtype, name):
-    import torch
-    if t is None:
-        raise ValueError(f"{name} is required")
-    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
-        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
-    return t
+def _tokens(t, name, H, d):
+    """Token count of a [..., H, d] tensor (any leading token dimensions)."""
+    if t.dim() < 2 or tuple(t.shape[-2:]) != (H, d):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected [..., {H}, {d}]")
+    return t.numel() // (H * d)
 
 
 # ------------------------------------------------------------------ entry points
@@ -156,10 +154,12 @@ def mla_absorb_q(q_nope, w_uk, q_lat, stream=None):
     """q_lat[t][h] = W_UK[h]^T q_nope[t][h]; q_nope [n_tok][H][128], w_uk [H][128][512],
     q_lat [n_tok][H][512], all bf16 on the device."""
     import torch
-    for t, n in ((q_nope, "q_nope"), (w_uk, "w_uk"), (q_lat, "q_lat")):
-        _dev(t, torch.bfloat16, n)
     H = w_uk.shape[0]
-    n_tok = q_nope.numel() // (H * D_N)
+    n_tok = _tokens(q_nope, "q_nope", H, D_N)
+    if _tokens(q_lat, "q_lat", H, D_C) != n_tok:
+        raise ValueError("q_lat must hold as many tokens as q_nope")
+    _want([(q_nope, "q_nope", torch.bfloat16, None, False), (w_uk, "w_uk", torch.bfloat16, (H, D_N, D_C), False),
+           (q_lat, "q_lat", torch.bfloat16, None, False)])
     _check("mla_absorb_q", load().mla_absorb_q(_ptr(q_nope), _ptr(w_uk), _ptr(q_lat), n_tok, H,
                                                w_uk.shape[1], w_uk.shape[2], _stream(stream)))
 
@@ -168,10 +168,12 @@ def mla_up_proj_v(o_lat, w_uv, out, stream=None):
     """out[t][h] = W_UV[h] o_lat[t][h]; o_lat [n_tok][H][512], w_uv [H][128][512],
     out [n_tok][H][128], all bf16 on the device."""
     import torch
-    for t, n in ((o_lat, "o_lat"), (w_uv, "w_uv"), (out, "out")):
-        _dev(t, torch.bfloat16, n)
     H = w_uv.shape[0]
-    n_tok = o_lat.numel() // (H * D_C)
+    n_tok = _tokens(o_lat, "o_lat", H, D_C)
+    if _tokens(out, "out", H, D_V) != n_tok:
+        raise ValueError("out must hold as many tokens as o_lat")
+    _want([(o_lat, "o_lat", torch.bfloat16, None, False), (w_uv, "w_uv", torch.bfloat16, (H, D_V, D_C), False),
+           (out, "out", torch.bfloat16, None, False)])
     _check("mla_up_proj_v", load().mla_up_proj_v(_ptr(o_lat), _ptr(w_uv), _ptr(out), n_tok, H,
                                                  w_uv.shape[1], w_uv.shape[2], _stream(stream)))
 

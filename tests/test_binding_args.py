@@ -82,3 +82,22 @@ def test_write_kv_args_fp8_cache_needs_scales():
     t["kv_scale"] = None
     with pytest.raises(ValueError, match="kv_scale is required"):
         mla.make_write_kv_args(**t)
+
+
+def test_projection_calls_check_shapes_before_the_device():
+    H = 4
+    q = torch.zeros(3, H, 128, dtype=bf16)
+    w = torch.zeros(H, 128, 512, dtype=bf16)
+    with pytest.raises(ValueError, match="q_lat must hold as many tokens"):
+        mla.mla_absorb_q(q, w, torch.zeros(2, H, 512, dtype=bf16))
+    with pytest.raises(ValueError, match="w_uk: shape"):
+        mla.mla_absorb_q(q, torch.zeros(H, 128, 256, dtype=bf16), torch.zeros(3, H, 512, dtype=bf16))
+    with pytest.raises(ValueError, match="q_nope: shape"):
+        mla.mla_absorb_q(torch.zeros(3, H, 64, dtype=bf16), w, torch.zeros(3, H, 512, dtype=bf16))
+    with pytest.raises(ValueError, match="q_nope must be a CUDA tensor"):
+        mla.mla_absorb_q(q, w, torch.zeros(3, H, 512, dtype=bf16))
+    x = torch.zeros(3, H, 512, dtype=bf16)
+    with pytest.raises(ValueError, match="out must hold as many tokens"):
+        mla.mla_up_proj_v(x, w, torch.zeros(4, H, 128, dtype=bf16))
+    with pytest.raises(ValueError, match="out: dtype"):
+        mla.mla_up_proj_v(x, w, torch.zeros(3, H, 128, dtype=f32))
