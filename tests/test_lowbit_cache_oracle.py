@@ -1,0 +1,101 @@
+"""Pins for the low-bit cache oracle (``oracle/lowbit_cache.py``).
+
+* the Hadamard matrix against scipy's construction (library routine), its
+  orthonormality and symmetry;
+* folding the rotation into W_DKV, W_UK and W_UV leaves attention unchanged: the
+  rotated cache with the folded weights gives the plain output and lse, and the
+  latent output comes out rotated (an identity of orthonormal matrices);
+* blockwise q8_0 / q4_0: every value within half a step of its block (plus the
+  fp16 rounding of the scale), block extremes on the outermost code, zero blocks,
+  blocks independent of one another;
+* the pages' claim that the rotation helps at low bit widths, on rows with an
+  outlier: the q4_0 error after rotate -> quantise -> rotate back is smaller.
+"""
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+from oracle import lowbit_cache as lb
+from oracle import mla_oracle as om
+
+
+@pytest.mark.parametrize("n", [1, 2, 64, 512])
+def test_hadamard_matches_scipy(n):
+    ref = scipy.linalg.hadamard(n).astype(np.float64) / np.sqrt(n)
+    assert np.array_equal(lb.hadamard(n), ref)
+
+
+def test_hadamard_is_orthonormal_and_symmetric():
+    h = lb.hadamard(512)
+    assert np.allclose(h @ h.T, np.eye(512), atol=1e-12)
+    assert np.array_equal(h, h.T)
+
+
+def test_folded_weights_leave_attention_unchanged():
+    rng = np.random.default_rng(0)
+    H, n, d_h = 4, 150, 96
+    q_nope = rng.standard_normal((H, 128))
+    q_pe = rng.standard_normal((H, 64))
+    w_uk = rng.standard_normal((H, 128, 512)) / np.sqrt(512)
+    w_uv = rng.standard_normal((H, 128, 512)) / np.sqrt(512)
+    w_dkv = rng.standard_normal((512, d_h)) / np.sqrt(d_h)
+    hs = rng.standard_normal((n, d_h))
+    C = np.concatenate([hs @ w_dkv.T, rng.standard_normal((n, 64))], axis=1)
+    scale = 1 / np.sqrt(192)
+    o_lat, lse = om.latent_attention(om.absorb_q(q_nope, w_uk), q_pe, C, scale)
+    o = om.up_proj_v(o_lat, w_uv)
+    f_dkv, f_uk, f_uv = lb.fold_hadamard(w_dkv, w_uk, w_uv)
+    C_rot = lb.rotate_latent(C)
+    # the cache written with the folded W_DKV is the rotated cache
+    assert np.allclose(hs @ f_dkv.T, C_rot[:, :512], atol=1e-12)
+    o_lat2, lse2 = om.latent_attention(om.absorb_q(q_nope, f_uk), q_pe, C_rot, scale)
+    o2 = om.up_proj_v(o_lat2, f_uv)
+    assert np.allclose(lse2, lse, atol=1e-12)
+    assert np.allclose(o2, o, atol=1e-12)
+    assert np.allclose(o_lat2, o_lat @ lb.hadamard(512).T, atol=1e-12)
+
+
+@pytest.mark.parametrize("kind,levels", [("q8_0", 127), ("q4_0", 7)])
+def test_blocks_within_half_a_step(kind, levels):
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal(576) * np.repeat(rng.uniform(1e-3, 1e2, 18), 32)
+    x[32:64] = 0.0                                           # a zero block
+    q, d = lb.quantise_blocks(x, kind)
+    assert q.shape == (576,) and d.shape == (18,)
+    assert np.all(np.abs(q) <= levels)
+    assert d[1] == 0 and np.all(q[32:64] == 0)
+    y = lb.dequantise_blocks(q, d)
+    bound = np.repeat(d / 2 + levels * d * 2.0 ** -10, 32)
+    assert np.all(np.abs(y - x) <= bound)
+    # the largest magnitude of each non-zero block sits on the outermost code
+    for b in range(18):
+        if d[b] > 0:
+            j = 32 * b + np.argmax(np.abs(x[32 * b:32 * b + 32]))
+            assert abs(q[j]) == levels
+    # fp16 scales
+    assert np.array_equal(d, d.astype(np.float16).astype(np.float64))
+
+
+def test_blocks_are_independent():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal(576)
+    q, d = lb.quantise_blocks(x, "q8_0")
+    x2 = x.copy()
+    x2[:32] *= 1000.0                                        # change block 0 only
+    q2, d2 = lb.quantise_blocks(x2, "q8_0")
+    assert np.array_equal(q2[32:], q[32:]) and np.array_equal(d2[1:], d[1:])
+
+
+def test_rotation_reduces_low_bit_error_with_outliers():
+    rng = np.random.default_rng(3)
+    h = lb.hadamard(512)
+    err_plain, err_rot = 0.0, 0.0
+    for _ in range(50):
+        c = rng.standard_normal(512)
+        c[rng.integers(0, 512, 3)] *= 30.0                   # a few outlier channels
+        q, d = lb.quantise_blocks(c, "q4_0")
+        err_plain += np.sum((lb.dequantise_blocks(q, d) - c) ** 2)
+        q, d = lb.quantise_blocks(h @ c, "q4_0")
+        err_rot += np.sum((h.T @ lb.dequantise_blocks(q, d) - c) ** 2)
+    assert err_rot < 0.5 * err_plain
