@@ -237,3 +237,25 @@ def test_tail_rows_of_last_page_are_not_attended():
     inp.kv[page, 6:] = _bf16(np.full((58, 576), 7.0))
     after = om.decode_nonabsorbed(inp)
     np.testing.assert_array_equal(before["o"], after["o"])
+
+
+@pytest.mark.parametrize("name", ["v3", "ragged", "fp8"])
+def test_absorbed_equals_definition_on_full_size_samples(name):
+    """The absorbed mode (the one the full-size GPU comparisons use) agrees with the
+    non-absorbed definition on sampled rows of the full-size workloads: the
+    shortest and longest sequence and one more, two heads each, to 1e-10."""
+    from mla_inputs import preset
+    w = make_workload(preset(name))
+    inp = oracle.from_workload(w)
+    lens = np.asarray(w.lens)
+    bs = sorted({int(np.argmin(lens)), int(np.argmax(lens)), len(lens) // 3})
+    rows = [(b, i) for b in bs for i in range(w.s_q)]
+    heads = [0, w.H - 1]
+    a = om.decode_absorbed(inp, rows=rows, heads=heads)
+    d = om.decode_nonabsorbed(inp, rows=rows, heads=heads)
+    for b, i in rows:
+        for key in ("o", "o_lat"):
+            x, y = a[key][b, i, heads], d[key][b, i, heads]
+            assert np.linalg.norm(x - y) <= 1e-10 * max(np.linalg.norm(y), 1e-300), (name, b, i, key)
+        x, y = a["lse"][b, i, heads], d["lse"][b, i, heads]
+        assert np.all(np.abs(x - y) <= 1e-10 * np.maximum(np.abs(y), 1.0))
