@@ -261,6 +261,77 @@ def run_reference(args):
     return 0
 
 
+WRITE_METRIC = "MLA cache write GB/s (latent + RoPE key into the paged cache) & % of HBM roofline"
+
+
+def run_write_kv(args):
+    """Times mla_write_kv for the new tokens of one decode step of the workload:
+    hidden states of width d_h -> latent c = W_DKV h and rotated RoPE key -> their
+    rows of the paged cache (bf16, or e4m3 with per-row scales).  One GPU; the
+    two launches are replayed from a CUDA graph with L2 flushed before each."""
+    import torch
+    import head_latent_attention_06_b200 as mla
+    from mla_inputs import make_workload, preset
+    torch.cuda.set_device(0)
+    mla.load()
+    spec = preset(args.config)
+    w = make_workload(spec)
+    d_h = args.d_h
+    g = torch.Generator().manual_seed(spec.seed + 1000)
+    h = torch.randn(w.B, w.s_q, d_h, generator=g).to(torch.bfloat16).cuda()
+    w_dkv = (torch.randn(576, d_h, generator=g) / d_h ** 0.5).to(torch.bfloat16).cuda()
+    kv = w.kv_cache.cuda()
+    sc = None if w.kv_scale is None else w.kv_scale.cuda()
+    bt, sl = w.block_table.cuda(), w.seq_lens.cuda()
+    a = mla.make_write_kv_args(h=h, w_dkv=w_dkv, kv_cache=kv, kv_scale=sc, block_table=bt, seq_lens=sl)
+    ws = mla.alloc_workspace(a)
+    stream = torch.cuda.current_stream()
+    mla.mla_write_kv(a)                      # outside capture: one-time host set-up
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        mla.mla_write_kv(a)
+    flush_w = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    flush_r = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    for _ in range(max(3, args.warmup)):
+        flush_w.zero_()
+        torch.sum(flush_r)
+        graph.replay()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    with ClockSampler(0) as clk:
+        for k in range(args.steps):
+            flush_w.zero_()
+            torch.sum(flush_r)
+            evs[k][0].record(stream)
+            graph.replay()
+            evs[k][1].record(stream)
+        torch.cuda.synchronize()
+    assert mla.mla_get_status(ws) == 0
+    ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    n_tok = w.B * w.s_q
+    row_bytes = 1152 if spec.kv_dtype == "bf16" else 580
+    algo_bytes = 576 * d_h * 2 + n_tok * d_h * 2 + n_tok * row_bytes
+    gbs = algo_bytes / (ms * 1e-3) / 1e9
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    cfg = _config_dict(args.config, w)
+    cfg.update({"path": "write_kv", "d_h": d_h, "new_tokens": n_tok})
+    line = {"metric": WRITE_METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 in, fp32 accumulate, " + ("bf16 cache" if spec.kv_dtype == "bf16" else "e4m3 cache"),
+            "data": "synthetic (seeded N(0,1) hidden states, N(0,1/d_h) weights)", "config": cfg,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "traffic": None,
+                         "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                         "kernel": "mla_write_kv (down-projection + finish)",
+                         "bytes_per_launch": algo_bytes},
+            "gpu_launches": 2 * args.steps, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def _config_dict(name, w, splits=None):
     from mla_inputs import preset
     s = preset(name)
@@ -283,9 +354,14 @@ def main(argv=None):
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", default="decode", choices=["decode", "write_kv"],
+                    help="decode: the decode step (default); write_kv: the cache write of its new tokens")
+    ap.add_argument("--d-h", dest="d_h", type=int, default=7168, help="hidden width for --path write_kv")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.path == "write_kv":
+        return run_write_kv(args)
 
     import torch
     import torch.distributed as dist
