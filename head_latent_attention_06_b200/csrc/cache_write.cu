@@ -160,7 +160,10 @@ template <bool FP8>
 __global__ void __launch_bounds__(128) kv_finish_kernel(const FinishParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 4 + warp;
-  pdl_trigger();
+  // No early trigger: the kernels after this one may start only once it has
+  // completed.  The decode reads its first cache page before waiting for its
+  // predecessor, and with an early trigger here a decode two launches later could
+  // start while these rows are still being written.
   pdl_wait();  // the partials come from the previous kernel
   if (t >= p.n_tok) return;
   const int b = t / p.s_q, i = t - b * p.s_q;

@@ -380,8 +380,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
         }
         return true;
       };
-      // The cache, block table and lengths are not written by the kernel this one
-      // may overlap with (the query absorption); q_lat is, so Q waits for it.
+      // The cache, block table and lengths are not written by any kernel this one
+      // may overlap with (the query absorption, or what the absorption overlaps;
+      // the cache write lets nothing after it start early); q_lat is, so Q waits
+      // for its producer.
       // page 0's score stage and Q first: every CTA asks for its first bytes at
       // the same moment, and these two gate the first score MMA; the L2
       // prefetch of the next pages only after them

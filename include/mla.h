@@ -220,7 +220,8 @@ mla_status_t mla_write_kv_workspace_size(const mla_write_kv_args_t* args, size_t
  * below s_q or beyond the block table (MLA_ERR_BAD_SEQ_LEN) or a page id outside
  * the cache (MLA_ERR_BAD_BLOCK_TABLE) is recorded in the workspace's status word
  * and that token is skipped.  Order this call before the decode that reads the
- * rows, on the same stream.
+ * rows, on the same stream: kernels enqueued after it start only once it has
+ * completed (it gives no early start to programmatic dependent launches).
  */
 mla_status_t mla_write_kv(const mla_write_kv_args_t* args, void* stream);
 
