@@ -32,6 +32,13 @@
  *    recorded in the workspace's status word and read by mla_get_status.
  *  - The library is built for sm_100a only; on another device the launch fails
  *    and MLA_ERR_CUDA is returned.
+ *  - Kernels are launched with programmatic dependent launch: one may start while
+ *    the previous kernel on the stream is still running, and waits for it before
+ *    reading anything that kernel may write.  mla_decode_paged reads the cache,
+ *    block table and lengths before that wait, so these must not be written by a
+ *    kernel that lets its dependents start early (no kernel of this library
+ *    that writes them does; a kernel that never signals an early start, the
+ *    default, and copies are safe).
  */
 #ifndef MLA_B200_H
 #define MLA_B200_H
