@@ -72,6 +72,21 @@ def compare_step(step, w, ref, rows=None):
     return res
 
 
+def report(label, res):
+    """Appends the achieved errors of one comparison as a JSON line to the file
+    named by MLA_PARITY_REPORT (nothing when it is unset)."""
+    import json
+    import os
+    path = os.environ.get("MLA_PARITY_REPORT")
+    if not path:
+        return
+    line = {"case": label}
+    for key, (ma, rl) in res.items():
+        line[key] = {"max_abs": ma, "rel_l2": rl}
+    with open(path, "a") as f:
+        f.write(json.dumps(line) + "\n")
+
+
 def oracle_of(w, rows=None, absorbed=False, heads=None):
     inp = oracle.from_workload(w)
     fn = om.decode_absorbed if absorbed else om.decode_nonabsorbed

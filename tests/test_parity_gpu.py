@@ -17,7 +17,7 @@ from mla_inputs import WorkloadSpec, make_workload, preset, PRESETS
 from oracle import mla_oracle as om
 import oracle
 
-from parity_util import TOL, check_close, check_lse, compare_step, errors, oracle_of, to_np
+from parity_util import TOL, check_close, check_lse, compare_step, errors, oracle_of, report, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -66,7 +66,7 @@ def test_small_cases_every_element(cuda_lib, kv, H, s_q, causal, lens, splits):
     w = make_workload(_spec(kv, H, s_q, lens, causal))
     st = _run(cuda_lib, w, splits)
     ref = oracle_of(w, absorbed=True)          # pinned equal to the definition (P1)
-    compare_step(st, w, ref)
+    report(f"small {kv} H={H} s_q={s_q} causal={causal} lens={lens} splits={splits}", compare_step(st, w, ref))
     # and the explicit K/V definition on a few heads of the longest sequence
     b = int(np.argmax(lens))
     heads = [0, H - 1]
@@ -227,7 +227,7 @@ def test_full_size_presets_sampled(cuda_lib, name):
     st = _run(cuda_lib, w)
     rows = _sample_rows(w)
     ref = oracle_of(w, rows=rows, absorbed=True)
-    compare_step(st, w, ref, rows=rows)
+    report(f"full-size {name} (sampled rows)", compare_step(st, w, ref, rows=rows))
     # the explicit-K/V definition on two heads of the first and last sampled row
     for (b, i) in (rows[0], rows[-1]):
         heads = [0, w.H - 1]
