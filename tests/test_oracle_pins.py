@@ -176,6 +176,25 @@ def test_causal_query0_equals_shorter_context():
     np.testing.assert_array_equal(out2["lse"][:, 1], out3["lse"][:, 0])
 
 
+def test_causal_multi_token_equals_single_token_prefixes():
+    """Eight new tokens with the causal mask (a chunked-prefill shape): query i
+    gives exactly the one-query result over the first L - 8 + i + 1 tokens,
+    through the definition itself."""
+    s_q = 8
+    w = _small(s_q=s_q, causal=True, lens=(8, 70, 140), H=2)
+    inp = oracle.from_workload(w)
+    out = om.decode_nonabsorbed(inp)
+    for i in range(s_q):
+        one = oracle.from_workload(w)
+        one.s_q, one.causal = 1, False
+        one.q_nope = inp.q_nope[:, i:i + 1].copy()
+        one.q_pe = inp.q_pe[:, i:i + 1].copy()
+        one.seq_lens = inp.seq_lens - s_q + i + 1
+        ref = om.decode_nonabsorbed(one)
+        for k in ("o", "o_lat", "lse"):
+            np.testing.assert_array_equal(out[k][:, i], ref[k][:, 0])
+
+
 # ---------------------------------------------------------------- P6 paging invariance
 
 @pytest.mark.parametrize("kv", ["bf16", "fp8"])
