@@ -29,8 +29,11 @@ STATUS = {
 # Every symbol include/mla.h declares.
 EXPORTS = ("mla_absorb_q", "mla_decode_workspace_size", "mla_decode_num_splits",
            "mla_decode_paged", "mla_combine_splits", "mla_up_proj_v", "mla_get_status",
-           "mla_status_string", "mla_decode_paged_noalloc", "mla_write_kv_workspace_size",
-           "mla_write_kv")
+           "mla_status_string", "mla_decode_paged_noalloc", "mla_noalloc_init",
+           "mla_get_status_noalloc", "mla_write_kv_workspace_size", "mla_write_kv",
+           "mla_set_decode_kernel")
+
+DECODE_AUTO, DECODE_WARP_MMA = 0, 1
 
 
 class MlaError(RuntimeError):
@@ -90,6 +93,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_decode_paged.argtypes = [pa, vp]
     lib.mla_combine_splits.argtypes = [pa, vp]
     lib.mla_decode_paged_noalloc.argtypes = [pa, vp]
+    lib.mla_noalloc_init.argtypes = []
+    lib.mla_get_status_noalloc.argtypes = [vp]
+    lib.mla_set_decode_kernel.argtypes = [i32]
     pw = ctypes.POINTER(WriteKvArgs)
     lib.mla_write_kv_workspace_size.argtypes = [pw, ctypes.POINTER(ctypes.c_size_t)]
     lib.mla_write_kv.argtypes = [pw, vp]
@@ -244,6 +250,23 @@ def mla_decode_paged_noalloc(args: DecodeArgs, stream=None):
     """Decode plus split merge with the library's built-in scratch (args.workspace is
     ignored); for callers that cannot allocate device memory."""
     _check("mla_decode_paged_noalloc", load().mla_decode_paged_noalloc(ctypes.byref(args), _stream(stream)))
+
+
+def mla_noalloc_init():
+    """Set-up of the built-in scratch on the current device (address lookup, status
+    word zeroed); call at start-up, before any stream capture."""
+    _check("mla_noalloc_init", load().mla_noalloc_init())
+
+
+def mla_get_status_noalloc(stream=None) -> int:
+    """Waits for the stream and returns (and clears) the built-in scratch's device
+    status word."""
+    return int(load().mla_get_status_noalloc(_stream(stream)))
+
+
+def mla_set_decode_kernel(kernel: int):
+    """Process-wide decode kernel choice: DECODE_AUTO or DECODE_WARP_MMA."""
+    _check("mla_set_decode_kernel", load().mla_set_decode_kernel(int(kernel)))
 
 
 def make_write_kv_args(*, h, w_dkv, kv_cache, kv_scale, block_table, seq_lens, workspace=None,

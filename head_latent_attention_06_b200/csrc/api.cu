@@ -26,8 +26,6 @@ using namespace mla;
 
 namespace {
 
-constexpr int kNumSMs = 148;
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 mla_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
@@ -48,7 +46,7 @@ mla_status_t check_decode_shape(const mla_decode_args_t* a) {
   if (a->B < 0 || a->H <= 0 || a->s_q <= 0 || a->num_pages < 0 || a->max_pages_per_seq <= 0)
     return MLA_ERR_INVALID_VALUE;
   if (a->d_c != kDc || a->d_r != kDr || a->page_size != kPage) return MLA_ERR_UNSUPPORTED;
-  if (a->H % 16 != 0 || a->H > 128 || a->s_q > 2) return MLA_ERR_UNSUPPORTED;
+  if (a->H % 16 != 0 || a->H > 128 || a->s_q > MLA_MAX_S_Q) return MLA_ERR_UNSUPPORTED;
   if (a->kv_dtype != MLA_KV_BF16 && a->kv_dtype != MLA_KV_FP8_E4M3) return MLA_ERR_UNSUPPORTED;
   if (a->num_splits < 0 || a->num_splits > MLA_MAX_SPLITS) return MLA_ERR_INVALID_VALUE;
   if (a->max_seq_len < 0) return MLA_ERR_INVALID_VALUE;
@@ -56,13 +54,14 @@ mla_status_t check_decode_shape(const mla_decode_args_t* a) {
   return MLA_OK;
 }
 
+// Process-wide kernel choice (mla_set_decode_kernel).
+std::atomic<int32_t> g_decode_kernel{MLA_DECODE_AUTO};
+
+bool forced_mma() { return g_decode_kernel.load(std::memory_order_relaxed) == MLA_DECODE_WARP_MMA; }
+
 // Which decode kernel runs: the tensor-memory kernel for the shapes it takes,
-// else the warp-MMA kernel.  MLA_DECODE_KERNEL=mma forces the latter (testing).
-bool use_tc(const mla_decode_args_t* a) {
-  const char* env = getenv("MLA_DECODE_KERNEL");
-  if (env && strcmp(env, "mma") == 0) return false;
-  return decode_tc_supported(a);
-}
+// else the warp-MMA kernel.
+bool use_tc(const mla_decode_args_t* a) { return !forced_mma() && decode_tc_supported(a); }
 
 // Split count.  Tensor-memory kernel: the count that minimises the modelled
 // makespan (waves of 74 CTA pairs x per-unit work), preferring fewer splits.  Warp-MMA
@@ -73,7 +72,7 @@ int choose_splits(const mla_decode_args_t* a) {
   if (use_tc(a)) {
     const int tiles = (max_len + kPage - 1) / kPage;
     const int units = decode_tc_clusters_per_split(a) > 0 ? decode_tc_clusters_per_split(a) : 1;
-    const int slots = kNumSMs / 2;
+    const int slots = device_sm_count() / 2;
     int best = 1;
     long best_cost = -1;
     for (int s = 1; s <= MLA_MAX_SPLITS && s <= (tiles > 0 ? tiles : 1); ++s) {
@@ -90,7 +89,7 @@ int choose_splits(const mla_decode_args_t* a) {
   }
   const int tiles = decode_mma_tiles(max_len);
   const int ctas = decode_mma_ctas_per_split(a->s_q, a->H, a->B > 0 ? a->B : 1);
-  int s = (kNumSMs + ctas - 1) / ctas;
+  int s = (device_sm_count() + ctas - 1) / ctas;
   int cap = tiles / 8;
   if (cap < 1) cap = 1;
   if (s > cap) s = cap;
@@ -225,6 +224,12 @@ mla_status_t mla_get_status(void* workspace, void* stream) {
     if (cudaStreamSynchronize(s) != cudaSuccess) return MLA_ERR_CUDA;
   }
   return (mla_status_t)word;
+}
+
+mla_status_t mla_set_decode_kernel(int32_t kernel) {
+  if (kernel != MLA_DECODE_AUTO && kernel != MLA_DECODE_WARP_MMA) return MLA_ERR_INVALID_VALUE;
+  g_decode_kernel.store(kernel, std::memory_order_relaxed);
+  return MLA_OK;
 }
 
 const char* mla_status_string(mla_status_t s) {

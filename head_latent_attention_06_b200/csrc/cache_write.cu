@@ -82,11 +82,13 @@ __global__ void __launch_bounds__(kWThreads) kv_down_proj_kernel(const __grid_co
   auto load_h = [&](int kc, int s) {
     tma_load_2d_local(sa + s * kWStage, &tm_h, bar0 + 8 * s, (c_begin + kc) * kWK, t0);
   };
+  int issued = 0;  // chunks whose loads thread 0 has issued
   if (tid == 0) {
     for (int s = 0; s < kWStages && s < nk; ++s) {
       mbar_arrive_expect_tx_local(bar0 + 8 * s, kWStage);
       load_w(s, s);
     }
+    issued = min(kWStages, nk);
   }
   pdl_wait();
   if (tid == 0)
@@ -130,6 +132,17 @@ __global__ void __launch_bounds__(kWThreads) kv_down_proj_kernel(const __grid_co
       mbar_arrive_expect_tx_local(bar0 + 8 * s, kWStage);
       load_w(next, s);
       load_h(next, s);
+      ++issued;
+    }
+  }
+  // A wait that ran out may leave loads in flight.  Before the CTA exits (and its
+  // shared memory goes to another CTA) the issuing thread waits, bounded again,
+  // for the last load issued into every stage: a stage's phases complete in order.
+  if (__syncthreads_or(aborted) && tid == 0) {
+    for (int s = 0; s < kWStages && s < issued; ++s) {
+      const int last = s + ((issued - 1 - s) / kWStages) * kWStages;
+      int give_up = 0;
+      mbar_wait(bar0 + 8 * s, (last / kWStages) & 1, &give_up, nullptr, kWriteWaitNs);
     }
   }
 
@@ -251,17 +264,13 @@ cudaError_t launch_write_kv(const mla_write_kv_args_t* a, cudaStream_t stream) {
   unsigned char* ws = static_cast<unsigned char*>(a->workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   float* part = reinterpret_cast<float*>(ws + 256);
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kv_down_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kWSmem);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
-  }
+  static PerDeviceOnce attrs;
+  cudaError_t e = once_per_device(attrs, [&]() {
+    return cudaFuncSetAttribute(kv_down_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWSmem);
+  });
+  if (e != cudaSuccess) return e;
   dim3 grid((n_tok + kWTok - 1) / kWTok, ks, kRow / kWCols);
-  cudaError_t e = launch_pdl(kv_down_proj_kernel, grid, dim3(kWThreads), kWSmem, stream, tm_h, tm_w, part,
+  e = launch_pdl(kv_down_proj_kernel, grid, dim3(kWThreads), kWSmem, stream, tm_h, tm_w, part,
                              n_tok, a->d_h / kWK, status);
   if (e != cudaSuccess) return e;
   FinishParams p;

@@ -6,6 +6,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/mla.h"
 
 #define MLA_DEVI __device__ __forceinline__
@@ -62,6 +65,45 @@ inline cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cud
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// One-time host set-up per device (kernel attributes and the like): `fn` runs
+// with the device current, under a lock, until it has succeeded once on that
+// device; later calls return at once.  Safe to call from several host threads.
+struct PerDeviceOnce {
+  static constexpr int kMaxDevices = 64;
+  std::mutex mu;
+  std::atomic<bool> done[kMaxDevices] = {};
+};
+
+template <typename Fn>
+inline cudaError_t once_per_device(PerDeviceOnce& once, Fn fn) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= PerDeviceOnce::kMaxDevices) return fn();  // not cached, still correct
+  if (once.done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  std::lock_guard<std::mutex> lock(once.mu);
+  if (once.done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+  e = fn();
+  if (e == cudaSuccess) once.done[dev].store(true, std::memory_order_release);
+  return e;
+}
+
+// Number of SMs of the current device, queried once per device (148 on a B200).
+inline int device_sm_count() {
+  static PerDeviceOnce once;
+  static std::atomic<int> count[PerDeviceOnce::kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= PerDeviceOnce::kMaxDevices) return 148;
+  once_per_device(once, [&]() {
+    int n = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess && n > 0) count[dev].store(n, std::memory_order_relaxed);
+    return e;
+  });
+  const int n = count[dev].load(std::memory_order_relaxed);
+  return n > 0 ? n : 148;
 }
 
 MLA_DEVI void set_status(uint32_t* status, uint32_t code) {

@@ -367,19 +367,18 @@ cudaError_t launch_decode_mma(const mla_decode_args_t* a, int splits, cudaStream
   p.scale_log2 = a->softmax_scale * kLog2e;
   const int groups = (a->s_q * a->H + ROWS - 1) / ROWS;
   dim3 grid(groups, splits, a->B);
-  cudaError_t e;
-  if (a->kv_dtype == MLA_KV_FP8_E4M3) {
-    e = cudaFuncSetAttribute(decode_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)Smem<true>::total);
-    if (e != cudaSuccess) return e;
+  static PerDeviceOnce attrs;
+  cudaError_t e = once_per_device(attrs, [&]() {
+    cudaError_t e2 = cudaFuncSetAttribute(decode_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)Smem<true>::total);
+    if (e2 != cudaSuccess) return e2;
+    return cudaFuncSetAttribute(decode_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)Smem<false>::total);
+  });
+  if (e != cudaSuccess) return e;
+  if (a->kv_dtype == MLA_KV_FP8_E4M3)
     return launch_pdl(decode_mma_kernel<true>, grid, dim3(NTHREADS), Smem<true>::total, stream, p);
-  } else {
-    e = cudaFuncSetAttribute(decode_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)Smem<false>::total);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(decode_mma_kernel<false>, grid, dim3(NTHREADS), Smem<false>::total, stream, p);
-  }
-  return cudaGetLastError();
+  return launch_pdl(decode_mma_kernel<false>, grid, dim3(NTHREADS), Smem<false>::total, stream, p);
 }
 
 int decode_mma_tiles(int len) { return (len + TT - 1) / TT; }

@@ -10,10 +10,11 @@
 //
 // The array lives in device global memory on every GPU that loads the library,
 // for the lifetime of the process.  Every call shares it and it keeps the last
-// call's contents: the status word is cleared at the start of each call, the
-// partials are always written before they are read.  Two calls whose work
-// overlaps on the GPU (different streams, no ordering between them) race on the
-// array; order them on one stream or with events.
+// call's contents: the status word is zeroed once at set-up and then only by
+// mla_get_status_noalloc (it is sticky, like a workspace's), the partials are
+// always written before they are read.  Two calls whose work overlaps on the GPU
+// (different streams, no ordering between them) race on the array; order them on
+// one stream or with events.
 #include <mutex>
 
 #include "common.cuh"
@@ -30,7 +31,8 @@ void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_scratch on the current device.  In host code the symbol
 // name is only a host-side stand-in; the address must come from
-// cudaGetSymbolAddress, once per device, with that device current.
+// cudaGetSymbolAddress, once per device, with that device current.  The first
+// lookup on a device also zeroes the status word (synchronously).
 mla_status_t scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
@@ -38,6 +40,7 @@ mla_status_t scratch_address(void** out) {
   if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) return MLA_ERR_CUDA;
+    if (cudaMemset(p, 0, 16) != cudaSuccess) return MLA_ERR_CUDA;
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];
@@ -45,6 +48,11 @@ mla_status_t scratch_address(void** out) {
 }
 
 }  // namespace
+
+extern "C" mla_status_t mla_noalloc_init(void) {
+  void* scratch = nullptr;
+  return scratch_address(&scratch);
+}
 
 extern "C" mla_status_t mla_decode_paged_noalloc(const mla_decode_args_t* args, void* stream) {
   if (!args) return MLA_ERR_INVALID_VALUE;
@@ -60,9 +68,14 @@ extern "C" mla_status_t mla_decode_paged_noalloc(const mla_decode_args_t* args, 
   if (st != MLA_OK) return st;
   a.workspace = scratch;
   a.workspace_bytes = kStaticScratchBytes;
-  // the sticky status word must start at zero for this call
-  if (cudaMemsetAsync(scratch, 0, 16, (cudaStream_t)stream) != cudaSuccess) return MLA_ERR_CUDA;
   st = mla_decode_paged(&a, stream);
   if (st != MLA_OK) return st;
   return mla_combine_splits(&a, stream);
+}
+
+extern "C" mla_status_t mla_get_status_noalloc(void* stream) {
+  void* scratch = nullptr;
+  mla_status_t st = scratch_address(&scratch);
+  if (st != MLA_OK) return st;
+  return mla_get_status(scratch, stream);
 }

@@ -279,13 +279,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FP8 ? kThreadsFp8 : 
   const bool bad_len = L_in < 0 || L_in > p.max_pages * kPage;
   const int L = bad_len ? 0 : L_in;
   if (bad_len && threadIdx.x == 0 && r == 0 && g == 0 && split == 0) set_status(p.status, MLA_ERR_BAD_SEQ_LEN);
-  const int n_tiles = (L + kPage - 1) / kPage;
+  // tokens this query sees: a causal query stops at its own position, so its
+  // work unit covers only the pages up to there
+  const int vis = p.causal ? max(0, L - p.s_q + g + 1) : L;
+  const int n_tiles = (vis + kPage - 1) / kPage;
   const int per = (n_tiles + p.splits - 1) / p.splits;
   const int t0 = min(n_tiles, split * per);
   const int t1 = min(n_tiles, t0 + per);
   const int n = t1 - t0;
-  const int j_end = min(L, t1 * kPage);
-  const int vis = p.causal ? L - p.s_q + g + 1 : L;
+  const int j_end = min(vis, t1 * kPage);
 
   if (warp == 0) {
     // =========================== TMA producer ===========================
@@ -922,16 +924,13 @@ cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t strea
   p.splits = splits;
   p.scale_log2 = a->softmax_scale * kLog2e;
   auto kern = decode_tc_kernel<FP8>;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
-  }
+  static PerDeviceOnce attrs;
+  cudaError_t e = once_per_device(attrs, [&]() {
+    cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e2 != cudaSuccess) return e2;
+    return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  });
+  if (e != cudaSuccess) return e;
   dim3 grid(2 * splits, a->s_q, a->B);
   return launch_pdl(kern, grid, dim3(FP8 ? kThreadsFp8 : kThreadsBf16), kSmemBytes, stream, tm_q, tm_qpe, tm_ks,
                     tm_kv, tm_o, p);

@@ -178,14 +178,10 @@ cudaError_t launch_proj(const void* X, const void* W, void* Y, int n_tok, int H,
                        : tma_map_2d(&tm_w, W, K, (uint64_t)H * N, (uint64_t)K * 2, 64, NC);
   if (!ok) return cudaErrorInvalidValue;
   auto kern = proj_kernel<K, N, NC, W_KN, STAGES>;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::smem);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
-  }
+  static PerDeviceOnce attrs;
+  cudaError_t e = once_per_device(
+      attrs, [&]() { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::smem); });
+  if (e != cudaSuccess) return e;
   dim3 grid((n_tok + TM - 1) / TM, H, N / NC);
   return launch_pdl(kern, grid, dim3(C::NT), C::smem, stream, tm_x, tm_w, static_cast<__nv_bfloat16*>(Y),
                     n_tok, H);

@@ -3,9 +3,9 @@
  *
  * Multi-Head Latent Attention decode over a paged latent KV cache.  Every cached
  * token holds one latent c (d_c = 512 values) followed by a decoupled RoPE key
- * k_pe (d_r = 64 values), shared by all heads: the 576-value record of the
- * snowgate forum thread 35 (replies on the latent record, "512-dim + 64-dim
- * rope").  Keys and values are up-projections of the latent, k = W_UK c and
+ * k_pe (d_r = 64 values), shared by all heads: the 576-value record worked
+ * out in snowgate forum thread 35 (replies on the KV-cache arithmetic).  Keys
+ * and values are up-projections of the latent, k = W_UK c and
  * v = W_UV c ("MLA: Multi-Head Latent Attention — DeepSeek-AI Explained",
  * section "Architecture"); decode never forms them, it folds W_UK into the query
  * and W_UV into the output (nnets.ru article, section "Суть MLA", the weight
@@ -65,17 +65,21 @@ typedef enum {
 typedef enum { MLA_KV_BF16 = 0, MLA_KV_FP8_E4M3 = 1 } mla_kv_dtype_t;
 
 /* Supported dimensions: d_c = 512, d_r = 64, d_n = d_v = 128, page_size = 64,
- * H a multiple of 16 up to 128, s_q in {1, 2}. */
+ * H a multiple of 16 up to 128, 1 <= s_q <= MLA_MAX_S_Q.  s_q > 1 covers
+ * speculative decoding and chunked prefill in the absorbed form: every query
+ * token is computed like a decode query (causal among the new tokens when
+ * `causal` is set). */
 #define MLA_D_C 512
 #define MLA_D_R 64
 #define MLA_D_QK_NOPE 128
 #define MLA_D_V 128
 #define MLA_PAGE_SIZE 64
 #define MLA_MAX_SPLITS 128
+#define MLA_MAX_S_Q 1024
 
 /*
  * mla_absorb_q — weight absorption of the query (nnets.ru article, section
- * "Суть MLA"; snowgate thread 35, "W_UK absorbing the query").
+ * "Суть MLA"; snowgate thread 35, the reply on folding W_UK into the query).
  *   q_lat[t][h][c] = sum_n q_nope[t][h][n] * w_uk[h][n][c]
  * q_nope : bf16 [n_tok][H][d_n]        (n_tok = B * s_q, token t = b * s_q + i)
  * w_uk   : bf16 [H][d_n][d_c]          (k = W_UK[h] c, so W_UK[h] is d_n x d_c)
@@ -170,14 +174,30 @@ mla_status_t mla_up_proj_v(const void* o_lat, const void* w_uv, void* out,
  * instead: 16 MiB of device memory on every GPU that loads the library, held
  * until the process exits.  A problem needing more scratch than that (see
  * mla_decode_workspace_size) is rejected with MLA_ERR_WORKSPACE_TOO_SMALL
- * before anything is enqueued.  The first call on a device looks up the
- * array's device address (cudaGetSymbolAddress); make that first call before
- * any stream capture.  Every call shares the array: calls that overlap on the
- * GPU race, so order them on one stream or with events.  The call allocates
- * nothing (it clears the array's status word with cudaMemsetAsync); device-side
- * status words are not reported through this entry point.
+ * before anything is enqueued.  The first use on a device looks up the
+ * array's device address (cudaGetSymbolAddress) and clears its status word;
+ * under CUDA's lazy module loading that lookup may be the moment the driver
+ * loads the library's device code and backs the array, so make it during
+ * start-up, before any allocation freeze or stream capture: call
+ * mla_noalloc_init once per device (or make a first decode call then).
+ * Every call shares the array: calls that overlap on the GPU race, so order
+ * them on one stream or with events.  The call allocates nothing.  Problems
+ * only the device sees (a page id outside the cache, a length beyond the block
+ * table, a wait that ran out) go to the array's sticky status word, read and
+ * cleared by mla_get_status_noalloc.
  */
 mla_status_t mla_decode_paged_noalloc(const mla_decode_args_t* args, void* stream);
+
+/* Set-up of mla_decode_paged_noalloc's built-in scratch on the current device:
+ * looks up its device address and zeroes its status word (synchronously).
+ * Idempotent; call it at start-up on every device that will decode without a
+ * workspace. */
+mla_status_t mla_noalloc_init(void);
+
+/* Waits for `stream`, returns the sticky device status word of the built-in
+ * scratch of the current device (MLA_OK if mla_decode_paged_noalloc recorded no
+ * device-side problem since the last read) and clears it. */
+mla_status_t mla_get_status_noalloc(void* stream);
 
 /*
  * Arguments of mla_write_kv / mla_write_kv_workspace_size.
@@ -235,6 +255,14 @@ mla_status_t mla_write_kv(const mla_write_kv_args_t* args, void* stream);
 /* Waits for `stream`, returns the sticky device status word of `workspace`
  * (MLA_OK if no device-side problem was recorded) and clears it. */
 mla_status_t mla_get_status(void* workspace, void* stream);
+
+/* Which decode kernel mla_decode_paged runs, process-wide.  MLA_DECODE_AUTO
+ * (the default) picks the tensor-memory (tcgen05) kernel for every shape it
+ * takes and the warp-MMA kernel otherwise; MLA_DECODE_WARP_MMA forces the
+ * latter (a cross-check for tests and diagnosis).  Takes effect for calls made
+ * after it returns; a CUDA graph keeps the kernels it captured. */
+typedef enum { MLA_DECODE_AUTO = 0, MLA_DECODE_WARP_MMA = 1 } mla_decode_kernel_t;
+mla_status_t mla_set_decode_kernel(int32_t kernel);
 
 /* Human-readable name of a status code (static storage). */
 const char* mla_status_string(mla_status_t status);

@@ -249,7 +249,3 @@ def combine_splits(o_parts: np.ndarray, lse_parts: np.ndarray):
     o = (wn[..., None] * o_parts).sum(axis=0)
     return o, lse
 
-
-def latent_attention_range(q_lat, q_pe, C, scale, j0: int, j1: int):
-    """Partial (o_lat, lse) of latent attention restricted to rows j0 <= j < j1."""
-    return latent_attention(q_lat, q_pe, C[j0:j1], scale)

@@ -85,7 +85,7 @@ def test_auto_split_count(lib):
 
 @pytest.mark.parametrize("field,value,code", [
     ("d_c", 256, UNSUPPORTED), ("d_r", 32, UNSUPPORTED), ("page_size", 32, UNSUPPORTED),
-    ("H", 24, UNSUPPORTED), ("H", 256, UNSUPPORTED), ("s_q", 3, UNSUPPORTED),
+    ("H", 24, UNSUPPORTED), ("H", 256, UNSUPPORTED), ("s_q", 1025, UNSUPPORTED),
     ("kv_dtype", 5, UNSUPPORTED), ("H", 0, INVALID), ("s_q", 0, INVALID), ("B", -1, INVALID),
     ("num_splits", 129, INVALID), ("max_pages_per_seq", 0, INVALID),
 ])

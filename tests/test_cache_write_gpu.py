@@ -78,9 +78,55 @@ CASES = [
 ]
 
 
+def _full_size_inputs(B, s_q, d_h, L, kv_dtype, seed=23):
+    """The new tokens of one decode step of a full-size workload (every sequence
+    L cached tokens, hidden width d_h).  Only the pages the new rows land in
+    matter to the write, so the cache holds 2 pages per sequence: each
+    sequence's last logical page maps to a page of its own, its other logical
+    pages to arbitrary ones (never written)."""
+    g = torch.Generator().manual_seed(seed)
+    max_pages = (L + 63) // 64
+    num_pages = 2 * B + 3
+    perm = torch.randperm(num_pages, generator=g).to(torch.int32)
+    bt = torch.randint(0, num_pages, (B, max_pages), generator=g, dtype=torch.int32)
+    bt[:, (L - s_q) // 64:] = perm[:B, None]          # the pages the new rows land in
+    h = torch.randn(B, s_q, d_h, generator=g).to(torch.bfloat16)
+    w = (torch.randn(576, d_h, generator=g) / d_h ** 0.5).to(torch.bfloat16)
+    if kv_dtype == "bf16":
+        kv = torch.randn(num_pages, 64, 576, generator=g).to(torch.bfloat16)
+        scale = None
+    else:
+        kv = torch.randn(num_pages, 64, 576, generator=g).to(torch.float8_e4m3fn)
+        scale = torch.rand(num_pages, 64, generator=g) + 0.5
+    return h, w, kv, scale, bt, torch.full((B,), L, dtype=torch.int32)
+
+
+FULL_SIZE = [
+    # the decode workloads' new tokens at a DeepSeek-V3-sized hidden width: 112
+    # K chunks of 64, split 16 ways, so every CTA's 4-stage chunk ring wraps
+    ("bf16", 64, 1, 7168, 4096),
+    ("fp8", 128, 2, 7168, 8192),
+]
+
+
+@pytest.mark.parametrize("kv_dtype,B,s_q,d_h,L", FULL_SIZE)
+def test_write_kv_full_size(cuda_lib, kv_dtype, B, s_q, d_h, L):
+    a = cuda_lib.WriteKvArgs()
+    a.B, a.s_q, a.d_h, a.d_c, a.d_r, a.page_size = B, s_q, d_h, 512, 64, 64
+    a.num_pages, a.max_pages_per_seq, a.rope_base = 1, 1, 10000.0
+    k_split = (cuda_lib.mla_write_kv_workspace_size(a) - 256) // (B * s_q * 576 * 4)
+    assert d_h // 64 > 4 * k_split          # more K chunks per CTA than ring stages
+    h, w, kv, scale, bt, sl = _full_size_inputs(B, s_q, d_h, L, kv_dtype)
+    _check_write(cuda_lib, h, w, kv, scale, bt, sl, kv_dtype, s_q)
+
+
 @pytest.mark.parametrize("kv_dtype,B,s_q,d_h,lens", CASES)
 def test_write_kv_matches_oracle(cuda_lib, kv_dtype, B, s_q, d_h, lens):
     h, w, kv, scale, bt, sl = _inputs(B, s_q, d_h, lens, kv_dtype)
+    _check_write(cuda_lib, h, w, kv, scale, bt, sl, kv_dtype, s_q)
+
+
+def _check_write(cuda_lib, h, w, kv, scale, bt, sl, kv_dtype, s_q):
     kv_g, sc_g, status = _run(cuda_lib, h, w, kv, scale, bt, sl)
     assert status == 0
     exact = _exact_rows(h, w, bt, sl, s_q)

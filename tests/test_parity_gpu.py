@@ -77,11 +77,14 @@ def test_small_cases_every_element(cuda_lib, kv, H, s_q, causal, lens, splits):
 
 
 @pytest.mark.parametrize("lens,splits", [([1, 63, 64, 65, 200, 1000], 1), ([700, 3], 4)])
-def test_warp_mma_kernel_on_128_heads(cuda_lib, monkeypatch, lens, splits):
+def test_warp_mma_kernel_on_128_heads(cuda_lib, lens, splits):
     """The portable warp-MMA kernel, forced for a shape the tensor-memory kernel takes."""
-    monkeypatch.setenv("MLA_DECODE_KERNEL", "mma")
     w = make_workload(_spec("bf16", 128, 1, lens))
-    st = _run(cuda_lib, w, splits)
+    cuda_lib.mla_set_decode_kernel(cuda_lib.DECODE_WARP_MMA)
+    try:
+        st = _run(cuda_lib, w, splits)
+    finally:
+        cuda_lib.mla_set_decode_kernel(cuda_lib.DECODE_AUTO)
     compare_step(st, w, oracle_of(w, absorbed=True))
 
 

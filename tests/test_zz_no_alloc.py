@@ -57,3 +57,21 @@ def test_noalloc_rejects_problems_beyond_its_scratch(cuda_lib):
     a.num_pages, a.max_pages_per_seq = 1024, 64
     a.num_splits, a.softmax_scale = 16, 0.07       # 512*2*128*16 partial rows: 1 GiB of scratch
     assert cuda_lib.load().mla_decode_paged_noalloc(ctypes.byref(a), None) == 4
+
+
+def test_noalloc_reports_device_status_through_its_accessor(cuda_lib):
+    """A page id outside the cache is recorded in the built-in scratch's status
+    word; mla_get_status_noalloc returns it once and clears it."""
+    from head_latent_attention_06_b200.step import step_from_workload
+    cuda_lib.mla_noalloc_init()
+    assert cuda_lib.mla_get_status_noalloc() == 0
+    w = make_workload(WorkloadSpec("na", B=2, H=128, s_q=1, lens=[130, 64], seed=22))
+    st = step_from_workload(w)
+    st.absorb()
+    st._keep[2][0, 1] = 10_000                  # beyond the cache: skipped and reported
+    cuda_lib.mla_decode_paged_noalloc(st.args)
+    assert cuda_lib.mla_get_status_noalloc() == 7          # MLA_ERR_BAD_BLOCK_TABLE
+    assert cuda_lib.mla_get_status_noalloc() == 0          # cleared by the read
+    st._keep[2][0, 1] = int(w.block_table[0, 1])
+    cuda_lib.mla_decode_paged_noalloc(st.args)
+    assert cuda_lib.mla_get_status_noalloc() == 0
