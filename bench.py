@@ -37,35 +37,44 @@ METRIC = "MLA decode cache GB/s, TFLOP/s & % of B200 roofline; tokens/s per step
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# DRAM bytes (read + write) of one decode launch from an ncu capture, recorded
-# with the sha256 prefix of the kernel source it was taken on: reported as the
-# roofline's ``traffic`` only while that source is unchanged.
-# (profiles/decode_tc_v3_bf16.md)
-MEASURED_TRAFFIC = {"v3": (311525632 + 5262080, "5a3679ac14259253")}
+# DRAM bytes (read + write) of one decode launch from an ncu capture of the
+# workload, recorded with the kernel's source file and the sha256 prefix of that
+# file and the device headers it includes, as they were when the capture was
+# taken: reported as the roofline's ``traffic`` only while they are unchanged.
+MEASURED_TRAFFIC = {}
+KERNEL_HEADERS = ("sm100.cuh", "common.cuh", "tma_host.cuh")
+
+
+def kernel_source_digest(src_name: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "head_latent_attention_06_b200", "csrc")
+    for name in (src_name,) + KERNEL_HEADERS:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def decode_traffic(config: str):
-    import hashlib
     entry = MEASURED_TRAFFIC.get(config)
     if entry is None:
         return None
-    src = os.path.join(ROOT, "head_latent_attention_06_b200", "csrc", "decode_tc.cu")
-    with open(src, "rb") as f:
-        digest = hashlib.sha256(f.read()).hexdigest()[:16]
-    return entry[0] if digest == entry[1] else None
+    nbytes, src_name, sha = entry
+    return nbytes if kernel_source_digest(src_name) == sha else None
 
 
 # Nominal B200 figures, the secondary denominators: HBM3e 7.7 TB/s (HGX), dense
-# bf16/f16 tensor 2.25 PFLOP/s.
-DATASHEET = {"hbm_gbs": 7700.0, "bf16_tflops": 2250.0}
+# bf16/f16 tensor 2.25 PFLOP/s, dense fp8 4.5 PFLOP/s.
+DATASHEET = {"hbm_gbs": 7700.0, "bf16_tflops": 2250.0, "fp8_tflops": 4500.0}
 
 
-def datasheet_fracs(cache_bytes: float, flops: float, seconds: float) -> dict:
+def datasheet_fracs(cache_bytes: float, flops: float, seconds: float, kv_dtype: str = "bf16") -> dict:
     """The decode's fractions of the nominal figures (the measured peaks are the
-    primary denominators)."""
+    primary denominators); the tensor figure is that of the MMA kind used."""
+    tc = DATASHEET["fp8_tflops"] if kv_dtype == "fp8" else DATASHEET["bf16_tflops"]
     t_mem = cache_bytes / (DATASHEET["hbm_gbs"] * 1e9)
-    t_tc = flops / (DATASHEET["bf16_tflops"] * 1e12)
-    return {"hbm_gbs": DATASHEET["hbm_gbs"], "bf16_tflops": DATASHEET["bf16_tflops"],
+    t_tc = flops / (tc * 1e12)
+    return {"hbm_gbs": DATASHEET["hbm_gbs"], "tensor_tflops": tc,
             "hbm_frac": round(t_mem / seconds, 4), "tensor_frac": round(t_tc / seconds, 4),
             "binding_frac": round(max(t_mem, t_tc) / seconds, 4)}
 
@@ -87,6 +96,20 @@ def load_peaks():
         d = json.load(open(p))
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def tensor_peak(peaks: dict, kv_dtype: str):
+    """Dense tensor peak (TFLOP/s) of the MMA kind the decode runs, and how it was
+    obtained: bf16 x bf16 for a bf16 cache (the measured cuBLAS bf16 figure);
+    e4m3 x e4m3 for an e4m3 cache: a measured fp8 figure if the peaks file has
+    one, else the measured bf16 figure x 2, the ratio of the nominal dense
+    figures (4.5 / 2.25 PFLOP/s)."""
+    bf16 = float(peaks["bf16_tflops"])
+    if kv_dtype != "fp8":
+        return bf16, "bf16 x bf16 (measured cuBLAS bf16 GEMM)"
+    if "fp8_tflops" in peaks:
+        return float(peaks["fp8_tflops"]), "e4m3 x e4m3 (measured fp8 GEMM)"
+    return 2.0 * bf16, "e4m3 x e4m3 (measured bf16 GEMM x 2, the nominal fp8 / bf16 ratio)"
 
 
 def step_flops(lens, H, s_q):
@@ -187,7 +210,8 @@ def oracle_cpu_baseline(spec_name: str, budget_s: float = 12.0):
     spec = preset(spec_name)
     w = make_workload(spec)
     inp = oracle.from_workload(w)
-    row_bytes = 1152 if spec.kv_dtype == "bf16" else 580
+    from mla_inputs import row_bytes as row_bytes_of
+    row_bytes = row_bytes_of(spec.kv_dtype)
     done_b, done_tokens, t0 = 0, 0, time.perf_counter()
     while done_b < w.B and time.perf_counter() - t0 < budget_s:
         om.decode_absorbed(inp, rows=[(done_b, i) for i in range(w.s_q)])
@@ -310,8 +334,8 @@ def run_write_kv(args):
     assert mla.mla_get_status(ws) == 0
     ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     n_tok = w.B * w.s_q
-    row_bytes = 1152 if spec.kv_dtype == "bf16" else 580
-    algo_bytes = 576 * d_h * 2 + n_tok * d_h * 2 + n_tok * row_bytes
+    from mla_inputs import row_bytes as row_bytes_of
+    algo_bytes = 576 * d_h * 2 + n_tok * d_h * 2 + n_tok * row_bytes_of(spec.kv_dtype)
     gbs = algo_bytes / (ms * 1e-3) / 1e9
     peaks, peak_kind = load_peaks()
     hbm = float(peaks["hbm_gbs"])
@@ -320,7 +344,8 @@ def run_write_kv(args):
     line = {"metric": WRITE_METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16 in, fp32 accumulate, " + ("bf16 cache" if spec.kv_dtype == "bf16" else "e4m3 cache"),
+            "dtype": "bf16 in, fp32 accumulate, " + {"bf16": "bf16", "fp8": "e4m3", "q8_0": "q8_0"}[spec.kv_dtype]
+                     + " cache",
             "data": "synthetic (seeded N(0,1) hidden states, N(0,1/d_h) weights)", "config": cfg,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "traffic": None,
@@ -348,7 +373,9 @@ def _config_dict(name, w, splits=None):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    # enough steps that the timed region lasts about a second (the clock sampler
+    # reads every 200 ms)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="v3")
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
@@ -424,18 +451,19 @@ def main(argv=None):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    # The clock record covers both timed loops: the steps, then the parts one by
+    # one (each after an L2 flush), whose decode figure is the roofline's.
     with ClockSampler(local) as clk:
         for k in range(args.steps):
             timed(g_step, evs[k])
         torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    # the parts one by one (each after an L2 flush), for the kernel rooflines
-    for k in range(args.steps):
-        timed(g_absorb, ev_abs[k])
-        timed(g_decode, ev_dec[k])
-        timed(g_tail, ev_tail[k])
-    torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        for k in range(args.steps):
+            timed(g_absorb, ev_abs[k])
+            timed(g_decode, ev_dec[k])
+            timed(g_tail, ev_tail[k])
+        torch.cuda.synchronize()
     assert mla.mla_get_status(st.workspace) == 0
     ms = lambda ev: [e[0].elapsed_time(e[1]) for e in ev]
     step_ms, dec_ms, absorb_ms, tail_ms = ms(evs), ms(ev_dec), ms(ev_abs), ms(ev_tail)
@@ -446,9 +474,11 @@ def main(argv=None):
     # End to end through the public API, the way a serving loop drives it: every
     # step's queries, block table and lengths come from pinned host memory and its
     # output goes back to pinned host memory.  Two sets of step buffers (the cache
-    # and weights are shared model state) let one step's copies, on a copy-in and a
-    # copy-out stream, overlap the other step's decode.  The cache (302 MB at V3)
-    # is larger than L2, so no flush is needed between these steps.
+    # and weights are shared model state), each with a CUDA graph of its whole
+    # step (host->device copies, the four library calls, the device->host copy),
+    # replayed alternately on two streams, so that one step's copies overlap the
+    # other step's decode and the host issues one call per step.  The cache
+    # (302 MB at V3) is larger than L2, so no flush is needed between these steps.
     from head_latent_attention_06_b200.step import DecodeStep
     st2 = DecodeStep(q_nope=torch.empty_like(st.q_nope), q_pe=torch.empty_like(st.q_pe), w_uk=st.w_uk,
                      w_uv=st.w_uv, kv_cache=st._keep[0], kv_scale=st._keep[1],
@@ -456,51 +486,52 @@ def main(argv=None):
                      causal=w.causal, softmax_scale=w.softmax_scale, num_splits=st.num_splits,
                      max_seq_len=max(w.lens) if w.lens else 0)
     sts = [st, st2]
-    st2.q_nope.copy_(st.q_nope)
-    st2.q_pe.copy_(st.q_pe)
-    st2._keep[2].copy_(st._keep[2])
-    st2._keep[3].copy_(st._keep[3])
-    graphs = [g_step, st2.capture()]
-    h_q_nope = w.q_nope.pin_memory()
-    h_q_pe = w.q_pe.pin_memory()
-    h_bt = w.block_table.pin_memory()
-    h_len = w.seq_lens.pin_memory()
+    h_in = [(w.q_nope.pin_memory(), w.q_pe.pin_memory(), w.block_table.pin_memory(), w.seq_lens.pin_memory())
+            for _ in range(2)]
     h_out = [torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory() for _ in range(2)]
-    h2d = sum(t.numel() * t.element_size() for t in (h_q_nope, h_q_pe, h_bt, h_len))
+    h2d = sum(t.numel() * t.element_size() for t in h_in[0])
     d2h = h_out[0].numel() * h_out[0].element_size()
-    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-    in_done = [torch.cuda.Event() for _ in range(2)]
-    comp_done = [torch.cuda.Event() for _ in range(2)]
-    out_done = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_step(x, hi, ho):
+        x.q_nope.copy_(hi[0], non_blocking=True)
+        x.q_pe.copy_(hi[1], non_blocking=True)
+        x._keep[2].copy_(hi[2], non_blocking=True)
+        x._keep[3].copy_(hi[3], non_blocking=True)
+        x.run()
+        ho.copy_(x.out, non_blocking=True)
+
+    e2e_graphs = []
+    for i, x in enumerate(sts):
+        e2e_step(x, h_in[i], h_out[i])         # outside capture: one-time host set-up
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            e2e_step(x, h_in[i], h_out[i])
+        e2e_graphs.append(g)
+    e2e_streams = [torch.cuda.Stream(), torch.cuda.Stream()]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def e2e_run(n):
+        for s2 in e2e_streams:
+            s2.wait_stream(stream)
+        for k in range(n):
+            with torch.cuda.stream(e2e_streams[k % 2]):
+                e2e_graphs[k % 2].replay()
+        for s2 in e2e_streams:
+            stream.wait_stream(s2)
+
+    e2e_run(max(3, args.warmup))
     torch.cuda.synchronize()
-    pre = 2
-    for k in range(pre + args.steps):
-        sl, x = k % 2, sts[k % 2]
-        with torch.cuda.stream(s_in):
-            if k == pre:
-                t_start.record(s_in)
-            if k >= 2:
-                s_in.wait_event(comp_done[sl])       # step k-2 has read this set's inputs
-            x.q_nope.copy_(h_q_nope, non_blocking=True)
-            x.q_pe.copy_(h_q_pe, non_blocking=True)
-            x._keep[2].copy_(h_bt, non_blocking=True)
-            x._keep[3].copy_(h_len, non_blocking=True)
-            in_done[sl].record(s_in)
-        stream.wait_event(in_done[sl])
-        if k >= 2:
-            stream.wait_event(out_done[sl])          # step k-2's output has left this set
-        graphs[sl].replay()
-        comp_done[sl].record(stream)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(comp_done[sl])
-            h_out[sl].copy_(x.out, non_blocking=True)
-            out_done[sl].record(s_out)
-    t_end.record(s_out)
+    if world > 1:
+        dist.barrier()
+    t_start.record(stream)
+    e2e_run(args.steps)
+    t_end.record(stream)
     torch.cuda.synchronize()
     e2e_ms = reduce_max(t_start.elapsed_time(t_end)) / args.steps
-    for x in sts:
+    for i, x in enumerate(sts):
         assert mla.mla_get_status(x.workspace) == 0
+        assert torch.equal(h_out[i], st.out.cpu())   # both buffer sets decode the same step
 
     peaks, peak_kind = load_peaks()
     hbm = float(peaks["hbm_gbs"])
@@ -508,14 +539,19 @@ def main(argv=None):
     dec_gbs = cache_bytes / (dec_avg_ms * 1e-3) / 1e9
     dec_tflops = flops / (dec_avg_ms * 1e-3) / 1e12
     t_mem = cache_bytes / (hbm * 1e9)
-    t_tc = flops / (float(peaks["bf16_tflops"]) * 1e12)
-    launches_per_step = 3 + (1 if st.num_splits > 1 else 0)
+    tc_peak, tc_peak_kind = tensor_peak(peaks, spec.kv_dtype)
+    t_tc = flops / (tc_peak * 1e12)
+    tensor_bound = t_tc > t_mem
+    # absorb, decode, up-projection, and the merge unless one split was used
+    launches_per_step = 3 + (1 if st.num_splits != 1 else 0)
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp8-e4m3 cache, bf16 MMA" if spec.kv_dtype == "fp8" else "bf16",
+        "dtype": {"fp8": "e4m3 cache, e4m3 x e4m3 MMA (two-term operand split)",
+                  "q8_0": "q8_0 cache (int8 codes x fp16 block scales formed in bf16), bf16 MMA",
+                  "bf16": "bf16"}[spec.kv_dtype],
         "data": "synthetic (seeded, N(0,1) activations and cache, N(0,1/512) weights)",
         "config": _config_dict(args.config, w, st.num_splits),
         "tflops": round(world * (flops + proj_flops(w.n_tok, w.H)) / (ms_per_step * 1e-3) / 1e12, 2),
@@ -524,21 +560,27 @@ def main(argv=None):
         "absorb_us": round(1e3 * sum(absorb_ms) / len(absorb_ms), 2),
         "combine_up_proj_us": round(1e3 * sum(tail_ms) / len(tail_ms), 2),
         "roofline": {
-            "bound": "hbm", "achieved": round(dec_gbs, 1), "peak": hbm, "unit": "GB/s",
-            "frac": round(dec_gbs / hbm, 4), "traffic": decode_traffic(args.config),
-            "peak_kind": f"{peak_kind} HBM copy bandwidth",
+            # the binding side: cache bytes at the HBM copy bandwidth, or the
+            # algorithmic FLOPs at the tensor peak of the MMA kind used
+            **({"bound": "tensor", "achieved": round(dec_tflops, 1), "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": round(dec_tflops / tc_peak, 4), "peak_kind": f"{peak_kind}: {tc_peak_kind}"}
+               if tensor_bound else
+               {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(dec_gbs / hbm, 4), "peak_kind": f"{peak_kind} HBM copy bandwidth"}),
+            "traffic": decode_traffic(args.config),
             "kernel": "mla_decode_paged",
-            "tensor": {"achieved_tflops": round(dec_tflops, 1),
-                       "peak_tflops": float(peaks["bf16_tflops"]),
-                       "frac": round(dec_tflops / float(peaks["bf16_tflops"]), 4)},
+            "hbm": {"achieved_gbs": round(dec_gbs, 1), "peak_gbs": hbm, "frac": round(dec_gbs / hbm, 4)},
+            "tensor": {"achieved_tflops": round(dec_tflops, 1), "peak_tflops": tc_peak,
+                       "peak_kind": tc_peak_kind, "frac": round(dec_tflops / tc_peak, 4)},
             "binding_roofline_frac": round(max(t_mem, t_tc) / (dec_avg_ms * 1e-3), 4),
-            "datasheet": datasheet_fracs(cache_bytes, flops, dec_avg_ms * 1e-3),
+            "datasheet": datasheet_fracs(cache_bytes, flops, dec_avg_ms * 1e-3, spec.kv_dtype),
         },
         "cached_tokens_per_s": round(world * sum(w.lens) / (dec_avg_ms * 1e-3), 1),
         "e2e": {"value": round(world * cache_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 5),
-                "pipeline": "two step buffer sets; host copies overlap the other step's decode"},
+                "pipeline": "two step buffer sets, one CUDA graph each (copies + step), replayed "
+                            "alternately on two streams; host copies overlap the other step's decode"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }

@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(PKG, "libmla_b200.so")
 
 D_C, D_R, D_N, D_V, PAGE = 512, 64, 128, 128, 64
 MAX_SPLITS = 128
-KV_BF16, KV_FP8_E4M3 = 0, 1
+KV_BF16, KV_FP8_E4M3, KV_Q8_0 = 0, 1, 2
+Q8_BLOCKS = (D_C + D_R) // 32   # q8_0: scale blocks of a 576-value row
 
 STATUS = {
     0: "MLA_OK", 1: "MLA_ERR_INVALID_VALUE", 2: "MLA_ERR_UNSUPPORTED", 3: "MLA_ERR_MISALIGNED",
@@ -31,7 +32,7 @@ EXPORTS = ("mla_absorb_q", "mla_decode_workspace_size", "mla_decode_num_splits",
            "mla_decode_paged", "mla_combine_splits", "mla_up_proj_v", "mla_get_status",
            "mla_status_string", "mla_decode_paged_noalloc", "mla_noalloc_init",
            "mla_get_status_noalloc", "mla_write_kv_workspace_size", "mla_write_kv",
-           "mla_set_decode_kernel")
+           "mla_set_decode_kernel", "mla_set_device_wait_limit")
 
 DECODE_AUTO, DECODE_WARP_MMA = 0, 1
 
@@ -96,6 +97,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_noalloc_init.argtypes = []
     lib.mla_get_status_noalloc.argtypes = [vp]
     lib.mla_set_decode_kernel.argtypes = [i32]
+    lib.mla_set_device_wait_limit.argtypes = [ctypes.c_uint64]
     pw = ctypes.POINTER(WriteKvArgs)
     lib.mla_write_kv_workspace_size.argtypes = [pw, ctypes.POINTER(ctypes.c_size_t)]
     lib.mla_write_kv.argtypes = [pw, vp]
@@ -184,24 +186,37 @@ def mla_up_proj_v(o_lat, w_uv, out, stream=None):
                                                  w_uv.shape[1], w_uv.shape[2], _stream(stream)))
 
 
+def _cache_kind(kv_cache):
+    """(kv_dtype code, scale dtype, scale shape tail) of a cache tensor's dtype:
+    bf16 values; float8_e4m3fn codes with fp32 row scales [pages][64]; int8 q8_0
+    codes with fp16 block scales [pages][64][18]."""
+    import torch
+    if kv_cache.dtype == torch.float8_e4m3fn:
+        return KV_FP8_E4M3, torch.float32, ()
+    if kv_cache.dtype == torch.int8:
+        return KV_Q8_0, torch.float16, (Q8_BLOCKS,)
+    return KV_BF16, None, ()
+
+
 def make_decode_args(*, q_lat, q_pe, kv_cache, kv_scale, block_table, seq_lens, o_lat, lse,
                      workspace=None, causal=False, softmax_scale, num_splits=0,
                      max_seq_len=0) -> DecodeArgs:
     """Fill a ``DecodeArgs`` from device tensors.  Shapes: q_lat [B][s_q][H][512],
-    q_pe [B][s_q][H][64], kv_cache [num_pages][64][576] (bf16 or float8_e4m3fn),
-    kv_scale [num_pages][64] fp32 or None, block_table [B][max_pages] int32,
-    seq_lens [B] int32, o_lat like q_lat, lse [B][s_q][H] fp32 or None."""
+    q_pe [B][s_q][H][64], kv_cache [num_pages][64][576] (bf16, float8_e4m3fn or
+    int8 for q8_0), kv_scale [num_pages][64] fp32 (e4m3), [num_pages][64][18] fp16
+    (q8_0) or None (bf16), block_table [B][max_pages] int32, seq_lens [B] int32,
+    o_lat like q_lat, lse [B][s_q][H] fp32 or None."""
     import torch
     bf16, f32, i32 = torch.bfloat16, torch.float32, torch.int32
     if q_lat.dim() != 4 or kv_cache.dim() != 3 or block_table.dim() != 2:
         raise ValueError("q_lat must be [B][s_q][H][512], kv_cache [pages][64][576], block_table [B][pages]")
     B, s_q, H, _ = q_lat.shape
     P = kv_cache.shape[0]
-    fp8 = kv_cache.dtype == torch.float8_e4m3fn
+    kind, sc_dtype, sc_tail = _cache_kind(kv_cache)
     _want([(q_lat, "q_lat", bf16, (B, s_q, H, D_C), False),
            (q_pe, "q_pe", bf16, (B, s_q, H, D_R), False),
-           (kv_cache, "kv_cache", (bf16, torch.float8_e4m3fn), (P, PAGE, D_C + D_R), False),
-           (kv_scale, "kv_scale", f32, (P, PAGE), not fp8),
+           (kv_cache, "kv_cache", (bf16, torch.float8_e4m3fn, torch.int8), (P, PAGE, D_C + D_R), False),
+           (kv_scale, "kv_scale", sc_dtype or f32, (P, PAGE) + sc_tail, kind == KV_BF16),
            (block_table, "block_table", i32, (B, block_table.shape[1]), False),
            (seq_lens, "seq_lens", i32, (B,), False),
            (o_lat, "o_lat", bf16, (B, s_q, H, D_C), False),
@@ -216,7 +231,7 @@ def make_decode_args(*, q_lat, q_pe, kv_cache, kv_scale, block_table, seq_lens, 
     a.d_c, a.d_r, a.page_size = D_C, D_R, PAGE
     a.num_pages = kv_cache.shape[0]
     a.max_pages_per_seq = block_table.shape[1]
-    a.kv_dtype = KV_FP8_E4M3 if fp8 else KV_BF16
+    a.kv_dtype = kind
     a.causal = int(bool(causal))
     a.num_splits = int(num_splits)
     a.max_seq_len = int(max_seq_len)
@@ -269,23 +284,29 @@ def mla_set_decode_kernel(kernel: int):
     _check("mla_set_decode_kernel", load().mla_set_decode_kernel(int(kernel)))
 
 
+def mla_set_device_wait_limit(ns: int):
+    """Process-wide limit of the decode kernels' bounded waits (0: the 2 s default)."""
+    _check("mla_set_device_wait_limit", load().mla_set_device_wait_limit(int(ns)))
+
+
 def make_write_kv_args(*, h, w_dkv, kv_cache, kv_scale, block_table, seq_lens, workspace=None,
                        rope_base=10000.0) -> WriteKvArgs:
     """Fill a ``WriteKvArgs`` from device tensors.  Shapes: h [B][s_q][d_h] bf16,
     w_dkv [576][d_h] bf16 (W_DKV rows, then W_KR rows), kv_cache [num_pages][64][576]
-    (bf16 or float8_e4m3fn), kv_scale [num_pages][64] fp32 or None,
-    block_table [B][max_pages] int32, seq_lens [B] int32."""
+    (bf16, float8_e4m3fn or int8 for q8_0), kv_scale [num_pages][64] fp32 (e4m3),
+    [num_pages][64][18] fp16 (q8_0) or None (bf16), block_table [B][max_pages]
+    int32, seq_lens [B] int32."""
     import torch
     bf16, f32, i32 = torch.bfloat16, torch.float32, torch.int32
     if h.dim() != 3 or kv_cache.dim() != 3 or block_table.dim() != 2:
         raise ValueError("h must be [B][s_q][d_h], kv_cache [pages][64][576], block_table [B][pages]")
     B, s_q, d_h = h.shape
     P = kv_cache.shape[0]
-    fp8 = kv_cache.dtype == torch.float8_e4m3fn
+    kind, sc_dtype, sc_tail = _cache_kind(kv_cache)
     _want([(h, "h", bf16, (B, s_q, d_h), False),
            (w_dkv, "w_dkv", bf16, (D_C + D_R, d_h), False),
-           (kv_cache, "kv_cache", (bf16, torch.float8_e4m3fn), (P, PAGE, D_C + D_R), False),
-           (kv_scale, "kv_scale", f32, (P, PAGE), not fp8),
+           (kv_cache, "kv_cache", (bf16, torch.float8_e4m3fn, torch.int8), (P, PAGE, D_C + D_R), False),
+           (kv_scale, "kv_scale", sc_dtype or f32, (P, PAGE) + sc_tail, kind == KV_BF16),
            (block_table, "block_table", i32, (B, block_table.shape[1]), False),
            (seq_lens, "seq_lens", i32, (B,), False),
            (workspace, "workspace", torch.uint8, None, True)])
@@ -297,7 +318,7 @@ def make_write_kv_args(*, h, w_dkv, kv_cache, kv_scale, block_table, seq_lens, w
     a.d_c, a.d_r, a.page_size = D_C, D_R, PAGE
     a.num_pages = kv_cache.shape[0]
     a.max_pages_per_seq = block_table.shape[1]
-    a.kv_dtype = KV_FP8_E4M3 if kv_cache.dtype == torch.float8_e4m3fn else KV_BF16
+    a.kv_dtype = kind
     a.rope_base = float(rope_base)
     if workspace is not None:
         a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()

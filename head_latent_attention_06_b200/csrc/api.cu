@@ -14,6 +14,7 @@ cudaError_t launch_up_proj_v(const void*, const void*, void*, int, int, cudaStre
 cudaError_t launch_decode_mma(const mla_decode_args_t*, int, cudaStream_t);
 cudaError_t launch_combine(const mla_decode_args_t*, int, cudaStream_t);
 cudaError_t launch_decode_tc(const mla_decode_args_t*, int, cudaStream_t);
+cudaError_t launch_decode_f8(const mla_decode_args_t*, int, cudaStream_t);
 bool decode_tc_supported(const mla_decode_args_t*);
 int decode_tc_clusters_per_split(const mla_decode_args_t*);
 int decode_mma_tiles(int len);
@@ -47,21 +48,30 @@ mla_status_t check_decode_shape(const mla_decode_args_t* a) {
     return MLA_ERR_INVALID_VALUE;
   if (a->d_c != kDc || a->d_r != kDr || a->page_size != kPage) return MLA_ERR_UNSUPPORTED;
   if (a->H % 16 != 0 || a->H > 128 || a->s_q > MLA_MAX_S_Q) return MLA_ERR_UNSUPPORTED;
-  if (a->kv_dtype != MLA_KV_BF16 && a->kv_dtype != MLA_KV_FP8_E4M3) return MLA_ERR_UNSUPPORTED;
+  if (a->kv_dtype != MLA_KV_BF16 && a->kv_dtype != MLA_KV_FP8_E4M3 && a->kv_dtype != MLA_KV_Q8_0)
+    return MLA_ERR_UNSUPPORTED;
   if (a->num_splits < 0 || a->num_splits > MLA_MAX_SPLITS) return MLA_ERR_INVALID_VALUE;
   if (a->max_seq_len < 0) return MLA_ERR_INVALID_VALUE;
   if (!(a->softmax_scale == a->softmax_scale)) return MLA_ERR_INVALID_VALUE;
   return MLA_OK;
 }
 
-// Process-wide kernel choice (mla_set_decode_kernel).
+// Process-wide kernel choice (mla_set_decode_kernel) and device wait limit
+// (mla_set_device_wait_limit).
 std::atomic<int32_t> g_decode_kernel{MLA_DECODE_AUTO};
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
 
 bool forced_mma() { return g_decode_kernel.load(std::memory_order_relaxed) == MLA_DECODE_WARP_MMA; }
 
 // Which decode kernel runs: the tensor-memory kernel for the shapes it takes,
 // else the warp-MMA kernel.
 bool use_tc(const mla_decode_args_t* a) { return !forced_mma() && decode_tc_supported(a); }
+
+// Workspace bytes the chosen path needs.
+size_t workspace_bytes(const mla_decode_args_t* a, int splits) {
+  return workspace_layout(a->B * a->s_q, a->H, splits).total;
+}
 
 // Split count.  Tensor-memory kernel: the count that minimises the modelled
 // makespan (waves of 74 CTA pairs x per-unit work), preferring fewer splits.  Warp-MMA
@@ -104,7 +114,8 @@ mla_status_t check_write_kv_shape(const mla_write_kv_args_t* a) {
     return MLA_ERR_INVALID_VALUE;
   if ((int64_t)a->B * a->s_q > (1 << 24)) return MLA_ERR_INVALID_VALUE;
   if (a->d_c != kDc || a->d_r != kDr || a->page_size != kPage || a->d_h % 64 != 0) return MLA_ERR_UNSUPPORTED;
-  if (a->kv_dtype != MLA_KV_BF16 && a->kv_dtype != MLA_KV_FP8_E4M3) return MLA_ERR_UNSUPPORTED;
+  if (a->kv_dtype != MLA_KV_BF16 && a->kv_dtype != MLA_KV_FP8_E4M3 && a->kv_dtype != MLA_KV_Q8_0)
+    return MLA_ERR_UNSUPPORTED;
   if (!(a->rope_base > 0.f) || !isfinite(a->rope_base)) return MLA_ERR_INVALID_VALUE;
   return MLA_OK;
 }
@@ -115,6 +126,11 @@ size_t write_kv_workspace(const mla_write_kv_args_t* a) {
 }
 
 }  // namespace
+
+namespace mla {
+// Limit of every bounded wait in the decode kernels, as set for this process.
+uint64_t device_wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
+}  // namespace mla
 
 extern "C" {
 
@@ -144,19 +160,18 @@ mla_status_t mla_decode_workspace_size(const mla_decode_args_t* a, size_t* bytes
   mla_status_t st = check_decode_shape(a);
   if (st != MLA_OK) return st;
   if (!bytes) return MLA_ERR_INVALID_VALUE;
-  *bytes = workspace_layout(a->B * a->s_q, a->H, choose_splits(a)).total;
+  *bytes = workspace_bytes(a, choose_splits(a));
   return MLA_OK;
 }
 
 static mla_status_t check_decode_ptrs(const mla_decode_args_t* a, int splits) {
   if (!a->workspace) return MLA_ERR_INVALID_VALUE;
   if (!aligned16(a->workspace)) return MLA_ERR_MISALIGNED;
-  if (a->workspace_bytes < workspace_layout(a->B * a->s_q, a->H, splits).total)
-    return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (a->workspace_bytes < workspace_bytes(a, splits)) return MLA_ERR_WORKSPACE_TOO_SMALL;
   if (a->B == 0) return MLA_OK;
   if (!a->q_lat || !a->q_pe || !a->kv_cache || !a->block_table || !a->seq_lens || !a->o_lat)
     return MLA_ERR_INVALID_VALUE;
-  if (a->kv_dtype == MLA_KV_FP8_E4M3 && !a->kv_scale) return MLA_ERR_INVALID_VALUE;
+  if (a->kv_dtype != MLA_KV_BF16 && !a->kv_scale) return MLA_ERR_INVALID_VALUE;
   if (a->num_pages <= 0) return MLA_ERR_INVALID_VALUE;
   if (!aligned16(a->q_lat) || !aligned16(a->q_pe) || !aligned16(a->kv_cache) ||
       !aligned16(a->o_lat))
@@ -174,7 +189,9 @@ mla_status_t mla_decode_paged(const mla_decode_args_t* a, void* stream) {
   const int splits = choose_splits(a);
   st = check_decode_ptrs(a, splits);
   if (st != MLA_OK || a->B == 0) return st;
-  if (use_tc(a)) return from_cuda(launch_decode_tc(a, splits, (cudaStream_t)stream));
+  if (use_tc(a))
+    return from_cuda(a->kv_dtype == MLA_KV_FP8_E4M3 ? launch_decode_f8(a, splits, (cudaStream_t)stream)
+                                                      : launch_decode_tc(a, splits, (cudaStream_t)stream));
   return from_cuda(launch_decode_mma(a, splits, (cudaStream_t)stream));
 }
 
@@ -183,7 +200,8 @@ mla_status_t mla_combine_splits(const mla_decode_args_t* a, void* stream) {
   if (st != MLA_OK) return st;
   const int splits = choose_splits(a);
   st = check_decode_ptrs(a, splits);
-  if (st != MLA_OK || a->B == 0 || splits == 1) return st;
+  if (st != MLA_OK || a->B == 0) return st;
+  if (splits == 1) return st;
   return from_cuda(launch_combine(a, splits, (cudaStream_t)stream));
 }
 
@@ -203,7 +221,7 @@ mla_status_t mla_write_kv(const mla_write_kv_args_t* a, void* stream) {
   if (a->workspace_bytes < write_kv_workspace(a)) return MLA_ERR_WORKSPACE_TOO_SMALL;
   if (a->B == 0) return MLA_OK;
   if (!a->h || !a->w_dkv || !a->kv_cache || !a->block_table || !a->seq_lens) return MLA_ERR_INVALID_VALUE;
-  if (a->kv_dtype == MLA_KV_FP8_E4M3 && !a->kv_scale) return MLA_ERR_INVALID_VALUE;
+  if (a->kv_dtype != MLA_KV_BF16 && !a->kv_scale) return MLA_ERR_INVALID_VALUE;
   if (a->num_pages <= 0) return MLA_ERR_INVALID_VALUE;
   if (!aligned16(a->h) || !aligned16(a->w_dkv) || !aligned16(a->kv_cache)) return MLA_ERR_MISALIGNED;
   if ((reinterpret_cast<uintptr_t>(a->block_table) & 3u) || (reinterpret_cast<uintptr_t>(a->seq_lens) & 3u) ||
@@ -224,6 +242,11 @@ mla_status_t mla_get_status(void* workspace, void* stream) {
     if (cudaStreamSynchronize(s) != cudaSuccess) return MLA_ERR_CUDA;
   }
   return (mla_status_t)word;
+}
+
+mla_status_t mla_set_device_wait_limit(uint64_t ns) {
+  g_wait_ns.store(ns == 0 ? kDefaultWaitNs : ns, std::memory_order_relaxed);
+  return MLA_OK;
 }
 
 mla_status_t mla_set_decode_kernel(int32_t kernel) {

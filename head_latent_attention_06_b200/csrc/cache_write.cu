@@ -24,6 +24,8 @@
 #include <cuda_fp8.h>
 #include <math_constants.h>
 
+#include <cuda_fp16.h>
+
 #include "sm100.cuh"
 #include "tma_host.cuh"
 
@@ -160,7 +162,7 @@ __global__ void __launch_bounds__(kWThreads) kv_down_proj_kernel(const __grid_co
 struct FinishParams {
   const float* part;
   uint8_t* kv;
-  float* kv_scale;
+  void* kv_scale;  // e4m3: fp32 [pages][64]; q8_0: fp16 [pages][64][18]
   const int32_t* block_table;
   const int32_t* seq_lens;
   uint32_t* status;
@@ -168,8 +170,9 @@ struct FinishParams {
   double log2_base;
 };
 
-// One warp per new token: sum the partials, rotate, quantise, store.
-template <bool FP8>
+// One warp per new token: sum the partials, rotate, quantise, store.  KIND: 0
+// bf16 cache, 1 e4m3 with a per-row scale, 2 q8_0 with per-block scales.
+template <int KIND>
 __global__ void __launch_bounds__(128) kv_finish_kernel(const FinishParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 4 + warp;
@@ -216,10 +219,31 @@ __global__ void __launch_bounds__(128) kv_finish_kernel(const FinishParams p) {
     const double x0 = v[8].x, x1 = v[8].y;
     v[8] = make_float2((float)(x0 * cs - x1 * sn), (float)(x0 * sn + x1 * cs));
   }
-  if constexpr (!FP8) {
+  if constexpr (KIND == 0) {
     __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(p.kv) + slot * kRow + 2 * lane;
 #pragma unroll
     for (int j = 0; j < 9; ++j) *reinterpret_cast<uint32_t*>(row + 64 * j) = pack_bf16(v[j].x, v[j].y);
+  } else if constexpr (KIND == 2) {
+    // q8_0: block 2j + lane / 16 is values 64j + 32 (lane / 16) .. +31, two per
+    // lane of its half-warp; scale d = amax / 127 rounded to fp16, codes the fp32
+    // quotients by d rounded to nearest even and clamped to [-127, 127]
+    int8_t* row = reinterpret_cast<int8_t*>(p.kv) + slot * kRow + 2 * lane;
+    __half* sc = static_cast<__half*>(p.kv_scale) + slot * (kRow / 32);
+#pragma unroll
+    for (int j = 0; j < 9; ++j) {
+      float amax = fmaxf(fabsf(v[j].x), fabsf(v[j].y));
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const __half d = __float2half_rn(__fdiv_rn(amax, 127.f));
+      const float df = __half2float(d);
+      int c0 = 0, c1 = 0;
+      if (df > 0.f) {
+        c0 = (int)fminf(fmaxf(rintf(__fdiv_rn(v[j].x, df)), -127.f), 127.f);
+        c1 = (int)fminf(fmaxf(rintf(__fdiv_rn(v[j].y, df)), -127.f), 127.f);
+      }
+      *reinterpret_cast<uint16_t*>(row + 64 * j) = (uint16_t)((uint8_t)c0 | ((uint16_t)(uint8_t)c1 << 8));
+      if ((lane & 15) == 0) sc[2 * j + (lane >> 4)] = d;
+    }
   } else {
     float amax = 0.f;
 #pragma unroll
@@ -236,7 +260,7 @@ __global__ void __launch_bounds__(128) kv_finish_kernel(const FinishParams p) {
       const __nv_fp8x2_storage_t code = __nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
       *reinterpret_cast<uint16_t*>(row + 64 * j) = (uint16_t)code;
     }
-    if (lane == 0) p.kv_scale[slot] = scale;
+    if (lane == 0) static_cast<float*>(p.kv_scale)[slot] = scale;
   }
 }
 
@@ -270,8 +294,8 @@ cudaError_t launch_write_kv(const mla_write_kv_args_t* a, cudaStream_t stream) {
   });
   if (e != cudaSuccess) return e;
   dim3 grid((n_tok + kWTok - 1) / kWTok, ks, kRow / kWCols);
-  e = launch_pdl(kv_down_proj_kernel, grid, dim3(kWThreads), kWSmem, stream, tm_h, tm_w, part,
-                             n_tok, a->d_h / kWK, status);
+  e = launch_pdl(kv_down_proj_kernel, grid, dim3(kWThreads), kWSmem, stream, tm_h, tm_w, part, n_tok,
+                 a->d_h / kWK, status);
   if (e != cudaSuccess) return e;
   FinishParams p;
   p.part = part;
@@ -287,8 +311,9 @@ cudaError_t launch_write_kv(const mla_write_kv_args_t* a, cudaStream_t stream) {
   p.num_pages = a->num_pages;
   p.log2_base = log2((double)a->rope_base);
   const dim3 fgrid((n_tok + 3) / 4);
-  return a->kv_dtype == MLA_KV_FP8_E4M3 ? launch_pdl(kv_finish_kernel<true>, fgrid, dim3(128), 0, stream, p)
-                                        : launch_pdl(kv_finish_kernel<false>, fgrid, dim3(128), 0, stream, p);
+  if (a->kv_dtype == MLA_KV_FP8_E4M3) return launch_pdl(kv_finish_kernel<1>, fgrid, dim3(128), 0, stream, p);
+  if (a->kv_dtype == MLA_KV_Q8_0) return launch_pdl(kv_finish_kernel<2>, fgrid, dim3(128), 0, stream, p);
+  return launch_pdl(kv_finish_kernel<0>, fgrid, dim3(128), 0, stream, p);
 }
 
 }  // namespace mla

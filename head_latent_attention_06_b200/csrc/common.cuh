@@ -117,6 +117,9 @@ MLA_DEVI uint32_t smem_u32(const void* p) {
 MLA_DEVI void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem)), "l"(gmem));
 }
+MLA_DEVI void cp_async4(void* smem, const void* gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(smem)), "l"(gmem));
+}
 MLA_DEVI void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 template <int N>
 MLA_DEVI void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }

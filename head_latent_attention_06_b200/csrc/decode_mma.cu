@@ -2,8 +2,16 @@
 //
 // This is the portable formulation of the decode step: legacy warp MMAs
 // (mma.sync, fp32 accumulation) with cp.async staging.  It handles every
-// supported shape (any H multiple of 16, s_q <= 2, bf16 or e4m3 cache) and is the
-// path for shapes the tensor-memory kernel does not take.
+// supported shape (any H multiple of 16, any s_q, bf16, e4m3 or q8_0 cache) and
+// is the path for shapes the tensor-memory kernels do not take: the q8_0 cache,
+// an e4m3 scale array not on 16 bytes.
+//
+// Cache formats.  bf16: the rows as they are.  e4m3: codes converted exactly to
+// bf16 in shared memory, the per-token scale folded into S and into P.  q8_0
+// (ik_llama.cpp docs "FlashMLA", section "KV cache with MLA"): int8 codes with
+// one fp16 scale per 32-value block; each value is formed as code * scale in
+// fp32 and rounded to bf16 in shared memory (relative error 2^-9, against the
+// format's own step of up to 1/254 of the block's largest value).
 //
 // For one sequence b, the rows of the attention problem are the (query i,
 // head h) pairs, r = i * H + h.  A CTA owns 64 rows and one split (a range of
@@ -14,6 +22,7 @@
 // (FlashAttention-style on-chip tiles, nnets.ru article, section
 // "MLA и FlashAttention"; V is the latent itself, so the tile loaded for S is
 // reused unchanged for P.C.)
+#include <cuda_fp16.h>
 #include <math_constants.h>
 
 #include "common.cuh"
@@ -32,7 +41,7 @@ struct DecodeParams {
   const __nv_bfloat16* q_lat;
   const __nv_bfloat16* q_pe;
   const uint8_t* kv;
-  const float* kv_scale;
+  const void* kv_scale;  // e4m3: fp32 [pages][64]; q8_0: fp16 [pages][64][18]
   const int32_t* block_table;
   const int32_t* seq_lens;
   __nv_bfloat16* o_lat;
@@ -44,14 +53,17 @@ struct DecodeParams {
   float scale_log2;  // softmax_scale * log2(e)
 };
 
-template <bool FP8>
+// KIND: 0 bf16 cache, 1 e4m3 (+ fp32 token scales), 2 q8_0 (+ fp16 block scales)
+constexpr int kQ8Blocks = kRow / 32;  // 18 scale blocks per row
+
+template <int KIND>
 struct Smem {
   static constexpr size_t q_bytes = (size_t)ROWS * CP * 2;
-  static constexpr size_t stage_bytes = FP8 ? (size_t)TT * kRow : (size_t)TT * CP * 2;
-  static constexpr size_t conv_bytes = FP8 ? (size_t)TT * CP * 2 : 0;
+  static constexpr size_t stage_bytes = KIND ? (size_t)TT * kRow : (size_t)TT * CP * 2;
+  static constexpr size_t conv_bytes = KIND ? (size_t)TT * CP * 2 : 0;
   static constexpr size_t p_bytes = (size_t)ROWS * PP * 2;
   static constexpr size_t red_bytes = 2 * ROWS * sizeof(float);
-  static constexpr size_t sc_bytes = NSTAGE * TT * sizeof(float);
+  static constexpr size_t sc_bytes = NSTAGE * TT * (KIND == 2 ? kQ8Blocks * 2 : sizeof(float));
   static constexpr size_t q_off = 0;
   static constexpr size_t stage_off = q_off + q_bytes;
   static constexpr size_t conv_off = stage_off + NSTAGE * stage_bytes;
@@ -61,15 +73,18 @@ struct Smem {
   static constexpr size_t total = sc_off + sc_bytes;
 };
 
-template <bool FP8>
+template <int KIND>
 __global__ void __launch_bounds__(NTHREADS, 1) decode_mma_kernel(DecodeParams p) {
-  using SM = Smem<FP8>;
+  constexpr bool CODED = KIND != 0;  // the cache holds codes converted in shared memory
+  using SM = Smem<KIND>;
   extern __shared__ __align__(16) unsigned char smem[];
   __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smem + SM::q_off);
   unsigned char* stages = smem + SM::stage_off;
   __nv_bfloat16* ps = reinterpret_cast<__nv_bfloat16*>(smem + SM::p_off);
   float* red = reinterpret_cast<float*>(smem + SM::red_off);  // [2 halves][ROWS]
-  float* scs = reinterpret_cast<float*>(smem + SM::sc_off);   // [NSTAGE][TT]
+  float* scs = reinterpret_cast<float*>(smem + SM::sc_off);   // e4m3: [NSTAGE][TT]
+  // q8_0: [NSTAGE][TT][18] fp16 block scales
+  __half* qsc = reinterpret_cast<__half*>(smem + SM::sc_off);
 
   const int g = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -111,11 +126,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_mma_kernel(DecodeParams p)
   auto load_tile = [&](int t, int stage) {
     unsigned char* st = stages + stage * SM::stage_bytes;
     const int jb = t * TT;
-    constexpr int VPR = FP8 ? kRow / 16 : kRow / 8;  // 16-byte vectors per token row
+    constexpr int VPR = CODED ? kRow / 16 : kRow / 8;  // 16-byte vectors per token row
     for (int v = tid; v < TT * VPR; v += NTHREADS) {
       int r = v / VPR, c = v % VPR;
       int j = jb + r;
-      unsigned char* dst = FP8 ? st + r * kRow + c * 16 : st + (r * CP + c * 8) * 2;
+      unsigned char* dst = CODED ? st + r * kRow + c * 16 : st + (r * CP + c * 8) * 2;
       bool ok = j < j_end;
       int page = ok ? bt[j / kPage] : 0;
       if (ok && (page < 0 || page >= p.num_pages)) {
@@ -124,19 +139,35 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_mma_kernel(DecodeParams p)
       }
       if (ok) {
         size_t rowi = (size_t)page * kPage + (j % kPage);
-        cp_async16(dst, p.kv + rowi * kRow * (FP8 ? 1 : 2) + c * 16);
+        cp_async16(dst, p.kv + rowi * kRow * (CODED ? 1 : 2) + c * 16);
       } else {
         *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
       }
     }
-    if (FP8 && tid < TT) {
+    if (KIND == 1 && tid < TT) {
       int j = jb + tid;
       float s = 0.f;
       if (j < j_end) {
         int page = bt[j / kPage];
-        if (page >= 0 && page < p.num_pages) s = p.kv_scale[(size_t)page * kPage + (j % kPage)];
+        if (page >= 0 && page < p.num_pages)
+          s = static_cast<const float*>(p.kv_scale)[(size_t)page * kPage + (j % kPage)];
       }
       scs[stage * TT + tid] = s;
+    }
+    if (KIND == 2) {
+      // the 18 fp16 block scales of each row: nine 4-byte words (36 bytes)
+      for (int v = tid; v < TT * (kQ8Blocks / 2); v += NTHREADS) {
+        const int r = v / (kQ8Blocks / 2), w = v % (kQ8Blocks / 2);
+        const int j = jb + r;
+        uint32_t* dst = reinterpret_cast<uint32_t*>(qsc + ((size_t)stage * TT + r) * kQ8Blocks) + w;
+        int page = j < j_end ? bt[j / kPage] : -1;
+        if (page >= 0 && page < p.num_pages) {
+          const size_t rowi = (size_t)page * kPage + (j % kPage);
+          cp_async4(dst, static_cast<const __half*>(p.kv_scale) + rowi * kQ8Blocks + 2 * w);
+        } else {
+          *dst = 0u;
+        }
+      }
     }
     cp_async_commit();
   };
@@ -179,17 +210,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_mma_kernel(DecodeParams p)
       else cp_async_commit();
     }
     const __nv_bfloat16* cs;
-    if (FP8) {
+    if (CODED) {
       const uint8_t* raw = stages + stage * SM::stage_bytes;
       __nv_bfloat16* conv = reinterpret_cast<__nv_bfloat16*>(smem + SM::conv_off);
       for (int v = tid; v < TT * (kRow / 8); v += NTHREADS) {
         int r = v / (kRow / 8), c = (v % (kRow / 8)) * 8;
         uint2 in = *reinterpret_cast<const uint2*>(raw + r * kRow + c);
         uint4 o;
-        o.x = e4m3x2_to_bf16x2((uint16_t)(in.x & 0xFFFF));
-        o.y = e4m3x2_to_bf16x2((uint16_t)(in.x >> 16));
-        o.z = e4m3x2_to_bf16x2((uint16_t)(in.y & 0xFFFF));
-        o.w = e4m3x2_to_bf16x2((uint16_t)(in.y >> 16));
+        if (KIND == 1) {
+          o.x = e4m3x2_to_bf16x2((uint16_t)(in.x & 0xFFFF));
+          o.y = e4m3x2_to_bf16x2((uint16_t)(in.x >> 16));
+          o.z = e4m3x2_to_bf16x2((uint16_t)(in.y & 0xFFFF));
+          o.w = e4m3x2_to_bf16x2((uint16_t)(in.y >> 16));
+        } else {
+          // 8 int8 codes of one 32-value block times its scale
+          const float d = __half2float(qsc[((size_t)stage * TT + r) * kQ8Blocks + (c >> 5)]);
+          const uint32_t w[2] = {in.x, in.y};
+          uint32_t out[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int8_t lo = (int8_t)((w[k >> 1] >> (16 * (k & 1))) & 0xFF);
+            const int8_t hi = (int8_t)((w[k >> 1] >> (16 * (k & 1) + 8)) & 0xFF);
+            out[k] = pack_bf16((float)lo * d, (float)hi * d);
+          }
+          o = make_uint4(out[0], out[1], out[2], out[3]);
+        }
         *reinterpret_cast<uint4*>(conv + r * CP + c) = o;
       }
       __syncthreads();
@@ -224,7 +269,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_mma_kernel(DecodeParams p)
       for (int e = 0; e < 2; ++e) {
         int jl = hf * 16 + n * 8 + 2 * (lane & 3) + e;
         int j = jb + jl;
-        float ksc = FP8 ? scs[stage * TT + jl] : 1.f;
+        float ksc = KIND == 1 ? scs[stage * TT + jl] : 1.f;
         tsc[n][e] = ksc;
         float f = p.scale_log2 * ksc;
         float vlo = (j < vis_lo && j < j_end) ? sacc[n][e] * f : -CUDART_INF_F;
@@ -369,16 +414,21 @@ cudaError_t launch_decode_mma(const mla_decode_args_t* a, int splits, cudaStream
   dim3 grid(groups, splits, a->B);
   static PerDeviceOnce attrs;
   cudaError_t e = once_per_device(attrs, [&]() {
-    cudaError_t e2 = cudaFuncSetAttribute(decode_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)Smem<true>::total);
+    cudaError_t e2 = cudaFuncSetAttribute(decode_mma_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)Smem<0>::total);
     if (e2 != cudaSuccess) return e2;
-    return cudaFuncSetAttribute(decode_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)Smem<false>::total);
+    e2 = cudaFuncSetAttribute(decode_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)Smem<1>::total);
+    if (e2 != cudaSuccess) return e2;
+    return cudaFuncSetAttribute(decode_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)Smem<2>::total);
   });
   if (e != cudaSuccess) return e;
   if (a->kv_dtype == MLA_KV_FP8_E4M3)
-    return launch_pdl(decode_mma_kernel<true>, grid, dim3(NTHREADS), Smem<true>::total, stream, p);
-  return launch_pdl(decode_mma_kernel<false>, grid, dim3(NTHREADS), Smem<false>::total, stream, p);
+    return launch_pdl(decode_mma_kernel<1>, grid, dim3(NTHREADS), Smem<1>::total, stream, p);
+  if (a->kv_dtype == MLA_KV_Q8_0)
+    return launch_pdl(decode_mma_kernel<2>, grid, dim3(NTHREADS), Smem<2>::total, stream, p);
+  return launch_pdl(decode_mma_kernel<0>, grid, dim3(NTHREADS), Smem<0>::total, stream, p);
 }
 
 int decode_mma_tiles(int len) { return (len + TT - 1) / TT; }

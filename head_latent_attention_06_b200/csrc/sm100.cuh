@@ -51,6 +51,21 @@ MLA_DEVI void mbar_arrive_remote_relaxed(uint32_t addr) {
 MLA_DEVI void mbar_arrive_expect_tx_local(uint32_t addr, uint32_t tx) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(addr), "r"(tx) : "memory");
 }
+// Arrive (count 1) on a barrier of this CTA.
+MLA_DEVI void mbar_arrive_local(uint32_t addr) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+// Counts `tx` bytes as arrived on a barrier of this CTA without any copy (the
+// teardown after a timeout uses it to stand in for bytes that will never come).
+MLA_DEVI void mbar_complete_tx_local(uint32_t addr, uint32_t tx) {
+  asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(addr), "r"(tx) : "memory");
+}
+// 32-bit load from shared memory of either CTA of the cluster (mapa address).
+MLA_DEVI uint32_t ld_shared_cluster_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
 // try_wait with acquire at CTA scope (TMA bytes and tcgen05 commits) or at
 // cluster scope (arrivals of the peer CTA's threads after their own writes).
 template <bool kCluster = false>
@@ -76,17 +91,53 @@ MLA_DEVI bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity (test_wait returns at
+// once, where try_wait may suspend the thread for a while).
+template <bool kCluster = false>
+MLA_DEVI bool mbar_test_wait(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  if (kCluster) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity)
+        : "memory");
+  }
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity.  Bounded: gives up after
 // `limit_ns` of wall time or as soon as *abort is set, records
-// MLA_ERR_DEVICE_TIMEOUT in `status` when it times out, and returns false.
+// MLA_ERR_DEVICE_TIMEOUT in `status` when it times out, and returns false.  The
+// clock and the abort flag are read after the second unsuccessful poll and then
+// every 256 polls.  A limit of 1 ns gives up as soon as a non-blocking test
+// finds the phase incomplete (the device clock may advance in steps much coarser
+// than 1 ns, and one try_wait may itself wait a while).
 template <bool kCluster = false>
 MLA_DEVI bool mbar_wait(uint32_t addr, uint32_t parity, volatile int* abort, uint32_t* status,
                         uint64_t limit_ns) {
-  if (mbar_try_wait<kCluster>(addr, parity)) return true;
+  if (limit_ns <= 1 ? mbar_test_wait<kCluster>(addr, parity) : mbar_try_wait<kCluster>(addr, parity)) return true;
+  if (limit_ns <= 1) {
+    if (!*abort) {
+      *abort = 1;
+      set_status(status, MLA_ERR_DEVICE_TIMEOUT);
+    }
+    return false;
+  }
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait<kCluster>(addr, parity)) return true;
-    if ((it & 255u) == 0) {
+    if ((it & 255u) == 0 || it == 1) {
       if (*abort) return false;
       if (globaltimer() - t0 > limit_ns) {
         *abort = 1;
@@ -102,11 +153,21 @@ MLA_DEVI bool mbar_wait(uint32_t addr, uint32_t parity, volatile int* abort, uin
 template <bool kCluster = false>
 MLA_DEVI bool mbar_wait_converged(uint32_t addr, uint32_t parity, volatile int* abort, uint32_t* status,
                                   uint64_t limit_ns) {
-  if (__all_sync(0xffffffffu, mbar_try_wait<kCluster>(addr, parity))) return true;
+  if (__all_sync(0xffffffffu, limit_ns <= 1 ? mbar_test_wait<kCluster>(addr, parity)
+                                             : mbar_try_wait<kCluster>(addr, parity)))
+    return true;
+  if (limit_ns <= 1) {
+    if ((threadIdx.x & 31) == 0 && !*abort) {
+      *abort = 1;
+      set_status(status, MLA_ERR_DEVICE_TIMEOUT);
+    }
+    __syncwarp();
+    return false;
+  }
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (__all_sync(0xffffffffu, mbar_try_wait<kCluster>(addr, parity))) return true;
-    if ((it & 255u) == 0) {
+    if ((it & 255u) == 0 || it == 1) {
       int stop = 0;
       if ((threadIdx.x & 31) == 0) {
         if (*abort) {
@@ -251,10 +312,30 @@ MLA_DEVI uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return d;
 }
 
+// Shared-memory matrix descriptor with a given swizzle: layout-type field
+// (bits 61..63) 2 = 128-byte, 4 = 64-byte, 6 = 32-byte swizzle.
+MLA_DEVI uint64_t desc_swz(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)layout << 61;
+  return d;
+}
+constexpr uint32_t kLayoutSw128 = 2, kLayoutSw64 = 4;
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
          ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// kind::f8f6f4 with e4m3 A and B and fp32 D: the e4m3 format code is 0, so the
+// bits equal those of f16 x f16 -> f32; only the instruction's kind differs.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // Same for f16 A and B (format fields 0).
@@ -303,6 +384,27 @@ MLA_DEVI void mma_pair_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// e4m3 x e4m3 (kind::f8f6f4, K = 32 per instruction) forms of the two above.
+MLA_DEVI void mma_pair_f8_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 rx;\n\t"
+      "elect.sync rx|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+MLA_DEVI void mma_pair_f8_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                   uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 rx;\n\t"
+      "elect.sync rx|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive once on the barrier at offset `bar` in every CTA of `cta_mask` when all
 // previously issued tcgen05 operations of this thread have completed.
 MLA_DEVI void commit_pair_mc_elect(uint32_t bar, uint16_t cta_mask) {
@@ -346,8 +448,23 @@ MLA_DEVI void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
       "r"(v[30]), "r"(v[31])
       : "memory");
 }
+MLA_DEVI void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
 MLA_DEVI void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 MLA_DEVI void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 2^x with the hardware approximation (MUFU), flushing subnormal results to 0.
+MLA_DEVI float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 MLA_DEVI void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

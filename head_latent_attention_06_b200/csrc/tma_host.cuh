@@ -1,5 +1,5 @@
-// Host-side TMA tensor maps (bf16, 128-byte swizzle), cached by their parameters
-// so that a repeated call re-encodes nothing.
+// Host-side TMA tensor maps (bf16 with 128-byte swizzle unless stated), cached by
+// their parameters so that a repeated call re-encodes nothing.
 #pragma once
 
 #include <cuda.h>
@@ -21,8 +21,9 @@ bool tma_map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint6
 // strides[i] the byte stride of dimension i + 1 (any order, multiples of 16),
 // boxes of box[i] values.  The box lands in shared memory with dimension 0
 // fastest, so a stride smaller than the row pitch can order several chunks of a
-// row one after another.
+// row one after another.  `bytes`: 1-byte elements (e4m3 codes) instead of bf16;
+// swizzle_bytes: 128, 64, 32 or 0 (none).
 bool tma_map_nd(CUtensorMap* m, const void* ptr, uint32_t rank, const uint64_t* dims, const uint64_t* strides,
-                const uint32_t* box);
+                const uint32_t* box, bool bytes = false, int swizzle_bytes = 128);
 
 }  // namespace mla

@@ -13,7 +13,7 @@
  *
  *   mla_absorb_q       q_lat = W_UK^T q_nope                 (per head)
  *   mla_decode_paged   scores, online softmax, o_lat = P c   (split-KV partials)
- *   mla_combine_splits log-sum-exp merge of the partials     (no-op for 1 split)
+ *   mla_combine_splits log-sum-exp merge of the partials     (no-op when none)
  *   mla_up_proj_v      o = W_UV o_lat                         (per head)
  * and mla_write_kv appends new tokens (latent, RoPE key, bf16 or e4m3) to the
  * cache before the decode that reads them.
@@ -62,7 +62,10 @@ typedef enum {
   MLA_ERR_BAD_SEQ_LEN = 8           /* seq_lens[b] < 0 or > max_pages_per_seq*page_size (device-side) */
 } mla_status_t;
 
-typedef enum { MLA_KV_BF16 = 0, MLA_KV_FP8_E4M3 = 1 } mla_kv_dtype_t;
+/* Cache formats of a 576-value row: bf16 values; e4m3 codes with one fp32 scale
+ * per row (value = code * scale); q8_0 int8 codes with one fp16 scale per block
+ * of 32 consecutive values (value = code * block scale, 18 blocks a row). */
+typedef enum { MLA_KV_BF16 = 0, MLA_KV_FP8_E4M3 = 1, MLA_KV_Q8_0 = 2 } mla_kv_dtype_t;
 
 /* Supported dimensions: d_c = 512, d_r = 64, d_n = d_v = 128, page_size = 64,
  * H a multiple of 16 up to 128, 1 <= s_q <= MLA_MAX_S_Q.  s_q > 1 covers
@@ -97,9 +100,11 @@ typedef struct {
   const void* q_lat;              /* bf16 [B][s_q][H][d_c], output of mla_absorb_q */
   const void* q_pe;               /* bf16 [B][s_q][H][d_r], RoPE already applied */
   const void* kv_cache;           /* [num_pages][page_size][d_c + d_r]: row = c || k_pe,
-                                     bf16 (MLA_KV_BF16) or e4m3 (MLA_KV_FP8_E4M3) */
-  const float* kv_scale;          /* fp32 [num_pages][page_size], per-token dequant scale of the
-                                     whole row (value = e4m3 * scale); NULL for bf16 */
+                                     bf16 (MLA_KV_BF16), e4m3 (MLA_KV_FP8_E4M3) or int8
+                                     (MLA_KV_Q8_0) */
+  const void* kv_scale;           /* e4m3: fp32 [num_pages][page_size], the scale of the whole
+                                     row; q8_0: fp16 [num_pages][page_size][18], the scale of
+                                     each 32-value block, 4-byte aligned; NULL for bf16 */
   const int32_t* block_table;     /* int32 [B][max_pages_per_seq]: physical page of each
                                      64-token logical page */
   const int32_t* seq_lens;        /* int32 [B], device: cached tokens of sequence b, including
@@ -127,7 +132,9 @@ typedef struct {
  * device access).  Depends on B, s_q, H and the split count that will be used. */
 mla_status_t mla_decode_workspace_size(const mla_decode_args_t* args, size_t* bytes);
 
-/* The split count mla_decode_paged will use for these arguments (host only). */
+/* The split count mla_decode_paged will use for these arguments (host only):
+ * args->num_splits when it is set, else the count that minimises a model of the
+ * kernel's makespan on this device's SMs. */
 mla_status_t mla_decode_num_splits(const mla_decode_args_t* args, int32_t* num_splits);
 
 /*
@@ -138,10 +145,11 @@ mla_status_t mla_decode_num_splits(const mla_decode_args_t* args, int32_t* num_s
  *   s_j   = softmax_scale * (q_lat . c_j + q_pe . k_pe_j)
  *   o_lat = sum_j softmax(s)_j c_j ,   lse = log sum_j exp(s_j)
  * Token j is row j % page_size of page block_table[b][j / page_size].  Rows of a
- * last page at positions >= L_b are read but weigh nothing; they must hold finite
- * values.  With one split the results go straight to o_lat / lse; with more,
- * fp32 partials go to the workspace and mla_combine_splits must follow on the
- * same stream.  A query with no visible token gets o_lat = 0 and lse = -inf.
+ * last page at positions >= L_b are read but weigh nothing, whatever they hold.
+ * With one split the results go straight to o_lat / lse; with more, fp32
+ * partials go to the workspace.  Always follow with mla_combine_splits on the
+ * same stream (it enqueues nothing when one split was used).  A query with no
+ * visible token gets o_lat = 0 and lse = -inf.
  */
 mla_status_t mla_decode_paged(const mla_decode_args_t* args, void* stream);
 
@@ -210,8 +218,8 @@ typedef struct {
                                      d_c .. d_c+d_r-1 the RoPE key's projection W_KR */
   void* kv_cache;                 /* [num_pages][page_size][d_c + d_r], bf16 or e4m3; only the
                                      new tokens' rows are written */
-  float* kv_scale;                /* fp32 [num_pages][page_size]: e4m3 only, written at the new
-                                     rows; NULL for bf16 */
+  void* kv_scale;                 /* written at the new rows: e4m3: fp32 [num_pages][page_size];
+                                     q8_0: fp16 [num_pages][page_size][18]; NULL for bf16 */
   const int32_t* block_table;     /* int32 [B][max_pages_per_seq]: physical page of each
                                      64-token logical page */
   const int32_t* seq_lens;        /* int32 [B], device: lengths including the s_q new tokens */
@@ -243,6 +251,9 @@ mla_status_t mla_write_kv_workspace_size(const mla_write_kv_args_t* args, size_t
  * "FlashMLA", "KV cache with MLA": the latent cache may be quantised): one fp32
  * scale per 576-value row, scale = amax / 448 (1 for an all-zero row), codes =
  * the fp32 quotients value / scale rounded to nearest even, saturated at +-448.
+ * q8_0 cache (the format those docs recommend): per block of 32 values, d =
+ * amax / 127 (computed in fp32) rounded to fp16, codes = the fp32 quotients
+ * value / d rounded to nearest even, clamped to +-127 (0 for an all-zero block).
  * The projections accumulate in fp32.  No other cache row is touched.  A length
  * below s_q or beyond the block table (MLA_ERR_BAD_SEQ_LEN) or a page id outside
  * the cache (MLA_ERR_BAD_BLOCK_TABLE) is recorded in the workspace's status word
@@ -263,6 +274,17 @@ mla_status_t mla_get_status(void* workspace, void* stream);
  * after it returns; a CUDA graph keeps the kernels it captured. */
 typedef enum { MLA_DECODE_AUTO = 0, MLA_DECODE_WARP_MMA = 1 } mla_decode_kernel_t;
 mla_status_t mla_set_decode_kernel(int32_t kernel);
+
+/* Limit, in nanoseconds, of every bounded wait inside the decode kernels
+ * (process-wide; 0 restores the default of 2 s).  A wait that runs out records
+ * MLA_ERR_DEVICE_TIMEOUT in the status word, and the kernel waits for its copies
+ * in flight, frees its tensor memory and returns, leaving the context usable.
+ * Takes effect for launches after it returns (a CUDA graph keeps the limit it
+ * captured).  A limit of 1 ns gives up at the first wait that a non-blocking
+ * test finds unsatisfied (the device clock may advance in steps much coarser
+ * than 1 ns).
+ * Meant for tests and diagnosis; the default suits every workload. */
+mla_status_t mla_set_device_wait_limit(uint64_t ns);
 
 /* Human-readable name of a status code (static storage). */
 const char* mla_status_string(mla_status_t status);

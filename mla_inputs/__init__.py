@@ -12,5 +12,6 @@ d_c = 512 latent ``c_KV`` plus a decoupled 64-wide RoPE key (DeepSeek-V2 summary
 
 from .workloads import (  # noqa: F401
     D_C, D_R, D_N, D_V, PAGE, ROW, SOFTMAX_SCALE,
-    Workload, WorkloadSpec, PRESETS, preset, make_workload, bf16_bits, fp8_bits,
+    Workload, WorkloadSpec, PRESETS, preset, make_workload, bf16_bits, fp8_bits, int8_bits, f16_bits,
+    row_bytes,
 )

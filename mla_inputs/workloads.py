@@ -10,6 +10,9 @@ Draw recipe (fixed; changing it changes every stored expectation):
   the cast, except the fp8 cache below;
 * fp8 cache: each 576-value row is scaled by ``amax(row) / 448`` and cast to
   float8 e4m3fn (round to nearest even); the fp32 scale is stored per token;
+* q8_0 cache: each block of 32 consecutive values of a row gets the scale
+  ``d = amax(block) / 127`` rounded to fp16, and int8 codes ``round(x / d)``
+  (nearest even, in fp32, clamped to [-127, 127]; 0 for an all-zero block);
 * rows of a sequence's last page at positions >= its length hold finite values
   50x larger than the real rows, so that a kernel that forgets to mask them
   produces a visibly wrong answer.
@@ -36,6 +39,8 @@ ROW = D_C + D_R  # 576 values per cached token
 SOFTMAX_SCALE = 1.0 / math.sqrt(D_N + D_R)  # 1/sqrt(192)
 TAIL_GAIN = 50.0
 FP8_MAX = 448.0
+Q8_BLOCK = 32     # q8_0: values per scale block
+Q8_LEVELS = 127   # q8_0: largest code
 
 
 @dataclass
@@ -45,7 +50,7 @@ class WorkloadSpec:
     H: int
     s_q: int
     lens: Optional[Sequence[int]]  # explicit lengths; None => ragged draw
-    kv_dtype: str = "bf16"  # "bf16" | "fp8"
+    kv_dtype: str = "bf16"  # "bf16" | "fp8" | "q8_0"
     causal: bool = False
     seed: int = 0
     permute_pages: bool = True
@@ -75,6 +80,10 @@ PRESETS = {
                         causal=True, seed=4,
                         note="batch 128, 128 heads, 8192 tokens, e4m3 cache + fp32 per-token "
                              "scale, 2 causal query tokens"),
+    # the V3 shape over the blockwise q8_0 cache (ik_llama.cpp's recommended MLA cache type)
+    "q8": WorkloadSpec("q8", B=64, H=128, s_q=1, lens=[4096] * 64, kv_dtype="q8_0", seed=5,
+                       note="DeepSeek-V3-shaped: batch 64, 128 heads, 4096 tokens, q8_0 cache "
+                            "(int8 codes, fp16 scale per 32 values)"),
 }
 
 
@@ -93,7 +102,7 @@ class Workload:
     w_uk: torch.Tensor            # bf16 [H][128][512]   k = W_UK[h] . c
     w_uv: torch.Tensor            # bf16 [H][128][512]   v = W_UV[h] . c
     kv_cache: torch.Tensor        # bf16 or float8_e4m3fn [num_pages][64][576]
-    kv_scale: Optional[torch.Tensor]  # fp32 [num_pages][64] (fp8 only)
+    kv_scale: Optional[torch.Tensor]  # fp32 [num_pages][64] (fp8), fp16 [num_pages][64][18] (q8_0)
     raw_rows: Optional[torch.Tensor] = None  # fp32 [num_pages][64][576] draws (keep_raw only)
     softmax_scale: float = SOFTMAX_SCALE
     extra: dict = field(default_factory=dict)
@@ -125,8 +134,12 @@ class Workload:
 
     def cache_bytes(self) -> int:
         """Bytes of cache rows the step must read: sum of lengths x row bytes."""
-        per = ROW * (2 if self.spec.kv_dtype == "bf16" else 1) + (4 if self.spec.kv_dtype == "fp8" else 0)
-        return sum(self.lens) * per
+        return sum(self.lens) * row_bytes(self.spec.kv_dtype)
+
+
+def row_bytes(kv_dtype: str) -> int:
+    """Bytes one cached token occupies: 576 values, plus their scales."""
+    return {"bf16": 2 * ROW, "fp8": ROW + 4, "q8_0": ROW + 2 * (ROW // Q8_BLOCK)}[kv_dtype]
 
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
@@ -141,11 +154,33 @@ def fp8_bits(t: torch.Tensor) -> np.ndarray:
     return t.contiguous().view(torch.uint8).numpy()
 
 
+def int8_bits(t: torch.Tensor) -> np.ndarray:
+    """uint8 view of an int8 tensor."""
+    assert t.dtype == torch.int8
+    return t.contiguous().view(torch.uint8).numpy()
+
+
+def f16_bits(t: torch.Tensor) -> np.ndarray:
+    """uint16 view of a float16 tensor."""
+    assert t.dtype == torch.float16
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
 def _quantise_rows_e4m3(rows: torch.Tensor):
     amax = rows.abs().amax(dim=-1, keepdim=True)
     scale = torch.where(amax > 0, amax / FP8_MAX, torch.ones_like(amax))
     q = (rows / scale).clamp_(-FP8_MAX, FP8_MAX).to(torch.float8_e4m3fn)
     return q, scale.squeeze(-1).to(torch.float32)
+
+
+def _quantise_rows_q8_0(rows: torch.Tensor):
+    blocks = rows.reshape(*rows.shape[:-1], ROW // Q8_BLOCK, Q8_BLOCK)
+    d = (blocks.abs().amax(dim=-1) / Q8_LEVELS).to(torch.float16)
+    df = d.to(torch.float32)
+    safe = torch.where(df > 0, df, torch.ones_like(df))
+    q = torch.round(blocks / safe[..., None]).clamp_(-Q8_LEVELS, Q8_LEVELS)
+    q = torch.where(df[..., None] > 0, q, torch.zeros_like(q))
+    return q.to(torch.int8).reshape(rows.shape), d
 
 
 def make_workload(spec: WorkloadSpec, keep_raw: bool = False) -> Workload:
@@ -181,9 +216,13 @@ def make_workload(spec: WorkloadSpec, keep_raw: bool = False) -> Workload:
     # Cache rows, drawn in logical order (sequence by sequence, page by page) and
     # stored at their physical page.  Tail rows of a last page get TAIL_GAIN.
     fp8 = spec.kv_dtype == "fp8"
+    q8 = spec.kv_dtype == "q8_0"
     if fp8:
         kv_cache = torch.zeros(num_pages, PAGE, ROW, dtype=torch.float8_e4m3fn)
         kv_scale = torch.ones(num_pages, PAGE, dtype=torch.float32)
+    elif q8:
+        kv_cache = torch.zeros(num_pages, PAGE, ROW, dtype=torch.int8)
+        kv_scale = torch.zeros(num_pages, PAGE, ROW // Q8_BLOCK, dtype=torch.float16)
     else:
         kv_cache = torch.zeros(num_pages, PAGE, ROW, dtype=torch.bfloat16)
         kv_scale = None
@@ -203,6 +242,10 @@ def make_workload(spec: WorkloadSpec, keep_raw: bool = False) -> Workload:
                 raw[idx] = rows
             if fp8:
                 q, sc = _quantise_rows_e4m3(rows)
+                kv_cache[idx] = q
+                kv_scale[idx] = sc
+            elif q8:
+                q, sc = _quantise_rows_q8_0(rows)
                 kv_cache[idx] = q
                 kv_scale[idx] = sc
             else:

@@ -12,9 +12,14 @@ from .mla_oracle import (  # noqa: F401
 
 def from_workload(w) -> OracleInputs:
     """Raw bits of a ``mla_inputs.Workload`` wrapped for the oracle."""
-    from mla_inputs import bf16_bits, fp8_bits
-    kv = bf16_bits(w.kv_cache) if w.spec.kv_dtype == "bf16" else fp8_bits(w.kv_cache)
-    scale = None if w.kv_scale is None else w.kv_scale.numpy()
+    from mla_inputs import bf16_bits, f16_bits, fp8_bits, int8_bits
+    kind = w.spec.kv_dtype
+    if kind == "bf16":
+        kv, scale = bf16_bits(w.kv_cache), None
+    elif kind == "q8_0":
+        kv, scale = int8_bits(w.kv_cache), f16_bits(w.kv_scale)
+    else:
+        kv, scale = fp8_bits(w.kv_cache), w.kv_scale.numpy()
     return OracleInputs(bf16_bits(w.q_nope), bf16_bits(w.q_pe), bf16_bits(w.w_uk),
                         bf16_bits(w.w_uv), kv, w.spec.kv_dtype, scale,
                         w.block_table.numpy(), w.seq_lens.numpy(), w.softmax_scale,

@@ -120,6 +120,23 @@ def quantise_row_e4m3(row: np.ndarray) -> Tuple[np.ndarray, np.float32]:
     return f64_to_e4m3fn(np.clip(q.astype(np.float64), -E4M3_MAX, E4M3_MAX)), scale
 
 
+def quantise_row_q8_0(row: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """One 576-value row -> (int8 codes [576], fp16 scales [18]) of the q8_0 format
+    (ik_llama.cpp docs "FlashMLA", section "KV cache with MLA"; blocks of 32
+    values, d = amax / 127 rounded to fp16, codes round(x / d) in [-127, 127]).
+    The row is taken at fp32 precision and amax / 127 and the quotients are fp32
+    IEEE operations, as for the e4m3 row."""
+    r32 = np.asarray(row, dtype=np.float64).astype(np.float32).reshape(-1, 32)
+    amax = np.max(np.abs(r32), axis=1)
+    d16 = (amax / np.float32(127.0)).astype(np.float32).astype(np.float16)
+    d32 = d16.astype(np.float32)
+    safe = np.where(d32 > 0, d32, np.float32(1.0))
+    q = np.rint((r32 / safe[:, None]).astype(np.float32))
+    q = np.clip(q, -127, 127)
+    q = np.where(d32[:, None] > 0, q, 0)
+    return q.astype(np.int8).reshape(-1), d16
+
+
 def slot_of(block_table: np.ndarray, seq_lens: np.ndarray, s_q: int, b: int, i: int,
             num_pages: int) -> Tuple[int, int]:
     """(physical page, row) of new token i of sequence b."""
@@ -141,13 +158,16 @@ def write_kv(h: np.ndarray, w_dkv: np.ndarray, w_kr: np.ndarray, kv: np.ndarray,
     returns (kv, kv_scale).
 
     h [B][s_q][d_h] (fp64 values), w_dkv [512][d_h], w_kr [64][d_h]; kv holds raw
-    bits [num_pages][64][576] (uint16 bf16 or uint8 e4m3) and kv_scale fp32
-    [num_pages][64] for e4m3.  Every row other than the new tokens' is left as it
-    was."""
-    assert kv_dtype in ("bf16", "fp8")
+    bits [num_pages][64][576] (uint16 bf16, uint8 e4m3, int8 q8_0 codes); kv_scale
+    is fp32 [num_pages][64] for e4m3, fp16 [num_pages][64][18] for q8_0.  Every
+    row other than the new tokens' is left as it was."""
+    assert kv_dtype in ("bf16", "fp8", "q8_0")
     B = h.shape[0]
     kv = np.array(kv, copy=True)
-    kv_scale = None if kv_scale is None else np.array(kv_scale, dtype=np.float32, copy=True)
+    if kv_dtype == "q8_0":
+        kv_scale = np.array(kv_scale, dtype=np.float16, copy=True)
+    else:
+        kv_scale = None if kv_scale is None else np.array(kv_scale, dtype=np.float32, copy=True)
     for b in range(B):
         c, kr = compress(h[b], w_dkv, w_kr)                       # [s_q][512], [s_q][64]
         pos = int(seq_lens[b]) - s_q + np.arange(s_q)
@@ -157,6 +177,8 @@ def write_kv(h: np.ndarray, w_dkv: np.ndarray, w_kr: np.ndarray, kv: np.ndarray,
             full = np.concatenate([c[i], k_pe[i]])
             if kv_dtype == "bf16":
                 kv[page, row] = f64_to_bf16(full)
+            elif kv_dtype == "q8_0":
+                kv[page, row], kv_scale[page, row] = quantise_row_q8_0(full)
             else:
                 kv[page, row], kv_scale[page, row] = quantise_row_e4m3(full)
     return kv, kv_scale

@@ -40,6 +40,7 @@ import numpy as np
 PAGE = 64
 D_C = 512
 D_R = 64
+Q8_BLOCK = 32
 
 
 # ----------------------------------------------------------------------------
@@ -65,6 +66,20 @@ def e4m3fn_to_f64(bits: np.ndarray) -> np.ndarray:
     return np.where((e == 15) & (m == 7), np.nan, v)
 
 
+def f16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """IEEE binary16: 1 sign, 5 exponent (bias 15), 10 mantissa bits; exponent 0
+    is subnormal (m/1024 * 2^-14); exponent 31 is inf (m = 0) or NaN."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.int64)
+    sign = np.where(b & 0x8000, -1.0, 1.0)
+    e = (b >> 10) & 0x1F
+    m = (b & 0x3FF).astype(np.float64)
+    normal = (1.0 + m / 1024.0) * np.exp2(e.astype(np.float64) - 15.0)
+    sub = (m / 1024.0) * 2.0 ** -14
+    v = np.where(e == 0, sub, normal)
+    v = np.where(e == 31, np.where(m == 0, np.inf, np.nan), v)
+    return v * sign
+
+
 # ----------------------------------------------------------------------------
 # Inputs
 # ----------------------------------------------------------------------------
@@ -73,10 +88,15 @@ class OracleInputs:
     """Raw bits of one decode step, as the cache and the queries hold them.
 
     q_nope [B][s_q][H][128] and q_pe [B][s_q][H][64] as bf16 bits; w_uk, w_uv
-    [H][128][512] bf16 bits; kv [num_pages][64][576] as bf16 (uint16) or e4m3
-    (uint8) bits; kv_scale fp32 [num_pages][64] for e4m3 (else None);
-    block_table int [B][max_pages]; seq_lens int [B] (lengths include the s_q new
-    tokens).
+    [H][128][512] bf16 bits; kv [num_pages][64][576] as bf16 (uint16), e4m3
+    (uint8) or q8_0 (int8 codes, as uint8) bits; kv_scale fp32 [num_pages][64]
+    for e4m3, fp16 bits [num_pages][64][18] (one scale per 32-value block) for
+    q8_0, else None; block_table int [B][max_pages]; seq_lens int [B] (lengths
+    include the s_q new tokens).
+
+    q8_0 (ik_llama.cpp docs "FlashMLA", section "KV cache with MLA": the
+    recommended quantised MLA cache): value = code * the block's scale, blocks of
+    32 consecutive values of the 576-value row.
     """
 
     def __init__(self, q_nope, q_pe, w_uk, w_uv, kv, kv_dtype, kv_scale, block_table,
@@ -87,13 +107,16 @@ class OracleInputs:
         self.w_uv = bf16_to_f64(w_uv)
         self.kv = np.asarray(kv)
         self.kv_dtype = kv_dtype
-        self.kv_scale = None if kv_scale is None else np.asarray(kv_scale, dtype=np.float64)
+        if kv_dtype == "q8_0":
+            self.kv_scale = f16_to_f64(kv_scale)
+        else:
+            self.kv_scale = None if kv_scale is None else np.asarray(kv_scale, dtype=np.float64)
         self.block_table = np.asarray(block_table, dtype=np.int64)
         self.seq_lens = np.asarray(seq_lens, dtype=np.int64)
         self.softmax_scale = float(softmax_scale)
         self.causal = bool(causal)
         self.B, self.s_q, self.H, _ = self.q_nope.shape
-        assert kv_dtype in ("bf16", "fp8")
+        assert kv_dtype in ("bf16", "fp8", "q8_0")
 
     def visible(self, b: int, i: int) -> int:
         """Number of cached tokens query i of sequence b attends to."""
@@ -112,6 +135,10 @@ class OracleInputs:
         raw = self.kv[pages].reshape(npg * PAGE, D_C + D_R)[:n]
         if self.kv_dtype == "bf16":
             return bf16_to_f64(raw)
+        if self.kv_dtype == "q8_0":
+            codes = raw.astype(np.uint8).view(np.int8).astype(np.float64)          # [n][576]
+            block = self.kv_scale[pages].reshape(npg * PAGE, -1)[:n]               # [n][18]
+            return codes * np.repeat(block, Q8_BLOCK, axis=1)
         scale = self.kv_scale[pages].reshape(npg * PAGE)[:n]
         return e4m3fn_to_f64(raw) * scale[:, None]
 

@@ -78,9 +78,11 @@ def test_auto_split_count(lib):
     assert mla.mla_decode_num_splits(_args(B=4, H=16, max_len=131072)) >= 16
     assert mla.mla_decode_num_splits(_args(B=4, H=128, max_len=131072)) >= 16
     assert mla.mla_decode_num_splits(_args(B=64, H=128, max_len=4096)) == 1
-    assert mla.mla_decode_num_splits(_args(B=128, H=128, max_len=8192, s_q=2)) <= 2
     assert mla.mla_decode_num_splits(_args(B=1, H=16, max_len=64)) == 1
     assert mla.mla_decode_num_splits(_args(B=4, H=16, splits=7)) == 7
+    # e4m3 cache: the same model
+    assert mla.mla_decode_num_splits(_args(B=4, H=128, max_len=131072, kv_dtype=1)) >= 16
+    assert mla.mla_decode_num_splits(_args(B=128, H=128, max_len=8192, s_q=2, kv_dtype=1)) <= 2
 
 
 @pytest.mark.parametrize("field,value,code", [

@@ -25,8 +25,9 @@ def test_traffic_reported_only_for_the_profiled_source():
     # the record names the sha256 of the kernel source it was measured on; any
     # other source (or workload) gets no traffic figure
     assert bench.decode_traffic("tiny") is None
-    value = bench.decode_traffic("v3")
-    assert value is None or value == bench.MEASURED_TRAFFIC["v3"][0]
+    for config, (nbytes, src, sha) in bench.MEASURED_TRAFFIC.items():
+        value = bench.decode_traffic(config)
+        assert value == (nbytes if bench.kernel_source_digest(src) == sha else None)
 
 
 def test_cpu_model_is_text():
@@ -40,3 +41,13 @@ def test_nonabsorbed_sample_extrapolates_by_tokens_and_heads():
     est = r["us_per_token_head"] * 256 * 16 * 1e-6
     assert abs(r["extrapolated_full_s"] - est) <= 1e-3 * est + 1e-4
     assert "extrapolated" in r["sample"]
+
+
+def test_tensor_peak_follows_the_mma_kind():
+    peaks = {"bf16_tflops": 1640.7, "hbm_gbs": 6550.4}
+    assert bench.tensor_peak(peaks, "bf16")[0] == 1640.7
+    # e4m3 x e4m3: the measured bf16 figure x the nominal fp8 / bf16 ratio (4.5 / 2.25)
+    assert bench.tensor_peak(peaks, "fp8")[0] == 2 * 1640.7
+    assert bench.tensor_peak(dict(peaks, fp8_tflops=3100.0), "fp8")[0] == 3100.0
+    f = bench.datasheet_fracs(608.2e6, 584.1e9, 1e-3, "fp8")
+    assert abs(f["tensor_frac"] - 584.1e9 / 4500e12 / 1e-3) < 1e-6

@@ -225,3 +225,41 @@ def test_single_written_token_decodes_to_w_uv_c():
         s = (om.bf16_to_f64(q_nope[0, 0, hh]) @ (om.bf16_to_f64(w_uk[hh]) @ c)
              + om.bf16_to_f64(q_pe[0, 0, hh]) @ k_pe) / np.sqrt(192.0)
         assert out["lse"][0, 0, hh] == pytest.approx(s, rel=2e-2, abs=2e-2)
+
+
+def test_q8_0_row_quantisation_matches_the_blockwise_format():
+    """The cache write's q8_0 row (fp32 arithmetic) against the low-bit oracle's
+    blockwise quantiser (fp64): scales equal, codes equal except where an fp32
+    quotient falls on the other side of a rounding boundary than the exact one."""
+    from oracle import lowbit_cache as lb
+    rng = np.random.default_rng(11)
+    diff = 0
+    for _ in range(200):
+        row = rng.standard_normal(576) * rng.uniform(0.01, 50.0)
+        row32 = row.astype(np.float32).astype(np.float64)
+        codes, d = cw.quantise_row_q8_0(row)
+        ref_codes, ref_d = lb.quantise_blocks(row32, "q8_0")
+        assert np.array_equal(d.astype(np.float64), ref_d)
+        diff += int((codes.astype(np.int64) != ref_codes).sum())
+        assert np.abs(codes.astype(np.int64) - ref_codes).max() <= 1
+    assert diff <= 2e-4 * 200 * 576
+
+
+def test_q8_0_write_touches_only_the_new_rows():
+    rng = np.random.default_rng(12)
+    B, s_q, d_h, P = 2, 2, 64, 6
+    h = rng.standard_normal((B, s_q, d_h))
+    w_dkv, w_kr = rng.standard_normal((512, d_h)) / 8, rng.standard_normal((64, d_h)) / 8
+    kv = rng.integers(-127, 128, size=(P, 64, 576)).astype(np.int8)
+    sc = rng.random((P, 64, 18)).astype(np.float16)
+    bt = np.array([[3, 1], [0, 5]])
+    lens = np.array([66, 10])
+    kv2, sc2 = cw.write_kv(h, w_dkv, w_kr, kv, sc, "q8_0", bt, lens, s_q)
+    changed = np.argwhere((kv2 != kv).any(axis=2) | (sc2 != sc).any(axis=2))
+    assert sorted(map(tuple, changed)) == [(0, 8), (0, 9), (1, 0), (1, 1)]
+    # the written row decodes to the compressed row within half a step per block
+    c, kr = cw.compress(h[0], w_dkv, w_kr)
+    full = np.concatenate([c[1], cw.rope(kr, np.array([65]), 10000.0)[1]])
+    got = kv2[1, 1].astype(np.float64) * np.repeat(sc2[1, 1].astype(np.float64), 32)
+    step = np.repeat(sc2[1, 1].astype(np.float64), 32)
+    assert np.all(np.abs(got - full) <= 0.5 * step + 1e-3 * np.abs(full) + 1e-9)

@@ -99,3 +99,48 @@ def test_rotation_reduces_low_bit_error_with_outliers():
         q, d = lb.quantise_blocks(h @ c, "q4_0")
         err_rot += np.sum((h.T @ lb.dequantise_blocks(q, d) - c) ** 2)
     assert err_rot < 0.5 * err_plain
+
+
+# ---------------------------------------------------------------- q8_0 cache in the decode oracle
+
+def test_f16_decoder_matches_numpy_on_every_code():
+    bits = np.arange(65536, dtype=np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = om.f16_to_f64(bits)
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(got))
+    assert np.array_equal(ref[~nan], got[~nan])
+
+
+def _q8_workload(lens=(70, 130), H=16, seed=3):
+    from mla_inputs import WorkloadSpec, make_workload
+    return make_workload(WorkloadSpec("q8", B=len(lens), H=H, s_q=1, lens=list(lens), kv_dtype="q8_0",
+                                      seed=seed), keep_raw=True)
+
+
+def test_q8_0_cache_rows_are_the_blockwise_dequantisation():
+    """The decode oracle reads a q8_0 cache row as code * block scale: the same
+    values the low-bit oracle's quantiser gives for the raw fp32 draw."""
+    import oracle
+    w = _q8_workload()
+    inp = oracle.from_workload(w)
+    raw = w.raw_rows.double().numpy()
+    for b, L in enumerate(w.lens):
+        C = inp.rows(b, L)
+        for j in (0, 31, L - 1):
+            pg, rr = int(w.block_table[b, j // 64]), j % 64
+            codes, d = lb.quantise_blocks(raw[pg, rr], "q8_0")
+            assert np.array_equal(C[j], lb.dequantise_blocks(codes, d))
+            # every value within half a step of its block (plus the fp16 rounding of d)
+            step = np.repeat(d, 32)
+            assert np.all(np.abs(C[j] - raw[pg, rr]) <= 0.5 * step + 1e-3 * np.abs(raw[pg, rr]) + 1e-12)
+
+
+def test_q8_0_decode_absorbed_equals_the_definition():
+    import oracle
+    w = _q8_workload(lens=(1, 200), H=16)
+    inp = oracle.from_workload(w)
+    a = om.decode_absorbed(inp)
+    d = om.decode_nonabsorbed(inp)
+    for key in ("o", "o_lat", "lse"):
+        assert np.allclose(a[key], d[key], rtol=1e-10, atol=1e-12)

@@ -174,9 +174,10 @@ def test_fp8_scale_magnitudes(cuda_lib, factor):
         assert np.abs(lse[b, 0] - ref_lse).max() <= amax
 
 
-def test_projections_against_oracle(cuda_lib):
+@pytest.mark.parametrize("n_tok,H", [(70, 128), (1, 16), (300, 16), (256, 128), (129, 48)])
+def test_projections_against_oracle(cuda_lib, n_tok, H):
+    """Token blocks of 64 / 128, a ragged last block, several CTAs per head (few heads)."""
     g = torch.Generator().manual_seed(5)
-    n_tok, H = 70, 128
     q = torch.randn(n_tok, H, 128, generator=g).to(torch.bfloat16)
     w_uk = (torch.randn(H, 128, 512, generator=g) / 512 ** 0.5).to(torch.bfloat16)
     x = torch.randn(n_tok, H, 512, generator=g).to(torch.bfloat16)
