@@ -357,6 +357,131 @@ def run_write_kv(args):
     return 0
 
 
+PREFILL_METRIC = "MLA chunked-prefill TFLOP/s (explicit K/V form) & % of tensor roofline; tokens/s"
+
+
+def prefill_flops(lens, H, s_q, causal):
+    """Algorithmic FLOPs of the explicit form: per (cached token, head) the two
+    up-projections k = W_UK c and v = W_UV c, 2 * 2 * 128 * 512; per (query,
+    visible token, head) the 192-wide score and the 128-wide value sum,
+    2 * (192 + 128)."""
+    up = sum(lens) * H * 2 * 2 * 128 * 512
+    vis = 0
+    for L in lens:
+        if causal:
+            vis += s_q * (L - s_q) + s_q * (s_q + 1) // 2
+        else:
+            vis += s_q * L
+    return up + vis * H * 2 * (192 + 128), up
+
+
+def run_prefill(args):
+    """Times mla_prefill on a chunked-prefill workload (s_q new tokens per
+    sequence on top of a cached prefix, causal): the per-head key / value
+    up-projection and the FlashAttention forward, replayed from a CUDA graph with
+    L2 flushed before each call.  The same chunk through the absorbed kernels is
+    timed beside it (the form the decode uses), and end to end with the queries
+    copied in from pinned host memory and the output copied back."""
+    import torch
+    import head_latent_attention_06_b200 as mla
+    from head_latent_attention_06_b200.step import prefill_from_workload, step_from_workload
+    from mla_inputs import make_workload, preset
+    torch.cuda.set_device(0)
+    mla.load()
+    spec = preset(args.config)
+    w = make_workload(spec)
+    st = prefill_from_workload(w)
+    stream = torch.cuda.current_stream()
+    st.run()                                 # outside capture: one-time host set-up
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        st.run()
+    flush_w = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    flush_r = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+
+    def timed_loop(g, n):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+        for k in range(n):
+            flush_w.zero_()
+            torch.sum(flush_r)
+            evs[k][0].record(stream)
+            g.replay()
+            evs[k][1].record(stream)
+        return evs
+
+    timed_loop(graph, max(3, args.warmup))
+    torch.cuda.synchronize()
+    assert mla.mla_get_status(st.workspace) == 0
+    with ClockSampler(0) as clk:
+        evs = timed_loop(graph, args.steps)
+        torch.cuda.synchronize()
+    assert mla.mla_get_status(st.workspace) == 0
+    ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+
+    absorbed_ms = None
+    if w.s_q <= 1024:
+        dec = step_from_workload(w)
+        g_dec = dec.capture()
+        timed_loop(g_dec, 3)
+        torch.cuda.synchronize()
+        n_dec = max(3, min(args.steps, 50))
+        ev = timed_loop(g_dec, n_dec)
+        torch.cuda.synchronize()
+        assert mla.mla_get_status(dec.workspace) == 0
+        absorbed_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / n_dec
+        del dec, g_dec
+
+    # end to end: queries, block table and lengths from pinned host memory, the
+    # output back to pinned host memory, every call
+    h_in = (w.q_nope.pin_memory(), w.q_pe.pin_memory(), w.block_table.pin_memory(), w.seq_lens.pin_memory())
+    d_in = (st._keep[0], st._keep[1], st._keep[5], st._keep[6])
+    h_out = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+    n_e2e = max(3, min(args.steps, 50))
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for rep in range(2):
+        n = 3 if rep == 0 else n_e2e
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(n):
+            for d, h in zip(d_in, h_in):
+                d.copy_(h, non_blocking=True)
+            st.run()
+            h_out.copy_(st.out, non_blocking=True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    e2e_ms = t0.elapsed_time(t1) / n_e2e
+    assert torch.equal(h_out, st.out.cpu())
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = h_out.numel() * h_out.element_size()
+
+    flops, up_flops = prefill_flops(w.lens, w.H, w.s_q, w.causal)
+    tflops = flops / (ms * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    tc_peak, tc_kind = tensor_peak(peaks, "bf16")
+    n_tok = w.B * w.s_q
+    cfg = _config_dict(args.config, w)
+    cfg.update({"path": "prefill", "form": "explicit: per-head K = [W_UK c ; k_pe], V = W_UV c, "
+                                           "then FlashAttention forward"})
+    line = {"metric": PREFILL_METRIC, "value": round(tflops, 2), "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 (fp32 accumulate; K, V and P in bf16)",
+            "data": "synthetic (seeded, N(0,1) activations and cache, N(0,1/512) weights)", "config": cfg,
+            "tokens_per_s": round(n_tok / (ms * 1e-3), 1),
+            "flops_per_step": flops, "kv_up_flops_per_step": up_flops,
+            "absorbed_form_ms": None if absorbed_ms is None else round(absorbed_ms, 4),
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tc_peak, "unit": "TFLOP/s",
+                         "frac": round(tflops / tc_peak, 4), "traffic": None,
+                         "peak_kind": f"{peak_kind}: {tc_kind}",
+                         "kernel": "mla_prefill (kv_up_kernel + prefill_attn_kernel, one call)"},
+            "e2e": {"value": round(flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
+            "gpu_launches": 2 * args.steps, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def _config_dict(name, w, splits=None):
     from mla_inputs import preset
     s = preset(name)
@@ -381,14 +506,17 @@ def main(argv=None):
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", default="decode", choices=["decode", "write_kv"],
-                    help="decode: the decode step (default); write_kv: the cache write of its new tokens")
+    ap.add_argument("--path", default="decode", choices=["decode", "write_kv", "prefill"],
+                    help="decode: the decode step (default); write_kv: the cache write of its new "
+                         "tokens; prefill: the explicit-form chunked prefill (--config prefill)")
     ap.add_argument("--d-h", dest="d_h", type=int, default=7168, help="hidden width for --path write_kv")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
     if args.path == "write_kv":
         return run_write_kv(args)
+    if args.path == "prefill":
+        return run_prefill(args)
 
     import torch
     import torch.distributed as dist

@@ -32,7 +32,8 @@ EXPORTS = ("mla_absorb_q", "mla_decode_workspace_size", "mla_decode_num_splits",
            "mla_decode_paged", "mla_combine_splits", "mla_up_proj_v", "mla_get_status",
            "mla_status_string", "mla_decode_paged_noalloc", "mla_noalloc_init",
            "mla_get_status_noalloc", "mla_write_kv_workspace_size", "mla_write_kv",
-           "mla_set_decode_kernel", "mla_set_device_wait_limit")
+           "mla_set_decode_kernel", "mla_set_device_wait_limit", "mla_prefill_workspace_size",
+           "mla_prefill")
 
 DECODE_AUTO, DECODE_WARP_MMA = 0, 1
 
@@ -74,6 +75,23 @@ class WriteKvArgs(ctypes.Structure):
     ]
 
 
+class PrefillArgs(ctypes.Structure):
+    """Mirror of ``mla_prefill_args_t`` (field order and types must match)."""
+    _fields_ = [
+        ("q_nope", ctypes.c_void_p), ("q_pe", ctypes.c_void_p),
+        ("w_uk", ctypes.c_void_p), ("w_uv", ctypes.c_void_p),
+        ("kv_cache", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+        ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("B", ctypes.c_int32), ("s_q", ctypes.c_int32), ("H", ctypes.c_int32),
+        ("d_c", ctypes.c_int32), ("d_r", ctypes.c_int32), ("page_size", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
+        ("kv_dtype", ctypes.c_int32), ("causal", ctypes.c_int32),
+        ("max_seq_len", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+    ]
+
+
 _lib: Optional[ctypes.CDLL] = None
 
 
@@ -101,6 +119,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     pw = ctypes.POINTER(WriteKvArgs)
     lib.mla_write_kv_workspace_size.argtypes = [pw, ctypes.POINTER(ctypes.c_size_t)]
     lib.mla_write_kv.argtypes = [pw, vp]
+    pp = ctypes.POINTER(PrefillArgs)
+    lib.mla_prefill_workspace_size.argtypes = [pp, ctypes.POINTER(ctypes.c_size_t)]
+    lib.mla_prefill.argtypes = [pp, vp]
     lib.mla_get_status.argtypes = [vp, vp]
     lib.mla_status_string.argtypes = [ctypes.c_int]
     lib.mla_status_string.restype = ctypes.c_char_p
@@ -336,6 +357,59 @@ def mla_write_kv(args: WriteKvArgs, stream=None):
     _check("mla_write_kv", load().mla_write_kv(ctypes.byref(args), _stream(stream)))
 
 
+def make_prefill_args(*, q_nope, q_pe, w_uk, w_uv, kv_cache, block_table, seq_lens, out, lse,
+                      max_seq_len, workspace=None, causal=True, softmax_scale) -> PrefillArgs:
+    """Fill a ``PrefillArgs`` from device tensors.  Shapes: q_nope [B][s_q][H][128],
+    q_pe [B][s_q][H][64], w_uk [H][128][512], w_uv [H][128][512], kv_cache
+    [num_pages][64][576] bf16, block_table [B][max_pages] int32, seq_lens [B] int32,
+    out [B][s_q][H][128] bf16, lse [B][s_q][H] fp32 or None; max_seq_len bounds
+    seq_lens and sizes the workspace."""
+    import torch
+    bf16, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    if q_nope.dim() != 4 or kv_cache.dim() != 3 or block_table.dim() != 2:
+        raise ValueError("q_nope must be [B][s_q][H][128], kv_cache [pages][64][576], block_table [B][pages]")
+    B, s_q, H, _ = q_nope.shape
+    P = kv_cache.shape[0]
+    _want([(q_nope, "q_nope", bf16, (B, s_q, H, D_N), False),
+           (q_pe, "q_pe", bf16, (B, s_q, H, D_R), False),
+           (w_uk, "w_uk", bf16, (H, D_N, D_C), False),
+           (w_uv, "w_uv", bf16, (H, D_V, D_C), False),
+           (kv_cache, "kv_cache", bf16, (P, PAGE, D_C + D_R), False),
+           (block_table, "block_table", i32, (B, block_table.shape[1]), False),
+           (seq_lens, "seq_lens", i32, (B,), False),
+           (out, "out", bf16, (B, s_q, H, D_V), False),
+           (lse, "lse", f32, (B, s_q, H), True),
+           (workspace, "workspace", torch.uint8, None, True)])
+    a = PrefillArgs()
+    a.q_nope, a.q_pe, a.w_uk, a.w_uv = _ptr(q_nope), _ptr(q_pe), _ptr(w_uk), _ptr(w_uv)
+    a.kv_cache = _ptr(kv_cache)
+    a.block_table, a.seq_lens = _ptr(block_table), _ptr(seq_lens)
+    a.out, a.lse = _ptr(out), _ptr(lse)
+    a.B, a.s_q, a.H = B, s_q, H
+    a.d_c, a.d_r, a.page_size = D_C, D_R, PAGE
+    a.num_pages = P
+    a.max_pages_per_seq = block_table.shape[1]
+    a.kv_dtype = KV_BF16
+    a.causal = int(bool(causal))
+    a.max_seq_len = int(max_seq_len)
+    a.softmax_scale = float(softmax_scale)
+    if workspace is not None:
+        a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    return a
+
+
+def mla_prefill_workspace_size(args: PrefillArgs) -> int:
+    n = ctypes.c_size_t(0)
+    _check("mla_prefill_workspace_size", load().mla_prefill_workspace_size(ctypes.byref(args), ctypes.byref(n)))
+    return int(n.value)
+
+
+def mla_prefill(args: PrefillArgs, stream=None):
+    """Explicit-form attention of the s_q new tokens of every sequence (per-head
+    keys and values formed in the workspace, then a FlashAttention forward)."""
+    _check("mla_prefill", load().mla_prefill(ctypes.byref(args), _stream(stream)))
+
+
 def mla_get_status(workspace, stream=None) -> int:
     """Waits for the stream and returns (and clears) the device status word."""
     return int(load().mla_get_status(_ptr(workspace), _stream(stream)))
@@ -346,10 +420,15 @@ def mla_status_string(code: int) -> str:
 
 
 def alloc_workspace(args, device="cuda"):
-    """A zeroed workspace tensor sized for ``args`` (``DecodeArgs`` or
-    ``WriteKvArgs``); also stored into ``args``."""
+    """A zeroed workspace tensor sized for ``args`` (``DecodeArgs``,
+    ``WriteKvArgs`` or ``PrefillArgs``); also stored into ``args``."""
     import torch
-    n = mla_write_kv_workspace_size(args) if isinstance(args, WriteKvArgs) else mla_decode_workspace_size(args)
+    if isinstance(args, WriteKvArgs):
+        n = mla_write_kv_workspace_size(args)
+    elif isinstance(args, PrefillArgs):
+        n = mla_prefill_workspace_size(args)
+    else:
+        n = mla_decode_workspace_size(args)
     ws = torch.zeros(n, dtype=torch.uint8, device=device)
     args.workspace, args.workspace_bytes = _ptr(ws), n
     return ws

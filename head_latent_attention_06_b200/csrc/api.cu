@@ -21,6 +21,8 @@ int decode_mma_tiles(int len);
 int decode_mma_ctas_per_split(int s_q, int H, int B);
 int write_kv_k_split(int n_tok, int d_h);
 cudaError_t launch_write_kv(const mla_write_kv_args_t*, cudaStream_t);
+size_t prefill_workspace_bytes(int B, int H, int Lmax);
+cudaError_t launch_prefill(const mla_prefill_args_t*, cudaStream_t);
 }  // namespace mla
 
 using namespace mla;
@@ -117,6 +119,22 @@ mla_status_t check_write_kv_shape(const mla_write_kv_args_t* a) {
   if (a->kv_dtype != MLA_KV_BF16 && a->kv_dtype != MLA_KV_FP8_E4M3 && a->kv_dtype != MLA_KV_Q8_0)
     return MLA_ERR_UNSUPPORTED;
   if (!(a->rope_base > 0.f) || !isfinite(a->rope_base)) return MLA_ERR_INVALID_VALUE;
+  return MLA_OK;
+}
+
+mla_status_t check_prefill_shape(const mla_prefill_args_t* a) {
+  if (!a) return MLA_ERR_INVALID_VALUE;
+  if (a->B < 0 || a->H <= 0 || a->s_q <= 0 || a->num_pages < 0 || a->max_pages_per_seq <= 0)
+    return MLA_ERR_INVALID_VALUE;
+  if (a->d_c != kDc || a->d_r != kDr || a->page_size != kPage) return MLA_ERR_UNSUPPORTED;
+  if (a->H > 128 || a->B > 65535 || a->kv_dtype != MLA_KV_BF16) return MLA_ERR_UNSUPPORTED;
+  if (a->max_seq_len < a->s_q) return MLA_ERR_INVALID_VALUE;
+  // TMA coordinates are 32-bit: rows of the per-head key / value arrays and
+  // query tokens must stay below 2^31
+  const int64_t lpad = ((int64_t)a->max_seq_len + 127) / 128 * 128;
+  if ((int64_t)a->B * a->H * lpad >= (int64_t)1 << 31 || (int64_t)a->B * a->s_q >= (int64_t)1 << 31)
+    return MLA_ERR_UNSUPPORTED;
+  if (!(a->softmax_scale == a->softmax_scale)) return MLA_ERR_INVALID_VALUE;
   return MLA_OK;
 }
 
@@ -228,6 +246,34 @@ mla_status_t mla_write_kv(const mla_write_kv_args_t* a, void* stream) {
       (reinterpret_cast<uintptr_t>(a->kv_scale) & 3u))
     return MLA_ERR_MISALIGNED;
   return from_cuda(launch_write_kv(a, (cudaStream_t)stream));
+}
+
+mla_status_t mla_prefill_workspace_size(const mla_prefill_args_t* a, size_t* bytes) {
+  mla_status_t st = check_prefill_shape(a);
+  if (st != MLA_OK) return st;
+  if (!bytes) return MLA_ERR_INVALID_VALUE;
+  *bytes = prefill_workspace_bytes(a->B, a->H, a->max_seq_len);
+  return MLA_OK;
+}
+
+mla_status_t mla_prefill(const mla_prefill_args_t* a, void* stream) {
+  mla_status_t st = check_prefill_shape(a);
+  if (st != MLA_OK) return st;
+  if (!a->workspace) return MLA_ERR_INVALID_VALUE;
+  if (!aligned16(a->workspace)) return MLA_ERR_MISALIGNED;
+  if (a->workspace_bytes < prefill_workspace_bytes(a->B, a->H, a->max_seq_len)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (a->B == 0) return MLA_OK;
+  if (!a->q_nope || !a->q_pe || !a->w_uk || !a->w_uv || !a->kv_cache || !a->block_table || !a->seq_lens ||
+      !a->out)
+    return MLA_ERR_INVALID_VALUE;
+  if (a->num_pages <= 0) return MLA_ERR_INVALID_VALUE;
+  if (!aligned16(a->q_nope) || !aligned16(a->q_pe) || !aligned16(a->w_uk) || !aligned16(a->w_uv) ||
+      !aligned16(a->kv_cache) || !aligned16(a->out))
+    return MLA_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(a->block_table) & 3u) || (reinterpret_cast<uintptr_t>(a->seq_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(a->lse) & 3u))
+    return MLA_ERR_MISALIGNED;
+  return from_cuda(launch_prefill(a, (cudaStream_t)stream));
 }
 
 mla_status_t mla_get_status(void* workspace, void* stream) {

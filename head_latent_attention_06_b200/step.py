@@ -1,16 +1,19 @@
-"""One MLA decode step through the C ABI: absorb -> paged decode -> combine -> up-project.
+"""One MLA attention step through the C ABI.
 
-``DecodeStep`` owns the intermediate device buffers (q_lat, o_lat, lse, out and
-the workspace) and replays the four calls on the current stream.  It does no
-arithmetic of its own.
+``DecodeStep``: absorb -> paged decode -> combine -> up-project (the absorbed
+form); it owns the intermediate device buffers (q_lat, o_lat, lse, out and the
+workspace) and replays the four calls on the current stream.  ``PrefillStep``:
+the explicit form for long chunks of new tokens (one call, two kernels).
+Neither does arithmetic of its own.
 """
 
 from __future__ import annotations
 
 import torch
 
-from . import (D_C, D_N, D_V, alloc_workspace, make_decode_args, mla_absorb_q,
-               mla_combine_splits, mla_decode_num_splits, mla_decode_paged, mla_up_proj_v)
+from . import (D_C, D_N, D_V, alloc_workspace, make_decode_args, make_prefill_args, mla_absorb_q,
+               mla_combine_splits, mla_decode_num_splits, mla_decode_paged, mla_prefill,
+               mla_up_proj_v)
 
 
 class DecodeStep:
@@ -76,3 +79,38 @@ def step_from_workload(w, device="cuda", num_splits=0):
                       block_table=d(w.block_table), seq_lens=d(w.seq_lens), causal=w.causal,
                       softmax_scale=w.softmax_scale, num_splits=num_splits,
                       max_seq_len=max(w.lens) if w.lens else 0)
+
+
+class PrefillStep:
+    """Explicit-form attention of s_q new tokens per sequence over the paged bf16
+    cache: owns out, lse and the workspace (the per-head keys and values)."""
+
+    def __init__(self, *, q_nope, q_pe, w_uk, w_uv, kv_cache, block_table, seq_lens, causal,
+                 softmax_scale, max_seq_len, out=None):
+        B, s_q, H, _ = q_nope.shape
+        dev = q_nope.device
+        self.B, self.s_q, self.H = B, s_q, H
+        self.lse = torch.empty(B, s_q, H, dtype=torch.float32, device=dev)
+        self.out = out if out is not None else torch.empty(B, s_q, H, D_V, dtype=torch.bfloat16,
+                                                           device=dev)
+        self.args = make_prefill_args(q_nope=q_nope, q_pe=q_pe, w_uk=w_uk, w_uv=w_uv,
+                                      kv_cache=kv_cache, block_table=block_table,
+                                      seq_lens=seq_lens, out=self.out, lse=self.lse,
+                                      max_seq_len=max_seq_len, causal=causal,
+                                      softmax_scale=softmax_scale)
+        self.workspace = alloc_workspace(self.args, device=dev)
+        self._keep = (q_nope, q_pe, w_uk, w_uv, kv_cache, block_table, seq_lens)
+
+    def run(self, stream=None):
+        mla_prefill(self.args, stream)
+        return self.out
+
+
+def prefill_from_workload(w, device="cuda", max_seq_len=None):
+    """Copy a bf16-cache ``mla_inputs.Workload`` to the device and build its
+    ``PrefillStep``."""
+    d = lambda t: t.to(device, non_blocking=False).contiguous()
+    return PrefillStep(q_nope=d(w.q_nope), q_pe=d(w.q_pe), w_uk=d(w.w_uk), w_uv=d(w.w_uv),
+                       kv_cache=d(w.kv_cache), block_table=d(w.block_table),
+                       seq_lens=d(w.seq_lens), causal=w.causal, softmax_scale=w.softmax_scale,
+                       max_seq_len=max_seq_len or max(max(w.lens), w.spec.s_q))

@@ -263,6 +263,60 @@ mla_status_t mla_write_kv_workspace_size(const mla_write_kv_args_t* args, size_t
  */
 mla_status_t mla_write_kv(const mla_write_kv_args_t* args, void* stream);
 
+/*
+ * Arguments of mla_prefill / mla_prefill_workspace_size.
+ * Zero-initialise the struct, then fill every field.
+ */
+typedef struct {
+  const void* q_nope;             /* bf16 [B][s_q][H][d_n] */
+  const void* q_pe;               /* bf16 [B][s_q][H][d_r], RoPE already applied */
+  const void* w_uk;               /* bf16 [H][d_n][d_c] (k = W_UK[h] c) */
+  const void* w_uv;               /* bf16 [H][d_v][d_c] (v = W_UV[h] c) */
+  const void* kv_cache;           /* bf16 [num_pages][page_size][d_c + d_r]: row = c || k_pe */
+  const int32_t* block_table;     /* int32 [B][max_pages_per_seq] */
+  const int32_t* seq_lens;        /* int32 [B], device: cached tokens including the s_q new ones */
+  void* out;                      /* bf16 [B][s_q][H][d_v], written */
+  float* lse;                     /* fp32 [B][s_q][H], natural log, written; may be NULL */
+  void* workspace;                /* device scratch, >= mla_prefill_workspace_size() bytes,
+                                     16-byte aligned; its first 16 bytes must be zero before the
+                                     first use (they hold the sticky status word) */
+  size_t workspace_bytes;
+  int32_t B, s_q, H;
+  int32_t d_c, d_r, page_size;
+  int32_t num_pages;              /* physical pages in kv_cache */
+  int32_t max_pages_per_seq;      /* row length of block_table */
+  int32_t kv_dtype;               /* MLA_KV_BF16 only */
+  int32_t causal;                 /* 1: query i of sequence b sees tokens 0 .. L_b - s_q + i */
+  int32_t max_seq_len;            /* host-known upper bound of seq_lens, >= s_q (sizes the
+                                     workspace; a longer sequence is MLA_ERR_BAD_SEQ_LEN) */
+  float softmax_scale;
+} mla_prefill_args_t;
+
+/* Bytes of workspace mla_prefill needs (host only): 256 plus the per-head keys
+ * and values of every sequence, 2 * B * H * roundup(max_seq_len, 128) * 128 bf16. */
+mla_status_t mla_prefill_workspace_size(const mla_prefill_args_t* args, size_t* bytes);
+
+/*
+ * mla_prefill — attention of many new tokens per sequence in the explicit form
+ * ("MLA: Multi-Head Latent Attention — DeepSeek-AI Explained", section
+ * "Architecture": k = [W_UK c ; k_pe], v = W_UV c per head).  Prefill is bound
+ * by compute, not by the cache (snowgate thread 35, the reply on prefill), and
+ * beyond about 170 queries per sequence forming K and V once costs fewer FLOPs
+ * than the absorbed form's 576 + 512 products per query and token.  Two kernels:
+ * the per-head keys and values of every cached token (bf16, into the
+ * workspace), then a FlashAttention forward with an online softmax over them.
+ * For query i of sequence b, head h and visible token j:
+ *   s_j = softmax_scale * ([q_nope ; q_pe] . [W_UK[h] c_j ; k_pe_j])
+ *   out = sum_j softmax(s)_j W_UV[h] c_j ,   lse = log sum_j exp(s_j)
+ * The result equals mla_absorb_q + mla_decode_paged + mla_combine_splits +
+ * mla_up_proj_v up to rounding (K and V are rounded to bf16 here, q_lat and
+ * o_lat there).  H 1 .. 128, 1 <= s_q <= max_seq_len, bf16 cache only.  A
+ * length below s_q or above max_seq_len or the block table (MLA_ERR_BAD_SEQ_LEN;
+ * that sequence's outputs are zero, lse -inf) or a page id outside the cache
+ * (MLA_ERR_BAD_BLOCK_TABLE) goes to the workspace's status word.
+ */
+mla_status_t mla_prefill(const mla_prefill_args_t* args, void* stream);
+
 /* Waits for `stream`, returns the sticky device status word of `workspace`
  * (MLA_OK if no device-side problem was recorded) and clears it. */
 mla_status_t mla_get_status(void* workspace, void* stream);

@@ -81,6 +81,9 @@ PRESETS = {
                         note="batch 128, 128 heads, 8192 tokens, e4m3 cache + fp32 per-token "
                              "scale, 2 causal query tokens"),
     # the V3 shape over the blockwise q8_0 cache (ik_llama.cpp's recommended MLA cache type)
+    "prefill": WorkloadSpec("prefill", B=4, H=128, s_q=1024, lens=[8192] * 4, causal=True, seed=6,
+                            note="chunked prefill: batch 4, 128 heads, 1024 new tokens appended "
+                                 "to 7168 cached (8192 in all), causal, bf16 paged"),
     "q8": WorkloadSpec("q8", B=64, H=128, s_q=1, lens=[4096] * 64, kv_dtype="q8_0", seed=5,
                        note="DeepSeek-V3-shaped: batch 64, 128 heads, 4096 tokens, q8_0 cache "
                             "(int8 codes, fp16 scale per 32 values)"),

@@ -203,3 +203,69 @@ def test_write_kv_with_empty_batch_enqueues_nothing(lib):
     a = _wargs(B=0)
     a.workspace, a.workspace_bytes = 0x20000, 256
     assert lib.mla_write_kv(ctypes.byref(a), None) == OK
+
+
+# ---------------------------------------------------------------- prefill
+
+def _pargs(B=4, s_q=1024, H=128, max_len=8192, **kw):
+    a = mla.PrefillArgs()
+    fake = 0x10000
+    for f in ("q_nope", "q_pe", "w_uk", "w_uv", "kv_cache", "block_table", "seq_lens", "out", "lse"):
+        setattr(a, f, fake)
+    a.B, a.s_q, a.H = B, s_q, H
+    a.d_c, a.d_r, a.page_size = 512, 64, 64
+    a.num_pages, a.max_pages_per_seq = 512, 128
+    a.kv_dtype, a.causal, a.max_seq_len = 0, 1, max_len
+    a.softmax_scale = 0.0722
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_prefill_workspace_holds_keys_and_values(lib):
+    # per-head keys and values (128 bf16 each) of every sequence, rows padded to 128
+    assert mla.mla_prefill_workspace_size(_pargs()) == 256 + 2 * 4 * 128 * 8192 * 256
+    assert mla.mla_prefill_workspace_size(_pargs(B=1, H=1, s_q=1, max_len=1)) == 256 + 2 * 128 * 256
+    assert mla.mla_prefill_workspace_size(_pargs(B=2, H=16, s_q=100, max_len=129)) == 256 + 2 * 32 * 256 * 256
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("d_c", 256, UNSUPPORTED), ("d_r", 32, UNSUPPORTED), ("page_size", 32, UNSUPPORTED),
+    ("kv_dtype", 1, UNSUPPORTED), ("kv_dtype", 2, UNSUPPORTED), ("H", 129, UNSUPPORTED),
+    ("H", 0, INVALID), ("s_q", 0, INVALID), ("B", -1, INVALID), ("max_pages_per_seq", 0, INVALID),
+    ("max_seq_len", 1023, INVALID), ("softmax_scale", float("nan"), INVALID),
+    ("max_seq_len", 1 << 30, UNSUPPORTED), ("B", 65536, UNSUPPORTED),
+])
+def test_prefill_rejects_bad_shapes(lib, field, value, code):
+    a = _pargs(**{field: value})
+    a.workspace, a.workspace_bytes = 0x20000, 1 << 40
+    assert lib.mla_prefill(ctypes.byref(a), None) == code
+    n = ctypes.c_size_t(0)
+    assert lib.mla_prefill_workspace_size(ctypes.byref(a), ctypes.byref(n)) == code
+
+
+def test_prefill_rejects_bad_pointers_and_workspace(lib):
+    a = _pargs()
+    assert lib.mla_prefill(ctypes.byref(a), None) == INVALID                # no workspace
+    a.workspace, a.workspace_bytes = 0x20008, 1 << 40
+    assert lib.mla_prefill(ctypes.byref(a), None) == MISALIGNED
+    a.workspace, a.workspace_bytes = 0x20000, 256
+    assert lib.mla_prefill(ctypes.byref(a), None) == WS_SMALL
+    a.workspace_bytes = 1 << 40
+    for f in ("q_nope", "w_uv", "out"):
+        setattr(a, f, None)
+        assert lib.mla_prefill(ctypes.byref(a), None) == INVALID, f
+        setattr(a, f, 0x10008)
+        assert lib.mla_prefill(ctypes.byref(a), None) == MISALIGNED, f
+        setattr(a, f, 0x10000)
+    a.lse = 0x10002
+    assert lib.mla_prefill(ctypes.byref(a), None) == MISALIGNED
+    a.lse = None                                                            # lse is optional
+    a.num_pages = 0
+    assert lib.mla_prefill(ctypes.byref(a), None) == INVALID
+
+
+def test_prefill_with_empty_batch_enqueues_nothing(lib):
+    a = _pargs(B=0)
+    a.workspace, a.workspace_bytes = 0x20000, 256
+    assert lib.mla_prefill(ctypes.byref(a), None) == OK
