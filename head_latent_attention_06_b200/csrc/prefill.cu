@@ -149,6 +149,7 @@ __global__ void __launch_bounds__(kUpThreads, 1)
   // the attention multiplies them by zero weights, which must not meet a NaN.
   int keep = 0;
   mbar_wait(done, 0, &keep, nullptr, kDrainNs);
+  __syncwarp();  // the tensor-memory loads below are warp-collective
   tc_fence_after();
   const int t = t0 + 32 * warp + lane;
   const bool ok = __shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(abort_flag), 0) == 0 && t < L;
@@ -194,14 +195,16 @@ constexpr uint32_t kAtVOff = kAtKOff + kKvStages * kKBytes;
 constexpr uint32_t kAtBarOff = kAtVOff + kKvStages * kVBytes;
 constexpr uint32_t kAtSmem = kAtBarOff + 256 + 1024;
 static_assert(kAtSmem <= 232448, "shared memory budget");
-// TMEM: S / P buffers at columns 0 and 128 (P, bf16, takes the first 64 of them), O at 256
-constexpr uint32_t kTmemO = 256;
+// TMEM: three S / P buffers at columns 0, 128 and 256 (P, bf16, takes the first
+// 64 columns of its buffer), O at 384
+constexpr int kSBufs = 3;
+constexpr uint32_t kTmemO = 384;
 constexpr uint32_t kAtIdescS = idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t kAtIdescPV = idesc_bf16_f32(128, 128, false, true);
 constexpr float kRescale = 8.0f;
 // barriers
-constexpr int A_Q = 0, A_KFULL = 1, A_KEMPTY = 3, A_VFULL = 5, A_VEMPTY = 7, A_SREADY = 9, A_PREADY = 11,
-              A_ODONE = 13, A_DRAIN = 15, A_NBARS = 16;
+constexpr int A_Q = 0, A_KFULL = 1, A_KEMPTY = 3, A_VFULL = 5, A_VEMPTY = 7, A_SREADY = 9, A_PREADY = 12,
+              A_ODONE = 15, A_DRAIN = 18, A_NBARS = 19;
 
 struct AtParams {
   const __nv_bfloat16* kn;
@@ -253,6 +256,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       mbar_init(bar(A_KEMPTY + i), 1);
       mbar_init(bar(A_VFULL + i), 1);
       mbar_init(bar(A_VEMPTY + i), 1);
+    }
+    for (int i = 0; i < kSBufs; ++i) {
       mbar_init(bar(A_SREADY + i), 1);
       mbar_init(bar(A_PREADY + i), 4);
       mbar_init(bar(A_ODONE + i), 1);
@@ -325,8 +330,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     if (n > 0 && nq > 0) {
       const uint64_t dq = desc_sw128(sa + kAtQOff, 16, 1024);
       bool ok = mbar_wait_converged(bar(A_Q), 0, abort_flag, p.status, wait_ns);
+      // S(j) = Q K(j)^T into S buffer j % 3
       auto issue_s = [&](int j) -> bool {
-        const int st = j & 1;
+        const int st = j & 1, sb = j % kSBufs;
         if (!mbar_wait_converged(bar(A_KFULL + st), (j >> 1) & 1, abort_flag, p.status, wait_ns)) return false;
         tc_fence_after();
         const uint64_t dk = desc_sw128(sa + kAtKOff + st * kKBytes, 16, 1024);
@@ -334,31 +340,33 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         for (int c = 0; c < 3; ++c)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_1_elect(tmem + 128u * st, dq + ((c * kQChunk) >> 4) + 2 * kk, dk + ((c * kQChunk) >> 4) + 2 * kk,
+            mma_1_elect(tmem + 128u * sb, dq + ((c * kQChunk) >> 4) + 2 * kk, dk + ((c * kQChunk) >> 4) + 2 * kk,
                         kAtIdescS, (c | kk) != 0);
         commit_1_elect(bar(A_KEMPTY + st));
-        commit_1_elect(bar(A_SREADY + st));
+        commit_1_elect(bar(A_SREADY + sb));
         return true;
       };
       if (ok) ok = issue_s(0);
       if (ok && n > 1) ok = issue_s(1);
       for (int j = 0; ok && j < n; ++j) {
-        const int st = j & 1;
+        const int st = j & 1, sb = j % kSBufs, ph = (j / kSBufs) & 1;
         // P(j) written over S(j) in TMEM by the softmax threads
-        if (!mbar_wait_converged(bar(A_PREADY + st), (j >> 1) & 1, abort_flag, p.status, wait_ns)) break;
+        if (!mbar_wait_converged(bar(A_PREADY + sb), ph, abort_flag, p.status, wait_ns)) break;
         if (!mbar_wait_converged(bar(A_VFULL + st), (j >> 1) & 1, abort_flag, p.status, wait_ns)) break;
         tc_fence_after();
         const uint64_t dv = desc_sw128(sa + kAtVOff + st * kVBytes, kQChunk, 1024);
         // K = 128 keys in steps of 16: P columns 8 kk (2 bf16 each), V rows 16 kk
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_1_ts_elect(tmem + kTmemO, tmem + 128u * st + 8u * kk, dv + ((kk * 2048) >> 4), kAtIdescPV,
+          mma_1_ts_elect(tmem + kTmemO, tmem + 128u * sb + 8u * kk, dv + ((kk * 2048) >> 4), kAtIdescPV,
                          (j > 0 || kk > 0) ? 1u : 0u);
         commit_1_elect(bar(A_VEMPTY + st));
-        commit_1_elect(bar(A_ODONE + st));
-        // S(j + 2) goes where P(j) is: only once P.V(j) has read it
+        commit_1_elect(bar(A_ODONE + sb));
+        // S(j + 2) goes where P(j - 1) was: only once P.V(j - 1) has read it
         if (j + 2 < n) {
-          if (!mbar_wait_converged(bar(A_ODONE + st), (j >> 1) & 1, abort_flag, p.status, wait_ns)) break;
+          if (j >= 1 && !mbar_wait_converged(bar(A_ODONE + (j - 1) % kSBufs), ((j - 1) / kSBufs) & 1, abort_flag,
+                                             p.status, wait_ns))
+            break;
           if (!issue_s(j + 2)) break;
         }
       }
@@ -374,14 +382,14 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     const int vis = p.causal ? L - p.s_q + qi + 1 : L;  // keys this query sees
     float m_used = -CUDART_INF_F, l = 0.f;
     for (int j = 0; j < n && nq > 0; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait_converged(bar(A_SREADY + st), (j >> 1) & 1, abort_flag, p.status, wait_ns)) break;
+      const int sb = j % kSBufs;
+      if (!mbar_wait_converged(bar(A_SREADY + sb), (j / kSBufs) & 1, abort_flag, p.status, wait_ns)) break;
       tc_fence_after();
       float s[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
-        tmem_ld32(tl + 128u * st + 32u * c, r);
+        tmem_ld32(tl + 128u * sb + 32u * c, r);
         tmem_wait_ld();
 #pragma unroll
         for (int k = 0; k < 32; ++k) s[32 * c + k] = __uint_as_float(r[k]);
@@ -408,7 +416,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       const float nref = m_used == -CUDART_INF_F ? 0.f : -m_used;
       // O of this row may be rescaled only once P.V(j-1) has accumulated into it
       if (__any_sync(0xffffffffu, resc) && j >= 1) {
-        if (!mbar_wait_converged(bar(A_ODONE + (st ^ 1)), ((j - 1) >> 1) & 1, abort_flag, p.status, wait_ns))
+        if (!mbar_wait_converged(bar(A_ODONE + (j - 1) % kSBufs), ((j - 1) / kSBufs) & 1, abort_flag, p.status,
+                                 wait_ns))
           break;
         tc_fence_after();
 #pragma unroll 1
@@ -432,34 +441,38 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           l += p0 + p1;
           pk[k] = pack_bf16(p0, p1);
         }
-        tmem_st32(tl + 128u * st + 32u * c, pk);
+        tmem_st32(tl + 128u * sb + 32u * c, pk);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_local(bar(A_PREADY + st));
+      if (lane == 0) mbar_arrive_local(bar(A_PREADY + sb));
     }
     // ---- epilogue: o = O / l, lse
     if (n > 0 && nq > 0) {
-      mbar_wait_converged(bar(A_ODONE + ((n - 1) & 1)), ((n - 1) >> 1) & 1, abort_flag, p.status, wait_ns);
+      mbar_wait_converged(bar(A_ODONE + (n - 1) % kSBufs), ((n - 1) / kSBufs) & 1, abort_flag, p.status, wait_ns);
       tc_fence_after();
     }
     const bool alive = __shfl_sync(0xffffffffu, *abort_flag, 0) == 0;
     const bool empty = !(l > 0.f) || !alive;
     const float inv = empty ? 0.f : 1.f / l;
-    if (qi < p.s_q && nq > 0) {
-      const size_t orow = ((size_t)b * p.s_q + qi) * p.H + h;
-      __nv_bfloat16* dst = p.out + orow * kDv;
+    // tcgen05.ld is a warp-collective instruction: every lane loads (the
+    // condition is warp-uniform), only the rows of real queries are stored
+    const bool live = n > 0 && nq > 0 && alive;
+    const bool mine = qi < p.s_q && nq > 0;
+    const size_t orow = ((size_t)b * p.s_q + qi) * p.H + h;
+    __nv_bfloat16* dst = p.out + orow * kDv;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        if (n > 0 && alive) {
-          tmem_ld32(tl + kTmemO + 32u * c, o);
-          tmem_wait_ld();
-        } else {
+    for (int c = 0; c < 4; ++c) {
+      uint32_t o[32];
+      if (live) {
+        tmem_ld32(tl + kTmemO + 32u * c, o);
+        tmem_wait_ld();
+      } else {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = 0u;
-        }
+        for (int k = 0; k < 32; ++k) o[k] = 0u;
+      }
+      if (mine) {
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           reinterpret_cast<uint4*>(dst + 32 * c)[k] =
@@ -468,8 +481,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                          pack_bf16(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv),
                          pack_bf16(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv));
       }
-      if (p.lse) p.lse[orow] = empty ? -CUDART_INF_F : (m_used + log2f(l)) * 0.6931471805599453f;
     }
+    if (mine && p.lse) p.lse[orow] = empty ? -CUDART_INF_F : (m_used + log2f(l)) * 0.6931471805599453f;
     tc_fence_before();
   }
 
