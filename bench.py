@@ -41,7 +41,16 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # workload, recorded with the kernel's source file and the sha256 prefix of that
 # file and the device headers it includes, as they were when the capture was
 # taken: reported as the roofline's ``traffic`` only while they are unchanged.
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    # ncu --set full, one launch of the V3 workload (profiles/decode_tc_v3_bf16.md)
+    "v3": (315_607_808, "decode_tc.cu", "a600c572d632e248"),
+    # one launch of the fp8 workload (profiles/decode_f8_fp8.md)
+    "fp8": (773_860_864, "decode_f8.cu", "46f792446c3adafd"),
+    # both prefill kernels on one sequence of the chunked-prefill workload
+    # (profiles/prefill_chunk_bf16.md): 1,155,835,392 bytes, times the 4 sequences
+    # of the full workload (traffic grows with the sequences processed)
+    "prefill": (4 * 1_155_835_392, "prefill.cu", "d9eeb2f7c6032754"),
+}
 KERNEL_HEADERS = ("sm100.cuh", "common.cuh", "tma_host.cuh")
 
 
@@ -472,7 +481,7 @@ def run_prefill(args):
             "flops_per_step": flops, "kv_up_flops_per_step": up_flops,
             "absorbed_form_ms": None if absorbed_ms is None else round(absorbed_ms, 4),
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tc_peak, "unit": "TFLOP/s",
-                         "frac": round(tflops / tc_peak, 4), "traffic": None,
+                         "frac": round(tflops / tc_peak, 4), "traffic": decode_traffic(args.config),
                          "peak_kind": f"{peak_kind}: {tc_kind}",
                          "kernel": "mla_prefill (kv_up_kernel + prefill_attn_kernel, one call)"},
             "e2e": {"value": round(flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",

@@ -84,6 +84,9 @@ PRESETS = {
     "prefill": WorkloadSpec("prefill", B=4, H=128, s_q=1024, lens=[8192] * 4, causal=True, seed=6,
                             note="chunked prefill: batch 4, 128 heads, 1024 new tokens appended "
                                  "to 7168 cached (8192 in all), causal, bf16 paged"),
+    "prefill1": WorkloadSpec("prefill1", B=1, H=128, s_q=1024, lens=[8192], causal=True, seed=6,
+                             note="one sequence of the chunked-prefill workload (for profiler "
+                                  "captures): 128 heads, 1024 new tokens on 7168 cached, causal"),
     "q8": WorkloadSpec("q8", B=64, H=128, s_q=1, lens=[4096] * 64, kv_dtype="q8_0", seed=5,
                        note="DeepSeek-V3-shaped: batch 64, 128 heads, 4096 tokens, q8_0 cache "
                             "(int8 codes, fp16 scale per 32 values)"),
