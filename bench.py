@@ -42,12 +42,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # file and the device headers it includes, as they were when the capture was
 # taken: reported as the roofline's ``traffic`` only while they are unchanged.
 MEASURED_TRAFFIC = {
-    # ncu --set full, one launch of the V3 workload (profiles/decode_tc_v3_bf16.md)
+    # ncu --set full, one launch of the V3 workload
     "v3": (315_607_808, "decode_tc.cu", "a600c572d632e248"),
-    # one launch of the fp8 workload (profiles/decode_f8_fp8.md)
+    # one launch of the fp8 workload
     "fp8": (773_860_864, "decode_f8.cu", "46f792446c3adafd"),
-    # both prefill kernels on one sequence of the chunked-prefill workload
-    # (profiles/prefill_chunk_bf16.md): 1,155,835,392 bytes, times the 4 sequences
+    # both prefill kernels on one sequence of the chunked-prefill workload:
+    # 1,155,835,392 bytes, times the 4 sequences
     # of the full workload (traffic grows with the sequences processed)
     "prefill": (4 * 1_155_835_392, "prefill.cu", "d9eeb2f7c6032754"),
 }
