@@ -131,7 +131,7 @@ mla_status_t check_prefill_shape(const mla_prefill_args_t* a) {
   if (a->max_seq_len < a->s_q) return MLA_ERR_INVALID_VALUE;
   // TMA coordinates are 32-bit: rows of the per-head key / value arrays and
   // query tokens must stay below 2^31
-  const int64_t lpad = ((int64_t)a->max_seq_len + 127) / 128 * 128;
+  const int64_t lpad = ((int64_t)a->max_seq_len + 255) / 256 * 256;
   if ((int64_t)a->B * a->H * lpad >= (int64_t)1 << 31 || (int64_t)a->B * a->s_q >= (int64_t)1 << 31)
     return MLA_ERR_UNSUPPORTED;
   if (!(a->softmax_scale == a->softmax_scale)) return MLA_ERR_INVALID_VALUE;

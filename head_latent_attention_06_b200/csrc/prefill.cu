@@ -13,9 +13,12 @@
 //
 // Two kernels:
 //   kv_up:   Kn[b][h][t] = W_UK[h] c_t and V[b][h][t] = W_UV[h] c_t (bf16, 128 each)
-//            for every cached token t of every sequence: a GEMM with M = 128 tokens
-//            (two pages, TMA from the paged cache), N = 256 (the head's W_UK and
-//            W_UV rows), K = 512 in chunks of 64, accumulated in TMEM.
+//            for every cached token t of every sequence: per CTA two GEMMs with
+//            M = 128 tokens (two pages each, TMA from the paged cache), sharing
+//            the B operand N = 256 (the head's W_UK and W_UV rows), K = 512 in
+//            chunks of 64, accumulated in two TMEM accumulators (256 columns
+//            each).  Sharing the weight chunk between 256 tokens cuts the
+//            operand bytes per MMA by a third against one 128-token tile.
 //   attn:    FlashAttention forward per (sequence, head, 128 queries): S = Q K^T
 //            with Q = [q_nope | q_pe] (192), K = [Kn | k_pe] (k_pe from the cache,
 //            shared by all heads), M = 128 queries, N = 128 keys; online softmax
@@ -43,9 +46,10 @@ constexpr uint64_t kDrainNs = 100000000ull;
 // ---------------------------------------------------------------- kv_up
 constexpr int kUpThreads = 128;
 constexpr int kUpStages = 3;
-constexpr uint32_t kUpA = 128 * 128;         // 128 tokens x 64 latent values (bf16)
+constexpr int kUpTok = 256;                  // tokens per CTA: two M = 128 tiles
+constexpr uint32_t kUpA = 128 * 128;         // one tile: 128 tokens x 64 latent values (bf16)
 constexpr uint32_t kUpB = 256 * 128;         // 256 weight rows x 64 values
-constexpr uint32_t kUpStage = kUpA + kUpB;   // 48 KB
+constexpr uint32_t kUpStage = 2 * kUpA + kUpB;  // 64 KB
 constexpr uint32_t kUpBarOff = kUpStages * kUpStage;
 constexpr uint32_t kUpSmem = kUpBarOff + 128 + 1024;
 constexpr uint32_t kUpIdesc = idesc_bf16_f32(128, 256, false, false);
@@ -53,7 +57,7 @@ constexpr uint32_t kUpIdesc = idesc_bf16_f32(128, 256, false, false);
 struct UpParams {
   const int32_t* block_table;
   const int32_t* seq_lens;
-  __nv_bfloat16* kn;   // [B][H][Lmax][128]
+  __nv_bfloat16* kn;   // [B][H][Lmax][128], Lmax a multiple of 256
   __nv_bfloat16* v;    // [B][H][Lmax][128]
   uint32_t* status;
   int H, max_pages, num_pages, Lmax, max_len;
@@ -77,7 +81,7 @@ __global__ void __launch_bounds__(kUpThreads, 1)
   pdl_wait();  // whatever wrote the cache, the block table or the lengths
   int L = p.seq_lens[b];
   if (L < 0 || L > p.max_pages * kPage || L > p.max_len) L = 0;  // reported by the attention kernel
-  const int t0 = tile * 128;
+  const int t0 = tile * kUpTok;
   if (t0 >= L) return;  // whole CTA: nothing of this sequence here
   if (threadIdx.x == 0) {
     for (int s = 0; s < kUpStages; ++s) {
@@ -89,15 +93,17 @@ __global__ void __launch_bounds__(kUpThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc_1(smem_u32(tmem_slot), 256);
+    tmem_alloc_1(smem_u32(tmem_slot), 512);
     tmem_relinquish_1();
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int32_t* bt = p.block_table + (size_t)b * p.max_pages;
-  int pg[2];
-  for (int k = 0; k < 2; ++k) {
+  // the four pages of the 256 tokens; pages past the length stand in with the
+  // first one (their rows are written as zeros)
+  int pg[4];
+  for (int k = 0; k < 4; ++k) {
     const int idx = t0 / kPage + k;
     int v = idx * kPage < L ? bt[idx] : bt[t0 / kPage];
     if (v < 0 || v >= p.num_pages) {
@@ -116,10 +122,9 @@ __global__ void __launch_bounds__(kUpThreads, 1)
       if (lane == 0) {
         const uint32_t dst = sa + s * kUpStage;
         mbar_arrive_expect_tx_local(full0 + 8 * s, kUpStage);
-        tma_load_2d_cta(dst, &tm_c, full0 + 8 * s, 64 * c, pg[0] * kPage);
-        tma_load_2d_cta(dst + 64 * 128, &tm_c, full0 + 8 * s, 64 * c, pg[1] * kPage);
-        tma_load_2d_cta(dst + kUpA, &tm_wuk, full0 + 8 * s, 64 * c, h * 128);
-        tma_load_2d_cta(dst + kUpA + 128 * 128, &tm_wuv, full0 + 8 * s, 64 * c, h * 128);
+        for (int k = 0; k < 4; ++k) tma_load_2d_cta(dst + k * 64 * 128, &tm_c, full0 + 8 * s, 64 * c, pg[k] * kPage);
+        tma_load_2d_cta(dst + 2 * kUpA, &tm_wuk, full0 + 8 * s, 64 * c, h * 128);
+        tma_load_2d_cta(dst + 2 * kUpA + 128 * 128, &tm_wuv, full0 + 8 * s, 64 * c, h * 128);
       }
       __syncwarp();
       issued = c + 1;
@@ -136,31 +141,37 @@ __global__ void __launch_bounds__(kUpThreads, 1)
       const int s = c % kUpStages;
       if (!mbar_wait_converged(full0 + 8 * s, (c / kUpStages) & 1, abort_flag, p.status, p.wait_ns)) break;
       tc_fence_after();
-      const uint64_t ad = desc_sw128(sa + s * kUpStage, 16, 1024);
-      const uint64_t bd = desc_sw128(sa + s * kUpStage + kUpA, 16, 1024);
+      const uint64_t bd = desc_sw128(sa + s * kUpStage + 2 * kUpA, 16, 1024);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) mma_1_elect(tmem, ad + 2 * kk, bd + 2 * kk, kUpIdesc, (c | kk) != 0);
+      for (int i = 0; i < 2; ++i) {
+        const uint64_t ad = desc_sw128(sa + s * kUpStage + i * kUpA, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_1_elect(tmem + 256u * i, ad + 2 * kk, bd + 2 * kk, kUpIdesc, (c | kk) != 0);
+      }
       commit_1_elect(empty0 + 8 * s);
     }
     commit_1_elect(done);
   }
-  // ---- epilogue: TMEM lane = token, columns 0..127 Kn, 128..255 V.  Rows of
-  // the tile past the length (and every row after a wait ran out) get zeros:
-  // the attention multiplies them by zero weights, which must not meet a NaN.
+  // ---- epilogue: tile i in TMEM columns 256 i .. 256 i + 255, lane = token,
+  // Kn in the first 128 columns, V in the next.  Rows past the length (and every
+  // row after a wait ran out) get zeros: the attention multiplies them by zero
+  // weights, which must not meet a NaN.
   int keep = 0;
   mbar_wait(done, 0, &keep, nullptr, kDrainNs);
   __syncwarp();  // the tensor-memory loads below are warp-collective
   tc_fence_after();
-  const int t = t0 + 32 * warp + lane;
-  const bool ok = __shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(abort_flag), 0) == 0 && t < L;
-  const size_t orow = ((size_t)b * p.H + h) * p.Lmax + t;
+  const bool alive = __shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(abort_flag), 0) == 0;
 #pragma unroll 1
-  for (int half = 0; half < 2; ++half) {
-    __nv_bfloat16* dst = (half ? p.v : p.kn) + orow * 128;
+  for (int q = 0; q < 4; ++q) {
+    const int i = q >> 1, half = q & 1;
+    const int t = t0 + 128 * i + 32 * warp + lane;
+    const bool ok = alive && t < L;
+    __nv_bfloat16* dst = (half ? p.v : p.kn) + (((size_t)b * p.H + h) * p.Lmax + t) * 128;
 #pragma unroll 1
     for (int c0 = 0; c0 < 128; c0 += 32) {
       uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + 128 * half + c0, r);
+      tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + 256 * i + 128 * half + c0, r);
       tmem_wait_ld();
       if (!ok) {
 #pragma unroll
@@ -179,7 +190,7 @@ __global__ void __launch_bounds__(kUpThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc_1(tmem, 256);
+  if (warp == 1) tmem_dealloc_1(tmem, 512);
 }
 
 // ---------------------------------------------------------------- attention
@@ -504,13 +515,13 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 }  // namespace
 
 size_t prefill_workspace_bytes(int B, int H, int Lmax) {
-  // status header, then Kn and V, each [B][H][Lmax rounded up to 128][128] bf16
-  const size_t lpad = ((size_t)Lmax + 127) / 128 * 128;
+  // status header, then Kn and V, each [B][H][Lmax rounded up to 256][128] bf16
+  const size_t lpad = ((size_t)Lmax + kUpTok - 1) / kUpTok * kUpTok;
   return 256 + 2 * (size_t)B * H * lpad * 128 * 2;
 }
 
 cudaError_t launch_prefill(const mla_prefill_args_t* a, cudaStream_t stream) {
-  const int Lmax = (a->max_seq_len + 127) / 128 * 128;
+  const int Lmax = (a->max_seq_len + kUpTok - 1) / kUpTok * kUpTok;
   unsigned char* ws = static_cast<unsigned char*>(a->workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   __nv_bfloat16* kn = reinterpret_cast<__nv_bfloat16*>(ws + 256);
@@ -548,7 +559,7 @@ cudaError_t launch_prefill(const mla_prefill_args_t* a, cudaStream_t stream) {
   up.Lmax = Lmax;
   up.max_len = a->max_seq_len;
   up.wait_ns = device_wait_limit_ns();
-  e = launch_pdl(kv_up_kernel, dim3(Lmax / 128, a->H, a->B), dim3(kUpThreads), kUpSmem, stream, tm_c, tm_wuk,
+  e = launch_pdl(kv_up_kernel, dim3(Lmax / kUpTok, a->H, a->B), dim3(kUpThreads), kUpSmem, stream, tm_c, tm_wuk,
                  tm_wuv, up);
   if (e != cudaSuccess) return e;
   AtParams at;

@@ -156,14 +156,28 @@ __global__ void __launch_bounds__(NWARPS * 32) proj_kernel(const __grid_constant
     }
   }
 
+  // epilogue: the bf16 tile goes through shared memory (the stages are free after
+  // the loop's last barrier), then out in 16-byte pieces, consecutive threads on
+  // consecutive pieces of a row
+  constexpr int kPitch = NC * 2 + 16;  // bytes per staged row; the pad spreads banks
+  static_assert(TM * kPitch <= (int)C::STAGE * STAGES, "output tile fits the stages");
+  unsigned char* stile = smem_raw + (sa - raw);
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {
-    const int t = t0 + warp * 16 + (lane >> 2) + hf * 8;
-    if (t >= n_tok) continue;
-    __nv_bfloat16* yrow = Y + ((size_t)t * H + h) * N + n0 + 2 * (lane & 3);
+    const int rl = warp * 16 + (lane >> 2) + hf * 8;
 #pragma unroll
     for (int j = 0; j < NJ; ++j)
-      *reinterpret_cast<uint32_t*>(yrow + j * 8) = pack_bf16(acc[j][2 * hf], acc[j][2 * hf + 1]);
+      *reinterpret_cast<uint32_t*>(stile + rl * kPitch + (j * 8 + 2 * (lane & 3)) * 2) =
+          pack_bf16(acc[j][2 * hf], acc[j][2 * hf + 1]);
+  }
+  __syncthreads();
+  constexpr int kPieces = NC / 8;  // 16-byte pieces per row
+  for (int i = tid; i < TM * kPieces; i += C::NT) {
+    const int rl = i / kPieces, pc = i % kPieces;
+    const int t = t0 + rl;
+    if (t < n_tok)
+      *reinterpret_cast<uint4*>(Y + ((size_t)t * H + h) * N + n0 + pc * 8) =
+          *reinterpret_cast<const uint4*>(stile + rl * kPitch + pc * 16);
   }
 }
 

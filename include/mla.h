@@ -293,7 +293,7 @@ typedef struct {
 } mla_prefill_args_t;
 
 /* Bytes of workspace mla_prefill needs (host only): 256 plus the per-head keys
- * and values of every sequence, 2 * B * H * roundup(max_seq_len, 128) * 128 bf16. */
+ * and values of every sequence, 2 * B * H * roundup(max_seq_len, 256) * 128 bf16. */
 mla_status_t mla_prefill_workspace_size(const mla_prefill_args_t* args, size_t* bytes);
 
 /*

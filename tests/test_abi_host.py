@@ -223,9 +223,9 @@ def _pargs(B=4, s_q=1024, H=128, max_len=8192, **kw):
 
 
 def test_prefill_workspace_holds_keys_and_values(lib):
-    # per-head keys and values (128 bf16 each) of every sequence, rows padded to 128
+    # per-head keys and values (128 bf16 each) of every sequence, rows padded to 256
     assert mla.mla_prefill_workspace_size(_pargs()) == 256 + 2 * 4 * 128 * 8192 * 256
-    assert mla.mla_prefill_workspace_size(_pargs(B=1, H=1, s_q=1, max_len=1)) == 256 + 2 * 128 * 256
+    assert mla.mla_prefill_workspace_size(_pargs(B=1, H=1, s_q=1, max_len=1)) == 256 + 2 * 256 * 256
     assert mla.mla_prefill_workspace_size(_pargs(B=2, H=16, s_q=100, max_len=129)) == 256 + 2 * 32 * 256 * 256
 
 
