@@ -1,8 +1,8 @@
-// Paged latent-attention decode over a bf16 cache on the 5th-generation tensor
-// cores (sm_100a): tcgen05 MMAs over a CTA pair, accumulators in tensor memory
-// (TMEM), cache pages streamed by TMA.  16 to 128 heads (fewer heads pad the
-// 128-row tile with zero rows: the step stays bound by the cache stream, so the
-// idle rows cost tensor work only).  An e4m3 cache runs on decode_f8.cu.
+// Paged latent-attention decode over a bf16 or q8_0 cache on the 5th-generation
+// tensor cores (sm_100a): tcgen05 MMAs over a CTA pair, accumulators in tensor
+// memory (TMEM), cache pages streamed by TMA.  16 to 128 heads (fewer heads pad
+// the 128-row tile with zero rows: the step stays bound by the cache stream, so
+// the idle rows cost tensor work only).  An e4m3 cache runs on decode_f8.cu.
 //
 // What it computes (absorbed MLA decode; nnets.ru article, sections "Суть MLA"
 // and "MLA и FlashAttention"; snowgate thread 35 on the 512 + 64 latent record):
@@ -46,12 +46,22 @@
 // P.V of t.  The output rescale is lazy: the reference maximum moves only when
 // the tile maximum exceeds it by more than 2^8, so O in TMEM is rarely touched.
 //
+// q8_0 cache (ik_llama.cpp docs "FlashMLA", section "KV cache with MLA": int8
+// codes with one fp16 scale per 32 values): the same MMAs on bf16 operands.  The
+// producer brings the raw codes (and their block scales) into the back half of
+// the score and value slots; four converter warps (12..15, 512 threads in all)
+// read a slot's raw bytes into registers, meet at a named barrier, and write the
+// values code * scale (fp32 product, exact, rounded once to bf16) over the whole
+// slot in the layout TMA gives a bf16 cache, zeros for rows past the sequence
+// end; then they arrive on the even CTA's full barrier of that slot.
+//
 // Every mbarrier wait is bounded (MLA_ERR_DEVICE_TIMEOUT in the status word);
 // after one runs out every role leaves its loop, issued MMAs are drained, the
 // even CTA reconciles and waits for every copy either CTA issued, and TMEM is
 // freed (see the teardown).
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_fp16.h>
 #include <math_constants.h>
 
 #include "sm100.cuh"
@@ -65,6 +75,8 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 384;                // warps 0..11
+constexpr int kConvWarps = 4;                // q8_0: converter warps 12..15
+constexpr int kThreadsQ8 = kThreads + 32 * kConvWarps;
 constexpr uint32_t kChunkQ = 64 * 128;              // 64 rows x 64 bf16
 #ifndef MLA_TC_Q_TMEM_CHUNKS
 #define MLA_TC_Q_TMEM_CHUNKS 6
@@ -105,7 +117,9 @@ constexpr int S_FREE = DRAIN + 3;         // [2] in the even CTA: the softmax ha
 constexpr int RAW_V = S_FREE + 2;         // [kVStages] a last page's value stage landed here
 constexpr int Q_STAGE = RAW_V + kVStages; // Q chunks 0..5 landed in the value ring (this CTA)
 constexpr int Q_MOVED = Q_STAGE + 1;      // the softmax warps have moved them into TMEM
-constexpr int NBARS = Q_MOVED + 1;
+constexpr int RAW_QS = Q_MOVED + 1;       // [kSStages] q8_0: raw codes of a score slot landed (this CTA)
+constexpr int RAW_QV = RAW_QS + kSStages; // [kVStages] q8_0: raw codes of a value slot landed (this CTA)
+constexpr int NBARS = RAW_QV + kVStages;
 constexpr int kSoftmaxWarps = 8;          // warps 4..11: two per TMEM lane quadrant
 constexpr int kPrefetchTiles = MLA_TC_PREFETCH;      // L2 prefetch distance of the cache stream
 constexpr uint32_t kMiscOff = kBarOff + 8 * NBARS;
@@ -114,6 +128,19 @@ constexpr uint32_t kXlOff = kXmaxOff + 4 * 128 * 4;  // float [2][128]
 constexpr uint32_t kSmemUsed = kXlOff + 2 * 128 * 4;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;    // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+// q8_0: fp16 block scales beside the rings: 32 rows x 18 per score slot, 64 rows
+// x 18 per value slot; raw codes in the back half of each slot
+constexpr uint32_t kQ8RowBytes = kRow;                  // 576 int8 codes
+constexpr uint32_t kQ8ScRow = 18 * 2;                   // 36 bytes of scales per row
+constexpr uint32_t kQ8RawS = 32 * kQ8RowBytes;          // 18432: the CTA's 32 rows
+constexpr uint32_t kQ8RawV = 2 * 64 * 128;              // 16384: 64 rows x the CTA's 256 latent columns
+constexpr uint32_t kQ8ScS = 32 * kQ8ScRow;              // 1152
+constexpr uint32_t kQ8ScV = 64 * kQ8ScRow;              // 2304
+constexpr uint32_t kQ8ScOff = kSmemUsed;
+constexpr uint32_t kQ8ScVOff = kQ8ScOff + kSStages * kQ8ScS;
+constexpr uint32_t kSmemBytesQ8 = kQ8ScVOff + kVStages * kQ8ScV + 1024;
+static_assert(kSmemBytesQ8 <= 232448, "shared memory budget (q8_0)");
+static_assert(kSStage == 2 * kQ8RawS && kVStage == 2 * kQ8RawV, "raw codes fill the back half of a slot");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 256;                     // S buffers at columns 256, 288
 constexpr uint32_t kTmemQ = 320;                     // Q chunks 0..5: columns 320..511 (2 bf16 each)
@@ -128,6 +155,7 @@ struct TcParams {
   const __nv_bfloat16* q_lat;
   const __nv_bfloat16* q_pe;
   const uint8_t* kv;
+  const uint8_t* kv_scale;  // q8_0: fp16 [pages][64][18], 16-byte aligned
   const int32_t* block_table;
   const int32_t* seq_lens;
   __nv_bfloat16* o_lat;
@@ -140,7 +168,15 @@ struct TcParams {
   uint64_t wait_ns;
 };
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+// q8_0 value of one code: the byte with its sign bit flipped, put under the
+// exponent of 2^23, is 2^23 + 128 + code exactly; subtracting gives the code,
+// and code * scale (8 x 11 significant bits) is exact in fp32.
+MLA_DEVI float q8_code(uint32_t word_flipped, int k) {
+  return __int_as_float((int)__byte_perm(word_flipped, 0x4B000000u, 0x7440u + k)) - 8388736.0f;
+}
+
+template <bool Q8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qpe,
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_kv,
                      const __grid_constant__ CUtensorMap tm_o, const TcParams p) {
@@ -178,14 +214,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // a full score stage is the even CTA's expect_tx plus both CTAs' TMA bytes, a
     // full value stage that and the odd CTA's arrival (a last, partial page
     // instead takes one arrival per CTA after its tail rows are zeroed)
+    // q8_0: a full stage is the arrival of both CTAs' converter warps instead
     for (int i = 0; i < kSStages; ++i) {
-      mbar_init(own_bar(S_FULL + i), 1);
+      mbar_init(own_bar(S_FULL + i), Q8 ? 2 * kConvWarps : 1);
       mbar_init(own_bar(S_EMPTY + i), 1);
+      mbar_init(own_bar(RAW_QS + i), 1);
     }
     for (int i = 0; i < kVStages; ++i) {
-      mbar_init(own_bar(V_FULL + i), 2);
+      mbar_init(own_bar(V_FULL + i), Q8 ? 2 * kConvWarps : 2);
       mbar_init(own_bar(V_EMPTY + i), 1);
       mbar_init(own_bar(RAW_V + i), 1);
+      mbar_init(own_bar(RAW_QV + i), 1);
     }
     mbar_init(own_bar(Q_TMEM), 2 * kSoftmaxWarps);
     mbar_init(own_bar(Q_FULL), 1);
@@ -251,7 +290,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // the CTA's half page (32 contiguous rows) of tile u, into L2 ahead of its TMA
       auto prefetch = [&](int u) {
         const int pg = page_of(u, blk_p, pg_p);
-        if (lane == 0) prefetch_l2_bulk(p.kv + ((size_t)pg * kPage + 32 * r) * kRow * 2, 32 * kRow * 2);
+        constexpr uint32_t kRowBytes = Q8 ? kQ8RowBytes : kRow * 2;
+        if (lane == 0) prefetch_l2_bulk(p.kv + ((size_t)pg * kPage + 32 * r) * kRowBytes, 32 * kRowBytes);
       };
       auto load_s = [&](int u) -> bool {
         const int st = u % kSStages;
@@ -259,6 +299,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!mbar_wait_converged(own_bar(S_EMPTY + st), ph, abort_flag, p.status, wait_ns)) return false;
         const int pg = page_of(u, blk_s, pg_s);
         const uint32_t dst = sa + kSOff + st * kSStage;
+        if constexpr (Q8) {
+          // the CTA's 32 rows of codes (contiguous) into the back half of the slot,
+          // their block scales beside the ring; the converters take it from there
+          if (lane == 0) {
+            const size_t row0 = (size_t)pg * kPage + 32 * r;
+            mbar_arrive_expect_tx_local(own_bar(RAW_QS + st), kQ8RawS + kQ8ScS);
+            bulk_load_cta(dst + kQ8RawS, p.kv + row0 * kQ8RowBytes, kQ8RawS, own_bar(RAW_QS + st));
+            bulk_load_cta(sa + kQ8ScOff + st * kQ8ScS, p.kv_scale + row0 * kQ8ScRow, kQ8ScS,
+                          own_bar(RAW_QS + st));
+          }
+          __syncwarp();
+          n_s = u + 1;
+          if (u > 0 && u + kPrefetchTiles < n) prefetch(u + kPrefetchTiles);
+          return true;
+        }
         // one box: (64 values, 32 rows, 9 chunks) lands chunk-major, 9 x 4 KB
         const uint32_t fb = lead_bar(S_FULL + st);
         if (r == 0) mbar_arrive_expect_tx_local_elect(own_bar(S_FULL + st), 2 * kSStage);
@@ -273,6 +328,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!mbar_wait_converged(own_bar(V_EMPTY + st), ph, abort_flag, p.status, wait_ns)) return false;
         const int pg = page_of(u, blk_v, pg_v);
         const uint32_t dst = sa + kVOff + st * kVStage;
+        if constexpr (Q8) {
+          // the page's 64 rows x the CTA's latent columns 128r .. +127 and
+          // 256 + 128r .. +127 (two boxes of 64 rows x 128 codes) into the back
+          // half of the slot, the page's block scales beside the ring
+          if (lane == 0) {
+            mbar_arrive_expect_tx_local(own_bar(RAW_QV + st), kQ8RawV + kQ8ScV);
+            tma_load_2d_cta(dst + kQ8RawV, &tm_kv, own_bar(RAW_QV + st), 128 * (int)r, pg * kPage);
+            tma_load_2d_cta(dst + kQ8RawV + kQ8RawV / 2, &tm_kv, own_bar(RAW_QV + st), 256 + 128 * (int)r,
+                            pg * kPage);
+            bulk_load_cta(sa + kQ8ScVOff + st * kQ8ScV, p.kv_scale + (size_t)pg * kPage * kQ8ScRow, kQ8ScV,
+                          own_bar(RAW_QV + st));
+          }
+          __syncwarp();
+          n_v = u + 1;
+          return true;
+        }
         const int nvalid = j_end - (t0 + u) * kPage;  // cached rows of this page inside the sequence
         if (nvalid >= kPage) {
           // one box: (64 values, 64 rows, chunks 2r and 2r+1, groups 0 and 1): latent
@@ -376,7 +447,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (u >= 2 && !mbar_wait_converged(own_bar(S_FREE + sb), ((u - 2) >> 1) & 1, abort_flag, p.status,
                                              wait_ns))
             break;
-          if (!mbar_wait_converged(own_bar(S_FULL + st), (u / kSStages) & 1, abort_flag, p.status, wait_ns))
+          if (!mbar_wait_converged<Q8>(own_bar(S_FULL + st), (u / kSStages) & 1, abort_flag, p.status, wait_ns))
             break;
           tc_fence_after();
           const uint32_t d = tmem + kTmemS + 32u * sb;
@@ -407,7 +478,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int pb = t & 1, st = t % kVStages;
           if (!mbar_wait_converged(own_bar(P_READY + pb), (t >> 1) & 1, abort_flag, p.status, wait_ns))
             break;
-          if (!mbar_wait_converged(own_bar(V_FULL + st), (t / kVStages) & 1, abort_flag, p.status, wait_ns))
+          if (!mbar_wait_converged<Q8>(own_bar(V_FULL + st), (t / kVStages) & 1, abort_flag, p.status, wait_ns))
             break;
           tc_fence_after();
           const uint64_t ap = dp + ((pb * kPBytes) >> 4);
@@ -429,7 +500,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int keep_waiting = 0;
       mbar_wait_converged(own_bar(db), 0, &keep_waiting, p.status, kDrainLimitNs);
     }
-  } else {
+  } else if (warp < 12) {
     // ====================== softmax / correction / epilogue ======================
     // Thread = (TMEM lane lt, column half ch).  Lane lt holds head row m = lt % 64
     // for tokens 32*half .. 32*half+31 of the page (half = lt / 64); the two warps
@@ -642,6 +713,97 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     }
     tc_fence_before();
+  } else if constexpr (Q8) {
+    // ====================== q8_0 converters (warps 12..15) ======================
+    // Per page: the score slot (this CTA's 32 rows x 576 values, 9 chunks of
+    // 32 rows x 128 bytes, 128-byte swizzle) and the value slot (64 rows x the
+    // CTA's latent chunks 2r, 2r+1, 4+2r, 5+2r, 4 chunks of 64 rows x 128 bytes).
+    // The raw codes sit in the back half of the slot they expand into, so every
+    // thread reads its share into registers before any thread writes.  The four
+    // warps meet at named barriers, so they leave the loop together: the
+    // outcome of each wait is combined over the group first.
+    const int ct = threadIdx.x - kThreads;  // 0 .. 127
+    const __half* scs = reinterpret_cast<const __half*>(sm + kQ8ScOff);
+    const __half* scv = reinterpret_cast<const __half*>(sm + kQ8ScVOff);
+    auto conv_s = [&](int u) -> bool {
+      const int tok0 = (t0 + u) * kPage;  // first token of the page
+      {
+        const int st = u % kSStages;
+        const bool got = mbar_wait_converged(own_bar(RAW_QS + st), (u / kSStages) & 1, abort_flag, p.status, wait_ns);
+        if (!named_bar_and(6, 32 * kConvWarps, got)) return false;
+        const uint32_t slot = sa + kSOff + st * kSStage;
+        uint4 raw[9];
+#pragma unroll
+        for (int i = 0; i < 9; ++i) {
+          const int q = ct + 128 * i, row = q / 36, k0 = 16 * (q % 36);
+          raw[i] = lds128(slot + kQ8RawS + row * kQ8RowBytes + k0);
+        }
+        named_bar_sync(6, 32 * kConvWarps);
+#pragma unroll
+        for (int i = 0; i < 9; ++i) {
+          const int q = ct + 128 * i, row = q / 36, k0 = 16 * (q % 36);
+          const bool live = tok0 + 32 * (int)r + row < j_end;
+          const float d = live ? __half2float(scs[(st * 32 + row) * 18 + (k0 >> 5)]) : 0.f;
+          const uint32_t w[4] = {raw[i].x ^ 0x80808080u, raw[i].y ^ 0x80808080u, raw[i].z ^ 0x80808080u,
+                                 raw[i].w ^ 0x80808080u};
+          uint32_t o[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            o[k] = pack_bf16(q8_code(w[k >> 1], 2 * (k & 1)) * d, q8_code(w[k >> 1], 2 * (k & 1) + 1) * d);
+          const int c = k0 >> 6, unit = (k0 & 63) >> 3;
+          const uint32_t base = slot + c * kChunkS + row * 128;
+          sts128(base + (((unit) ^ (row & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
+          sts128(base + (((unit + 1) ^ (row & 7)) << 4), make_uint4(o[4], o[5], o[6], o[7]));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote_release_cluster(lead_bar(S_FULL + st));
+      }
+      return true;
+    };
+    auto conv_v = [&](int u) -> bool {
+      const int tok0 = (t0 + u) * kPage;  // first token of the page
+      {
+        const int st = u % kVStages;
+        const bool got = mbar_wait_converged(own_bar(RAW_QV + st), (u / kVStages) & 1, abort_flag, p.status, wait_ns);
+        if (!named_bar_and(6, 32 * kConvWarps, got)) return false;
+        const uint32_t slot = sa + kVOff + st * kVStage;
+        uint4 raw[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) raw[i] = lds128(slot + kQ8RawV + 16 * (ct + 128 * i));
+        named_bar_sync(6, 32 * kConvWarps);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          // box nb (latent columns 128r.. or 256 + 128r..), row, 16 codes from column 16 c16
+          const int q = ct + 128 * i, nb = q >> 9, row = (q >> 3) & 63, c16 = q & 7;
+          const int col = 256 * nb + 128 * (int)r + 16 * c16;
+          const bool live = tok0 + row < j_end;
+          const float d = live ? __half2float(scv[(st * 64 + row) * 18 + (col >> 5)]) : 0.f;
+          const uint32_t w[4] = {raw[i].x ^ 0x80808080u, raw[i].y ^ 0x80808080u, raw[i].z ^ 0x80808080u,
+                                 raw[i].w ^ 0x80808080u};
+          uint32_t o[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            o[k] = pack_bf16(q8_code(w[k >> 1], 2 * (k & 1)) * d, q8_code(w[k >> 1], 2 * (k & 1) + 1) * d);
+          const int j = 2 * nb + (c16 >> 2), unit = 2 * (c16 & 3);
+          const uint32_t base = slot + j * kChunkV + row * 128;
+          sts128(base + ((unit ^ (row & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
+          sts128(base + (((unit + 1) ^ (row & 7)) << 4), make_uint4(o[4], o[5], o[6], o[7]));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote_release_cluster(lead_bar(V_FULL + st));
+      }
+      return true;
+    };
+    // score slots one page ahead of value slots, in the order the producer
+    // requests them: the score MMA of page u + 1 never waits for the value
+    // conversion of page u, whose raw codes are requested later
+    bool ok = n > 0 ? conv_s(0) : true;
+    for (int u = 0; ok && u < n; ++u) {
+      if (u + 1 < n) ok = conv_s(u + 1);
+      if (ok) ok = conv_v(u);
+    }
   }
 
   // ---- teardown: both CTAs are done with TMEM and shared memory
@@ -664,7 +826,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int ns1 = (int)ld_shared_cluster_u32(mapa(sa + kMiscOff + 8, 1));
     const int nv1 = (int)ld_shared_cluster_u32(mapa(sa + kMiscOff + 12, 1));
     int give_up = 0;
-    if (r == 0) {
+    if constexpr (Q8) {
+      // q8_0: the raw codes of every slot land on this CTA's own barriers; the
+      // full barriers count the converters' arrivals only (no bytes in flight)
+      const int ns = r == 0 ? ns0 : ns1, nv = r == 0 ? nv0 : nv1;
+      for (int u = max(0, ns - kSStages); u < ns; ++u)
+        mbar_wait(own_bar(RAW_QS + u % kSStages), (u / kSStages) & 1, &give_up, nullptr, kDrainLimitNs);
+      for (int u = max(0, nv - kVStages); u < nv; ++u)
+        mbar_wait(own_bar(RAW_QV + u % kVStages), (u / kVStages) & 1, &give_up, nullptr, kDrainLimitNs);
+      if (r == 0 && issued[3]) mbar_wait(own_bar(Q_FULL), 0, &give_up, nullptr, kDrainLimitNs);
+    } else if (r == 0) {
       for (int u = min(ns0, ns1); u < max(ns0, ns1); ++u) {
         if (ns0 > ns1) mbar_complete_tx_local(own_bar(S_FULL + u % kSStages), kSStage);
         else mbar_arrive_expect_tx_local(own_bar(S_FULL + u % kSStages), kSStage);
@@ -706,16 +877,27 @@ cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t strea
   // score operand: (64 values, rows, 9 chunks 128 bytes apart), one box per stage;
   // value operand: (64 values, rows, 4 chunks 128 bytes apart, 2 groups 512 bytes
   // apart), one box of 2 x 2 chunks per stage
-  const uint64_t dks[3] = {64, rows_kv, 9}, sks[2] = {kRow * 2, 128};
-  const uint32_t bks[3] = {64, 32, 9};
-  const uint64_t dkv[4] = {64, rows_kv, 4, 2}, skv[3] = {kRow * 2, 128, 512};
-  const uint32_t bkv[4] = {64, 64, 2, 2};
-  if (!tma_map_nd(&tm_ks, a->kv_cache, 3, dks, sks, bks) || !tma_map_nd(&tm_kv, a->kv_cache, 4, dkv, skv, bkv))
-    return cudaErrorInvalidValue;
+  const bool q8 = a->kv_dtype == MLA_KV_Q8_0;
+  if (q8) {
+    // q8_0: the value operand's raw codes, boxes of 64 rows x 128 codes (no
+    // swizzle); the score operand comes by bulk copies (tm_ks is not read)
+    const uint64_t dq[2] = {kRow, rows_kv}, sq[1] = {kRow};
+    const uint32_t bq[2] = {128, 64};
+    if (!tma_map_nd(&tm_kv, a->kv_cache, 2, dq, sq, bq, true, 0)) return cudaErrorInvalidValue;
+    tm_ks = tm_kv;
+  } else {
+    const uint64_t dks[3] = {64, rows_kv, 9}, sks[2] = {kRow * 2, 128};
+    const uint32_t bks[3] = {64, 32, 9};
+    const uint64_t dkv[4] = {64, rows_kv, 4, 2}, skv[3] = {kRow * 2, 128, 512};
+    const uint32_t bkv[4] = {64, 64, 2, 2};
+    if (!tma_map_nd(&tm_ks, a->kv_cache, 3, dks, sks, bks) || !tma_map_nd(&tm_kv, a->kv_cache, 4, dkv, skv, bkv))
+      return cudaErrorInvalidValue;
+  }
   TcParams p;
   p.q_lat = static_cast<const __nv_bfloat16*>(a->q_lat);
   p.q_pe = static_cast<const __nv_bfloat16*>(a->q_pe);
   p.kv = static_cast<const uint8_t*>(a->kv_cache);
+  p.kv_scale = static_cast<const uint8_t*>(a->kv_scale);
   p.block_table = a->block_table;
   p.seq_lens = a->seq_lens;
   p.o_lat = static_cast<__nv_bfloat16*>(a->o_lat);
@@ -734,16 +916,24 @@ cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t strea
   p.splits = splits;
   p.scale_log2 = a->softmax_scale * kLog2e;
   p.wait_ns = device_wait_limit_ns();
-  auto kern = decode_tc_kernel;
-  static PerDeviceOnce attrs;
-  cudaError_t e = once_per_device(attrs, [&]() {
-    cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  dim3 grid(2 * splits, a->s_q, a->B);
+  auto set_attrs = [](auto kern, uint32_t smem) {
+    cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e2 != cudaSuccess) return e2;
     return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-  });
+  };
+  if (q8) {
+    static PerDeviceOnce attrs_q8;
+    cudaError_t e = once_per_device(attrs_q8, [&]() { return set_attrs(decode_tc_kernel<true>, kSmemBytesQ8); });
+    if (e != cudaSuccess) return e;
+    return launch_pdl(decode_tc_kernel<true>, grid, dim3(kThreadsQ8), kSmemBytesQ8, stream, tm_q, tm_qpe, tm_ks,
+                      tm_kv, tm_o, p);
+  }
+  static PerDeviceOnce attrs;
+  cudaError_t e = once_per_device(attrs, [&]() { return set_attrs(decode_tc_kernel<false>, kSmemBytes); });
   if (e != cudaSuccess) return e;
-  dim3 grid(2 * splits, a->s_q, a->B);
-  return launch_pdl(kern, grid, dim3(kThreads), kSmemBytes, stream, tm_q, tm_qpe, tm_ks, tm_kv, tm_o, p);
+  return launch_pdl(decode_tc_kernel<false>, grid, dim3(kThreads), kSmemBytes, stream, tm_q, tm_qpe, tm_ks, tm_kv,
+                    tm_o, p);
 }
 
 }  // namespace
@@ -752,10 +942,11 @@ cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t strea
 // an e4m3 cache) take these arguments.
 bool decode_tc_supported(const mla_decode_args_t* a) {
   // any head count up to 128 (rows beyond H pad the 128-row tile); a bf16 cache,
-  // or an e4m3 cache whose scale array starts on 16 bytes (bulk copies)
+  // or an e4m3 or q8_0 cache whose scale array starts on 16 bytes (bulk copies)
   if (a->H % 16 != 0 || a->H > 128) return false;
   if (a->kv_dtype == MLA_KV_BF16) return true;
-  return a->kv_dtype == MLA_KV_FP8_E4M3 && (reinterpret_cast<uintptr_t>(a->kv_scale) & 15u) == 0;
+  return (a->kv_dtype == MLA_KV_FP8_E4M3 || a->kv_dtype == MLA_KV_Q8_0) &&
+         (reinterpret_cast<uintptr_t>(a->kv_scale) & 15u) == 0;
 }
 
 int decode_tc_clusters_per_split(const mla_decode_args_t* a) { return a->B * a->s_q; }

@@ -43,6 +43,11 @@ MLA_DEVI void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.clus
 MLA_DEVI void mbar_arrive_remote(uint32_t addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
 }
+// Arrive on a barrier of either CTA of the pair, releasing this thread's prior
+// writes at cluster scope (for data the other CTA's waiters then read).
+MLA_DEVI void mbar_arrive_remote_release_cluster(uint32_t addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
 // Arrive on a barrier of either CTA of the pair with no ordering of this thread's
 // memory operations (for arrivals that only count).
 MLA_DEVI void mbar_arrive_remote_relaxed(uint32_t addr) {
@@ -516,6 +521,20 @@ MLA_DEVI float ex2_approx(float x) {
 
 MLA_DEVI void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Named barrier that also returns whether `pred` held in every participating
+// thread (so that a group of warps takes one decision together).
+MLA_DEVI bool named_bar_and(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 }  // namespace sm100

@@ -18,7 +18,8 @@ TIMEOUT = 6
 
 
 # split count 0: the automatic choice
-@pytest.mark.parametrize("kv,splits", [("bf16", 0), ("bf16", 1), ("bf16", 3), ("fp8", 1), ("fp8", 2)])
+@pytest.mark.parametrize("kv,splits", [("bf16", 0), ("bf16", 1), ("bf16", 3), ("fp8", 1), ("fp8", 2), ("q8_0", 1),
+                                      ("q8_0", 2)])
 def test_wait_that_runs_out_is_reported_and_the_context_stays_usable(cuda_lib, kv, splits):
     from head_latent_attention_06_b200.step import step_from_workload
     w = make_workload(WorkloadSpec("to", B=3, H=128, s_q=1, lens=[1000, 300, 70], kv_dtype=kv, seed=31,

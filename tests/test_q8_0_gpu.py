@@ -12,11 +12,16 @@ from parity_util import check_close, compare_step, oracle_of, report, to_np
 pytestmark = pytest.mark.gpu
 
 
-def _run(cuda_lib, w, splits=0):
+def _run(cuda_lib, w, splits=0, kernel=None):
     from head_latent_attention_06_b200.step import step_from_workload
-    st = step_from_workload(w, num_splits=splits)
-    st.run()
-    torch.cuda.synchronize()
+    if kernel is not None:
+        cuda_lib.mla_set_decode_kernel(kernel)
+    try:
+        st = step_from_workload(w, num_splits=splits)
+        st.run()
+        torch.cuda.synchronize()
+    finally:
+        cuda_lib.mla_set_decode_kernel(cuda_lib.DECODE_AUTO)
     assert cuda_lib.mla_get_status(st.workspace) == 0
     return st
 
@@ -31,12 +36,16 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("kernel", ["tensor_memory", "warp_mma"])
 @pytest.mark.parametrize("H,s_q,causal,lens,splits", CASES)
-def test_q8_0_decode_every_element(cuda_lib, H, s_q, causal, lens, splits):
+def test_q8_0_decode_every_element(cuda_lib, H, s_q, causal, lens, splits, kernel):
+    """Both decode kernels: the tensor-memory one (converter warps expand the
+    codes into bf16 operands) and the warp-MMA one."""
     w = make_workload(WorkloadSpec("q8c", B=len(lens), H=H, s_q=s_q, lens=lens, kv_dtype="q8_0",
                                    causal=causal, seed=17))
-    st = _run(cuda_lib, w, splits)
-    report(f"q8_0 H={H} s_q={s_q} lens={lens} splits={splits}", compare_step(st, w, oracle_of(w, absorbed=True)))
+    st = _run(cuda_lib, w, splits, None if kernel == "tensor_memory" else cuda_lib.DECODE_WARP_MMA)
+    report(f"q8_0 {kernel} H={H} s_q={s_q} lens={lens} splits={splits}",
+           compare_step(st, w, oracle_of(w, absorbed=True)))
     # and the explicit-K/V definition on two heads of the longest sequence
     b = int(np.argmax(lens))
     rows = [(b, i) for i in range(s_q)]
@@ -53,14 +62,16 @@ def test_q8_0_full_size_sampled(cuda_lib):
     assert torch.isfinite(st.out).all()
 
 
-def test_q8_0_bytes_past_the_sequence_end_never_reach_the_output(cuda_lib):
+@pytest.mark.parametrize("kernel", ["tensor_memory", "warp_mma"])
+def test_q8_0_bytes_past_the_sequence_end_never_reach_the_output(cuda_lib, kernel):
+    k = None if kernel == "tensor_memory" else cuda_lib.DECODE_WARP_MMA
     w = make_workload(WorkloadSpec("q8t", B=2, H=128, s_q=1, lens=[70, 129], kv_dtype="q8_0", seed=19))
-    clean = to_np(_run(cuda_lib, w).out)
+    clean = to_np(_run(cuda_lib, w, kernel=k).out)
     for b, L in enumerate(w.lens):
         pg = int(w.block_table[b, L // 64])
         w.kv_cache[pg, L % 64:] = 127
         w.kv_scale[pg, L % 64:] = float("nan")
-    st = _run(cuda_lib, w)
+    st = _run(cuda_lib, w, kernel=k)
     assert torch.isfinite(st.out).all()
     assert np.abs(to_np(st.out) - clean).max() <= 1e-2
 
