@@ -396,22 +396,25 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       const int sb = j % kSBufs;
       if (!mbar_wait_converged(bar(A_SREADY + sb), (j / kSBufs) & 1, abort_flag, p.status, wait_ns)) break;
       tc_fence_after();
-      float s[128];
+      // the row's 128 raw scores: four loads in flight, one wait
+      uint32_t sr[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tl + 128u * sb + 32u * c, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int k = 0; k < 32; ++k) s[32 * c + k] = __uint_as_float(r[k]);
-      }
+      for (int c = 0; c < 4; ++c) tmem_ld32(tl + 128u * sb + 32u * c, sr[c]);
+      tmem_wait_ld();
       const int nv = max(0, min(128, vis - 128 * j));  // visible keys of this tile
-      float mx = -CUDART_INF_F;
+      float s[128];
+      // eight independent running maxima (the softmax scale is positive, so it
+      // commutes with the maximum and is applied once)
+      float mx8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx8[k] = -CUDART_INF_F;
 #pragma unroll
       for (int k = 0; k < 128; ++k) {
-        s[k] = k < nv ? s[k] * p.scale_log2 : -CUDART_INF_F;
-        mx = fmaxf(mx, s[k]);
+        s[k] = k < nv ? __uint_as_float(sr[k >> 5][k & 31]) : -CUDART_INF_F;
+        mx8[k & 7] = fmaxf(mx8[k & 7], s[k]);
       }
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
       float alpha = 1.f;
       bool resc = false;
       if (mx > -CUDART_INF_F) {
@@ -442,18 +445,21 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         }
         tmem_wait_st();
       }
-      // P over S in place: 128 keys -> 64 columns of bf16 pairs
+      // P over S in place: 128 keys -> 64 columns of bf16 pairs; p = 2^(s * scale - m)
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t pk[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
-          const float p0 = ex2_approx(s[64 * c + 2 * k] + nref), p1 = ex2_approx(s[64 * c + 2 * k + 1] + nref);
-          l += p0 + p1;
+          const float p0 = ex2_approx(fmaf(s[64 * c + 2 * k], p.scale_log2, nref));
+          const float p1 = ex2_approx(fmaf(s[64 * c + 2 * k + 1], p.scale_log2, nref));
+          l4[k & 3] += p0 + p1;
           pk[k] = pack_bf16(p0, p1);
         }
         tmem_st32(tl + 128u * sb + 32u * c, pk);
       }
+      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
