@@ -43,13 +43,15 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # taken: reported as the roofline's ``traffic`` only while they are unchanged.
 MEASURED_TRAFFIC = {
     # ncu --set full, one launch of the V3 workload
-    "v3": (315_607_808, "decode_tc.cu", "a600c572d632e248"),
+    "v3": (315_950_848, "decode_tc.cu", "bb57f78a60d746ba"),
     # one launch of the fp8 workload
     "fp8": (773_860_864, "decode_f8.cu", "46f792446c3adafd"),
+    # one launch of the q8_0 workload (the same kernel file, its q8_0 variant)
+    "q8": (173_924_608, "decode_tc.cu", "bb57f78a60d746ba"),
     # both prefill kernels on one sequence of the chunked-prefill workload:
-    # 1,155,835,392 bytes, times the 4 sequences
-    # of the full workload (traffic grows with the sequences processed)
-    "prefill": (4 * 1_155_835_392, "prefill.cu", "d9eeb2f7c6032754"),
+    # 1,158,377,984 bytes, times the 4 sequences of the full workload (traffic
+    # grows with the sequences processed)
+    "prefill": (4 * 1_158_377_984, "prefill.cu", "c1b4e194ba1d3b2b"),
 }
 KERNEL_HEADERS = ("sm100.cuh", "common.cuh", "tma_host.cuh")
 
