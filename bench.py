@@ -45,7 +45,10 @@ MEASURED_TRAFFIC = {
     # ncu --set full, one launch of the V3 workload
     "v3": (315_950_848, "decode_tc.cu", "bb57f78a60d746ba"),
     # one launch of the fp8 workload
-    "fp8": (773_860_864, "decode_f8.cu", "46f792446c3adafd"),
+    "fp8": (773_830_144, "decode_f8.cu", "08afb13fc61221a1"),
+    # one launch of each long-context workload
+    "long16": (608_961_280, "decode_tc.cu", "bb57f78a60d746ba"),
+    "long128": (608_796_160, "decode_tc.cu", "bb57f78a60d746ba"),
     # one launch of the q8_0 workload (the same kernel file, its q8_0 variant)
     "q8": (173_924_608, "decode_tc.cu", "bb57f78a60d746ba"),
     # both prefill kernels on one sequence of the chunked-prefill workload:
