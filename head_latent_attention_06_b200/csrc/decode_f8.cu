@@ -99,7 +99,9 @@ constexpr int DRAIN = O_DONE + 2;          // [3] one per MMA-issuing warp
 constexpr int S_FREE = DRAIN + 3;          // [2] even CTA: the softmax has read S buffer sb
 constexpr int RAW_V = S_FREE + 2;          // [kVStages] a last page's value stage landed (this CTA)
 constexpr int SC_FULL = RAW_V + kVStages;  // [kScRing] token scales of a tile landed (this CTA)
-constexpr int NBARS = SC_FULL + kScRing;
+constexpr int Q_STAGE = SC_FULL + kScRing; // this CTA's Q rows (bf16) landed in the staging areas
+constexpr int Q_FREE = Q_STAGE + 1;        // the softmax warps have read them: the value ring is free
+constexpr int NBARS = Q_FREE + 1;
 // A scale slot is reloaded for tile u + kScRing only after the score stage of
 // tile u + kScRing - kSStages was consumed; that score MMA waited for every
 // softmax warp to release the S buffer of tile u + kScRing - kSStages - 2, which
@@ -111,8 +113,15 @@ constexpr int kPrefetchTiles = 2;          // L2 prefetch distance of the cache 
 constexpr uint32_t kMiscOff = kBarOff + 8 * NBARS;      // tmem slot, abort flag, issue counts
 constexpr uint32_t kXmaxOff = kMiscOff + 32;            // float [2 tiles][2 column halves][128 lanes]
 constexpr uint32_t kXlOff = kXmaxOff + 4 * 128 * 4;     // float [2][128]
-constexpr uint32_t kSmemUsed = kXlOff + 2 * 128 * 4;
+// Q (bf16, the CTA's 64 head rows) is staged by TMA before it is split: K 0..383
+// (the TMEM part, six 64-value chunks of 64 rows x 128 bytes, 128-byte swizzle) in
+// the value ring, idle until the first value stage; K 384..575 (two latent chunks
+// and q_pe) in an area of its own
+constexpr uint32_t kQStChunk = 64 * 128;
+constexpr uint32_t kQStOff = (kXlOff + 2 * 128 * 4 + 1023) / 1024 * 1024;
+constexpr uint32_t kSmemUsed = kQStOff + 3 * kQStChunk;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;       // + alignment slack
+static_assert(kVStages * kVStage >= 6 * kQStChunk, "Q staging in the value ring");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 256;                        // S buffers at columns 256, 288
@@ -165,7 +174,8 @@ MLA_DEVI float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_f8_kernel(const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_kv,
-                     const __grid_constant__ CUtensorMap tm_o, const F8Params p) {
+                     const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_qpe, const F8Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
@@ -179,7 +189,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kMiscOff + 4);
   // producer's issue counts, read by the teardown: score tiles, full value pages,
-  // last (partial) value page issued, token-scale tiles
+  // last (partial) value page issued, Q staged
   uint32_t* issued = reinterpret_cast<uint32_t*>(sm + kMiscOff + 8);
   float* xmax = reinterpret_cast<float*>(sm + kXmaxOff);
   float* xl = reinterpret_cast<float*>(sm + kXlOff);
@@ -204,6 +214,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(own_bar(RAW_V + i), 1);
     }
     for (int i = 0; i < kScRing; ++i) mbar_init(own_bar(SC_FULL + i), 1);
+    mbar_init(own_bar(Q_STAGE), 1);
+    mbar_init(own_bar(Q_FREE), kSoftmaxWarps);
     mbar_init(own_bar(Q_TMEM), 2 * kSoftmaxWarps);
     for (int i = 0; i < 2; ++i) {
       mbar_init(own_bar(S_READY + i), 1);
@@ -241,7 +253,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // =========================== TMA producer ===========================
-    int n_s = 0, n_v = 0, v_part = 0;
+    int n_s = 0, n_v = 0, v_part = 0, q_iss = 0;
     if (n > 0) {
       // physical pages, fetched 32 at a time by the whole warp
       int blk_s = -1, pg_s = 0, blk_v = -1, pg_v = 0, blk_p = -1, pg_p = 0;
@@ -321,15 +333,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         return true;
       };
       // The cache, block table and lengths are not written by any kernel this one
-      // may overlap with (the cache write lets nothing after it start early); Q is
-      // read by the softmax warps after their own wait for the previous kernel.
+      // may overlap with (the cache write lets nothing after it start early); Q is,
+      // so it is requested after the wait for the previous kernel.
       bool ok = load_s(0);
       pdl_wait();
+      if (lane == 0) {
+        // this CTA's 64 head rows of Q (3-D maps: heads >= H read as zeros): K 0..383
+        // into the value ring, K 384..575 into the Q staging area
+        const int qtok = b * p.s_q + g, h0 = 64 * (int)r;
+        mbar_arrive_expect_tx_local(own_bar(Q_STAGE), 9 * kQStChunk);
+        for (int c = 0; c < 6; ++c)
+          tma_load_3d_cta(sa + kVOff + c * kQStChunk, &tm_q, own_bar(Q_STAGE), 64 * c, h0, qtok);
+        for (int c = 6; c < 8; ++c)
+          tma_load_3d_cta(sa + kQStOff + (c - 6) * kQStChunk, &tm_q, own_bar(Q_STAGE), 64 * c, h0, qtok);
+        tma_load_3d_cta(sa + kQStOff + 2 * kQStChunk, &tm_qpe, own_bar(Q_STAGE), 0, h0, qtok);
+      }
+      __syncwarp();
+      q_iss = 1;
       for (int u = 1; u < n && u <= kPrefetchTiles; ++u) prefetch(u);
-      // score stages two tiles ahead of value stages
+      // score stages two tiles ahead of value stages; the first value stage waits
+      // until the softmax warps have read Q out of the value ring
       if (ok && n > 1) ok = load_s(1);
       for (int u = 0; ok && u < n; ++u) {
         if (u + 2 < n) ok = load_s(u + 2);
+        if (u == 0 && ok) ok = mbar_wait_converged(own_bar(Q_FREE), 0, abort_flag, p.status, wait_ns);
         if (ok) ok = load_v(u);
       }
     }
@@ -337,6 +364,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       issued[0] = n_s;
       issued[1] = n_v;
       issued[2] = v_part;
+      issued[3] = q_iss;
     }
   } else if (warp >= 1 && warp <= 3) {
     // ==== MMA issuers (even CTA): warps 1 and 3 scores (even / odd pages), warp 2 P.V ====
@@ -430,14 +458,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const size_t qr = ((size_t)b * p.s_q + g) * p.H + (row_ok ? head : 0);
     float s_h = 1.f;                        // the Q row's power-of-two scale
     if (n > 0) {
-      // This thread's Q values: K [192 ch, 192 ch + 192) of the TMEM part, and 48
-      // of the shared-memory part (K 384 + 48 qi ..), qi = 2 half + ch.
+      // This thread's Q values, read from the staging areas (64 head rows, 64-value
+      // chunks of 128-byte rows, 128-byte swizzle): K [192 ch, 192 ch + 192) of the
+      // TMEM part (chunks 3 ch .. 3 ch + 2, in the value ring), and 48 of the
+      // shared-memory part (K 384 + 48 qi .., chunks 6..8), qi = 2 half + ch.
       const int qi = 2 * half + ch;
-      const uint4* qt = reinterpret_cast<const uint4*>(p.q_lat + qr * kDc + 192 * ch);
-      auto q_smem_src = [&](int k) -> const uint4* {  // 8 values K = 384 + 48 qi + 8k ..
-        const int kv = 384 + 48 * qi + 8 * k;
-        return kv < kDc ? reinterpret_cast<const uint4*>(p.q_lat + qr * kDc + kv)
-                        : reinterpret_cast<const uint4*>(p.q_pe + qr * kDr + (kv - kDc));
+      auto q_unit = [&](int kv) -> uint32_t {  // 16-byte unit holding K values kv .. kv+7 of row m
+        const int c = kv >> 6, u = (kv & 63) >> 3;
+        const uint32_t base = c < 6 ? sa + kVOff + c * kQStChunk : sa + kQStOff + (c - 6) * kQStChunk;
+        return base + m * 128 + ((u ^ (m & 7)) << 4);
       };
       auto absmax8 = [](const uint4 v) {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -446,15 +475,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 4; ++e) a = fmaxf(a, fmaxf(fabsf(bf16_lo(w[e])), fabsf(bf16_hi(w[e]))));
         return a;
       };
-      // pass 1: the largest magnitude of this thread's values (they are read again
-      // below; Q is small and stays in L2)
+      mbar_wait(own_bar(Q_STAGE), 0, abort_flag, p.status, wait_ns);
+      __syncwarp();
+      // pass 1: the largest magnitude of this thread's values (rows past H are zeros)
       float amax = 0.f;
-      if (row_ok) {
-#pragma unroll 4
-        for (int k = 0; k < 24; ++k) amax = fmaxf(amax, absmax8(__ldg(qt + k)));
+#pragma unroll 8
+      for (int k = 0; k < 24; ++k) amax = fmaxf(amax, absmax8(lds128(q_unit(192 * ch + 8 * k))));
 #pragma unroll
-        for (int k = 0; k < 6; ++k) amax = fmaxf(amax, absmax8(__ldg(q_smem_src(k))));
-      }
+      for (int k = 0; k < 6; ++k) amax = fmaxf(amax, absmax8(lds128(q_unit(384 + 48 * qi + 8 * k))));
       // the row's maximum over its four threads
       xmax[ch * 128 + lt] = amax;
       named_bar_sync(grp_bar, 128);
@@ -468,7 +496,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int grp = 0; grp < 3; ++grp) {
         uint4 raw[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) raw[k] = row_ok ? __ldg(qt + 8 * grp + k) : make_uint4(0u, 0u, 0u, 0u);
+        for (int k = 0; k < 8; ++k) raw[k] = lds128(q_unit(192 * ch + 64 * grp + 8 * k));
         uint32_t hi[16], lo[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
@@ -485,8 +513,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // shared-memory part: 48 values = three 16-byte units per term
 #pragma unroll 1
       for (int k = 0; k < 3; ++k) {
-        const uint4 raw2[2] = {row_ok ? __ldg(q_smem_src(2 * k)) : make_uint4(0u, 0u, 0u, 0u),
-                               row_ok ? __ldg(q_smem_src(2 * k + 1)) : make_uint4(0u, 0u, 0u, 0u)};
+        const uint4 raw2[2] = {lds128(q_unit(384 + 48 * qi + 16 * k)), lds128(q_unit(384 + 48 * qi + 16 * k + 8))};
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
@@ -501,7 +528,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         sts128(sa + kQOff + (0 * kQSmemChunks + cs) * kQChunk + off, make_uint4(hi[0], hi[1], hi[2], hi[3]));
         sts128(sa + kQOff + (1 * kQSmemChunks + cs) * kQChunk + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
       }
+      // the staging areas have been read: the value ring may take its first stage
       fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_local(own_bar(Q_FREE));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -740,6 +770,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int u = max(0, ns_own - kScRing); u < ns_own; ++u)
       mbar_wait(own_bar(SC_FULL + u % kScRing), (u / kScRing) & 1, &give_up, nullptr, kDrainLimitNs);
     if (issued[2]) mbar_wait(own_bar(RAW_V + (n - 1) % kVStages), 0, &give_up, nullptr, kDrainLimitNs);
+    if (issued[3]) mbar_wait(own_bar(Q_STAGE), 0, &give_up, nullptr, kDrainLimitNs);
   }
   cluster_arrive();
   cluster_wait();
@@ -749,9 +780,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_decode_f8(const mla_decode_args_t* a, int splits, cudaStream_t stream) {
-  CUtensorMap tm_ks, tm_kv, tm_o;
+  CUtensorMap tm_ks, tm_kv, tm_o, tm_q, tm_qpe;
   const uint64_t rows_kv = (uint64_t)a->num_pages * kPage;
   const int n_tok = a->B * a->s_q;
+  // query maps (values, heads, tokens), boxes of 64 values x 64 heads x 1 token:
+  // a box past H reads zeros
+  if (!tma_map_3d(&tm_q, a->q_lat, kDc, a->H, n_tok, kDc * 2, (uint64_t)a->H * kDc * 2, 64, 64, 1) ||
+      !tma_map_3d(&tm_qpe, a->q_pe, kDr, a->H, n_tok, kDr * 2, (uint64_t)a->H * kDr * 2, 64, 64, 1))
+    return cudaErrorInvalidValue;
   // score operand: (64 codes, rows, 9 chunks 64 bytes apart), 64-byte swizzle;
   // value operand: (128 codes, rows, column group 128 bytes apart, N tile 256
   // bytes apart), 128-byte swizzle
@@ -791,7 +827,8 @@ cudaError_t launch_decode_f8(const mla_decode_args_t* a, int splits, cudaStream_
   });
   if (e != cudaSuccess) return e;
   dim3 grid(2 * splits, a->s_q, a->B);
-  return launch_pdl(decode_f8_kernel, grid, dim3(kThreads), kSmemBytes, stream, tm_ks, tm_kv, tm_o, p);
+  return launch_pdl(decode_f8_kernel, grid, dim3(kThreads), kSmemBytes, stream, tm_ks, tm_kv, tm_o, tm_q, tm_qpe,
+                    p);
 }
 
 }  // namespace mla
