@@ -48,12 +48,17 @@
 //
 // q8_0 cache (ik_llama.cpp docs "FlashMLA", section "KV cache with MLA": int8
 // codes with one fp16 scale per 32 values): the same MMAs on bf16 operands.  The
-// producer brings the raw codes (and their block scales) into the back half of
-// the score and value slots; four converter warps (12..15, 512 threads in all)
-// read a slot's raw bytes into registers, meet at a named barrier, and write the
-// values code * scale (fp32 product, exact, rounded once to bf16) over the whole
-// slot in the layout TMA gives a bf16 cache, zeros for rows past the sequence
-// end; then they arrive on the even CTA's full barrier of that slot.
+// producer brings the CTA's raw codes (and their block scales) into the back half
+// of its score slot; four converter warps (12..15, 512 threads in all) read them
+// into registers, meet at a named barrier, and write the values code * scale
+// (fp32 product, exact, rounded once to bf16) over the whole slot in the layout
+// TMA gives a bf16 cache, zeros for rows past the sequence end; then they arrive
+// on the even CTA's full barrier of that slot.  The value operand is not
+// converted again: the converted latent chunks of the CTA's 32 rows go by eight
+// 4 KB shared-memory bulk copies into rows 32r .. 32r+31 of the value slot of the
+// CTA that holds their columns (four to itself, four to the peer; the 128-byte
+// swizzle depends on the row mod 8 only, so the layout survives the move), and a
+// converter thread relays the landing of its CTA's value slot to the even CTA.
 //
 // Every mbarrier wait is bounded (MLA_ERR_DEVICE_TIMEOUT in the status word);
 // after one runs out every role leaves its loop, issued MMAs are drained, the
@@ -118,8 +123,9 @@ constexpr int RAW_V = S_FREE + 2;         // [kVStages] a last page's value stag
 constexpr int Q_STAGE = RAW_V + kVStages; // Q chunks 0..5 landed in the value ring (this CTA)
 constexpr int Q_MOVED = Q_STAGE + 1;      // the softmax warps have moved them into TMEM
 constexpr int RAW_QS = Q_MOVED + 1;       // [kSStages] q8_0: raw codes of a score slot landed (this CTA)
-constexpr int RAW_QV = RAW_QS + kSStages; // [kVStages] q8_0: raw codes of a value slot landed (this CTA)
-constexpr int NBARS = RAW_QV + kVStages;
+constexpr int VQ_LAND = RAW_QS + kSStages; // [kVStages] q8_0: both CTAs' copies into this value slot landed
+constexpr int SRC_FREE = VQ_LAND + kVStages;  // [kSStages] q8_0: the copies out of this score slot are done
+constexpr int NBARS = SRC_FREE + kSStages;
 constexpr int kSoftmaxWarps = 8;          // warps 4..11: two per TMEM lane quadrant
 constexpr int kPrefetchTiles = MLA_TC_PREFETCH;      // L2 prefetch distance of the cache stream
 constexpr uint32_t kMiscOff = kBarOff + 8 * NBARS;
@@ -128,19 +134,17 @@ constexpr uint32_t kXlOff = kXmaxOff + 4 * 128 * 4;  // float [2][128]
 constexpr uint32_t kSmemUsed = kXlOff + 2 * 128 * 4;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;    // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-// q8_0: fp16 block scales beside the rings: 32 rows x 18 per score slot, 64 rows
-// x 18 per value slot; raw codes in the back half of each slot
+// q8_0: fp16 block scales beside the ring (32 rows x 18 per score slot); raw
+// codes in the back half of each score slot
 constexpr uint32_t kQ8RowBytes = kRow;                  // 576 int8 codes
 constexpr uint32_t kQ8ScRow = 18 * 2;                   // 36 bytes of scales per row
 constexpr uint32_t kQ8RawS = 32 * kQ8RowBytes;          // 18432: the CTA's 32 rows
-constexpr uint32_t kQ8RawV = 2 * 64 * 128;              // 16384: 64 rows x the CTA's 256 latent columns
 constexpr uint32_t kQ8ScS = 32 * kQ8ScRow;              // 1152
-constexpr uint32_t kQ8ScV = 64 * kQ8ScRow;              // 2304
-constexpr uint32_t kQ8ScOff = kSmemUsed;
-constexpr uint32_t kQ8ScVOff = kQ8ScOff + kSStages * kQ8ScS;
-constexpr uint32_t kSmemBytesQ8 = kQ8ScVOff + kVStages * kQ8ScV + 1024;
+constexpr uint32_t kQ8ScOff = (kSmemUsed + 127) / 128 * 128;  // bulk-copy destination: 16-byte aligned
+constexpr uint32_t kSmemBytesQ8 = kQ8ScOff + kSStages * kQ8ScS + 1024;
 static_assert(kSmemBytesQ8 <= 232448, "shared memory budget (q8_0)");
-static_assert(kSStage == 2 * kQ8RawS && kVStage == 2 * kQ8RawV, "raw codes fill the back half of a slot");
+static_assert(kQ8ScOff % 16 == 0 && kQ8ScS % 16 == 0, "bulk copies into the scale area start on 16 bytes");
+static_assert(kSStage == 2 * kQ8RawS, "raw codes fill the back half of a score slot");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 256;                     // S buffers at columns 256, 288
 constexpr uint32_t kTmemQ = 320;                     // Q chunks 0..5: columns 320..511 (2 bf16 each)
@@ -220,16 +224,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
       mbar_init(own_bar(S_EMPTY + i), 1);
       mbar_init(own_bar(RAW_QS + i), 1);
     }
+    // (a full value stage: two arrivals either way; q8_0: one relay per CTA)
     for (int i = 0; i < kVStages; ++i) {
-      mbar_init(own_bar(V_FULL + i), Q8 ? 2 * kConvWarps : 2);
+      mbar_init(own_bar(V_FULL + i), 2);
       mbar_init(own_bar(V_EMPTY + i), 1);
       mbar_init(own_bar(RAW_V + i), 1);
-      mbar_init(own_bar(RAW_QV + i), 1);
+      mbar_init(own_bar(VQ_LAND + i), 1);
     }
+    for (int i = 0; i < kSStages; ++i) mbar_init(own_bar(SRC_FREE + i), 1);
     mbar_init(own_bar(Q_TMEM), 2 * kSoftmaxWarps);
     mbar_init(own_bar(Q_FULL), 1);
     mbar_init(own_bar(Q_STAGE), 1);
-    mbar_init(own_bar(Q_MOVED), kSoftmaxWarps);
+    // q8_0: the value ring of either CTA takes copies from both, so Q must have
+    // left the ring in both CTAs
+    mbar_init(own_bar(Q_MOVED), Q8 ? 2 * kSoftmaxWarps : kSoftmaxWarps);
     for (int i = 0; i < 2; ++i) {
       mbar_init(own_bar(S_READY + i), 1);
       mbar_init(own_bar(P_READY + i), 2 * kSoftmaxWarps);
@@ -301,7 +309,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
         const uint32_t dst = sa + kSOff + st * kSStage;
         if constexpr (Q8) {
           // the CTA's 32 rows of codes (contiguous) into the back half of the slot,
-          // their block scales beside the ring; the converters take it from there
+          // their block scales beside the ring; the converters take it from there.
+          // The slot's last page must also have been copied out to the value slots.
+          if (!mbar_wait_converged(own_bar(SRC_FREE + st), ph, abort_flag, p.status, wait_ns)) return false;
           if (lane == 0) {
             const size_t row0 = (size_t)pg * kPage + 32 * r;
             mbar_arrive_expect_tx_local(own_bar(RAW_QS + st), kQ8RawS + kQ8ScS);
@@ -323,27 +333,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
         return true;
       };
       auto load_v = [&](int u) -> bool {
+        if constexpr (Q8) {
+          // the value slots are filled by the converters' copies
+          n_v = u + 1;
+          return true;
+        }
         const int st = u % kVStages;
         const uint32_t ph = ((u / kVStages) & 1) ^ 1;
         if (!mbar_wait_converged(own_bar(V_EMPTY + st), ph, abort_flag, p.status, wait_ns)) return false;
         const int pg = page_of(u, blk_v, pg_v);
         const uint32_t dst = sa + kVOff + st * kVStage;
-        if constexpr (Q8) {
-          // the page's 64 rows x the CTA's latent columns 128r .. +127 and
-          // 256 + 128r .. +127 (two boxes of 64 rows x 128 codes) into the back
-          // half of the slot, the page's block scales beside the ring
-          if (lane == 0) {
-            mbar_arrive_expect_tx_local(own_bar(RAW_QV + st), kQ8RawV + kQ8ScV);
-            tma_load_2d_cta(dst + kQ8RawV, &tm_kv, own_bar(RAW_QV + st), 128 * (int)r, pg * kPage);
-            tma_load_2d_cta(dst + kQ8RawV + kQ8RawV / 2, &tm_kv, own_bar(RAW_QV + st), 256 + 128 * (int)r,
-                            pg * kPage);
-            bulk_load_cta(sa + kQ8ScVOff + st * kQ8ScV, p.kv_scale + (size_t)pg * kPage * kQ8ScRow, kQ8ScV,
-                          own_bar(RAW_QV + st));
-          }
-          __syncwarp();
-          n_v = u + 1;
-          return true;
-        }
         const int nvalid = j_end - (t0 + u) * kPage;  // cached rows of this page inside the sequence
         if (nvalid >= kPage) {
           // one box: (64 values, 64 rows, chunks 2r and 2r+1, groups 0 and 1): latent
@@ -412,14 +411,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
       if (ok && n > 1) ok = load_s(1);
       for (int u = 0; ok && u < n; ++u) {
         if (u + 2 < n) ok = load_s(u + 2);
-        if (u == 0 && ok) ok = mbar_wait_converged(own_bar(Q_MOVED), 0, abort_flag, p.status, wait_ns);
+        if (!Q8 && u == 0 && ok) ok = mbar_wait_converged(own_bar(Q_MOVED), 0, abort_flag, p.status, wait_ns);
         if (ok) ok = load_v(u);
       }
     }
     if (lane == 0) {
       issued[0] = n_s;
       issued[1] = n_v;
-      issued[2] = v_part;
+      if (!Q8) issued[2] = v_part;  // q8_0: the converters' copy count
       issued[3] = q_iss;
     }
   } else if (warp >= 1 && warp <= 3) {
@@ -481,6 +480,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
           if (!mbar_wait_converged<Q8>(own_bar(V_FULL + st), (t / kVStages) & 1, abort_flag, p.status, wait_ns))
             break;
           tc_fence_after();
+          if constexpr (Q8) {
+            // every copy out of page t's score slots has landed: both producers may
+            // refill them (once the score MMAs are done with them too)
+            if (lane == 0) {
+              mbar_arrive_remote(own_bar(SRC_FREE + t % kSStages));
+              mbar_arrive_remote(mapa(own_bar(SRC_FREE + t % kSStages), 1));
+            }
+          }
           const uint64_t ap = dp + ((pb * kPBytes) >> 4);
           const uint64_t bv = dv + ((st * kVStage) >> 4);
 #pragma unroll
@@ -545,6 +552,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
       if (lane == 0) {
         mbar_arrive_remote(lead_bar(Q_TMEM));
         mbar_arrive_remote(own_bar(Q_MOVED));
+        if (Q8) mbar_arrive_remote(mapa(own_bar(Q_MOVED), r ^ 1));
       }
     }
     float m_used = -CUDART_INF_F, l = 0.f;
@@ -724,7 +732,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
     // outcome of each wait is combined over the group first.
     const int ct = threadIdx.x - kThreads;  // 0 .. 127
     const __half* scs = reinterpret_cast<const __half*>(sm + kQ8ScOff);
-    const __half* scv = reinterpret_cast<const __half*>(sm + kQ8ScVOff);
     auto conv_s = [&](int u) -> bool {
       const int tok0 = (t0 + u) * kPage;  // first token of the page
       {
@@ -758,52 +765,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive_remote_release_cluster(lead_bar(S_FULL + st));
-      }
-      return true;
-    };
-    auto conv_v = [&](int u) -> bool {
-      const int tok0 = (t0 + u) * kPage;  // first token of the page
-      {
-        const int st = u % kVStages;
-        const bool got = mbar_wait_converged(own_bar(RAW_QV + st), (u / kVStages) & 1, abort_flag, p.status, wait_ns);
-        if (!named_bar_and(6, 32 * kConvWarps, got)) return false;
-        const uint32_t slot = sa + kVOff + st * kVStage;
-        uint4 raw[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) raw[i] = lds128(slot + kQ8RawV + 16 * (ct + 128 * i));
+        // every converter warp's stores are visible to the bulk copies below
         named_bar_sync(6, 32 * kConvWarps);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          // box nb (latent columns 128r.. or 256 + 128r..), row, 16 codes from column 16 c16
-          const int q = ct + 128 * i, nb = q >> 9, row = (q >> 3) & 63, c16 = q & 7;
-          const int col = 256 * nb + 128 * (int)r + 16 * c16;
-          const bool live = tok0 + row < j_end;
-          const float d = live ? __half2float(scv[(st * 64 + row) * 18 + (col >> 5)]) : 0.f;
-          const uint32_t w[4] = {raw[i].x ^ 0x80808080u, raw[i].y ^ 0x80808080u, raw[i].z ^ 0x80808080u,
-                                 raw[i].w ^ 0x80808080u};
-          uint32_t o[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            o[k] = pack_bf16(q8_code(w[k >> 1], 2 * (k & 1)) * d, q8_code(w[k >> 1], 2 * (k & 1) + 1) * d);
-          const int j = 2 * nb + (c16 >> 2), unit = 2 * (c16 & 3);
-          const uint32_t base = slot + j * kChunkV + row * 128;
-          sts128(base + ((unit ^ (row & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
-          sts128(base + (((unit + 1) ^ (row & 7)) << 4), make_uint4(o[4], o[5], o[6], o[7]));
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote_release_cluster(lead_bar(V_FULL + st));
       }
       return true;
     };
-    // score slots one page ahead of value slots, in the order the producer
-    // requests them: the score MMA of page u + 1 never waits for the value
-    // conversion of page u, whose raw codes are requested later
+    // Warp 12 copies the converted latent chunks of page u out of the score slot:
+    // latent chunk c (32 rows x 128 bytes) of this CTA's rows goes to rows
+    // 32r .. 32r+31 of value chunk j of the CTA that holds chunk c's columns
+    // (chunks 0, 1, 4, 5 to the even CTA, 2, 3, 6, 7 to the odd one, j = 2 (c / 4)
+    // + c % 2), landing on that CTA's value-slot barrier.  A wait that gives up
+    // here sets the abort flag; the group leaves at its next reduction barrier.
+    int copied = 0;
+    auto copy_v = [&](int u) {
+      if (warp != 12) return;
+      const int vs = u % kVStages;
+      bool got = u > 0 || mbar_wait_converged<true>(own_bar(Q_MOVED), 0, abort_flag, p.status, wait_ns);
+      if (got) got = mbar_wait_converged(own_bar(V_EMPTY + vs), ((u / kVStages) & 1) ^ 1, abort_flag, p.status, wait_ns);
+      if (!got) return;
+      if (lane == 0) {
+        mbar_arrive_expect_tx_local(own_bar(VQ_LAND + vs), kVStage);  // 4 chunks from each CTA
+        const uint32_t src = sa + kSOff + (u % kSStages) * kSStage;
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t to = (c >> 1) & 1, j = 2 * (c >> 2) + (c & 1);
+          bulk_copy_s2s(mapa(sa + kVOff + vs * kVStage + j * kChunkV + 32 * r * 128, to), src + c * kChunkS,
+                        kChunkS, mapa(own_bar(VQ_LAND + vs), to));
+        }
+      }
+      __syncwarp();
+      copied = u + 1;
+    };
+    // ... and tells the even CTA once both CTAs' copies into this value slot landed
+    auto relay = [&](int u) {
+      if (warp != 12) return;
+      const int vs = u % kVStages;
+      if (!mbar_wait_converged<true>(own_bar(VQ_LAND + vs), (u / kVStages) & 1, abort_flag, p.status, wait_ns))
+        return;
+      if (lane == 0) mbar_arrive_remote_release_cluster(lead_bar(V_FULL + vs));
+    };
+    // score slots one page ahead of the value slots' relay; control flow stays
+    // uniform across the four warps (only conv_s ends the loop)
     bool ok = n > 0 ? conv_s(0) : true;
+    if (ok && n > 0) copy_v(0);
     for (int u = 0; ok && u < n; ++u) {
-      if (u + 1 < n) ok = conv_s(u + 1);
-      if (ok) ok = conv_v(u);
+      if (u + 1 < n) {
+        ok = conv_s(u + 1);
+        if (ok) copy_v(u + 1);
+      }
+      if (ok) relay(u);
     }
+    if (warp == 12 && lane == 0) issued[2] = copied;
   }
 
   // ---- teardown: both CTAs are done with TMEM and shared memory
@@ -829,11 +840,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
     if constexpr (Q8) {
       // q8_0: the raw codes of every slot land on this CTA's own barriers; the
       // full barriers count the converters' arrivals only (no bytes in flight)
-      const int ns = r == 0 ? ns0 : ns1, nv = r == 0 ? nv0 : nv1;
+      const int ns = r == 0 ? ns0 : ns1;
       for (int u = max(0, ns - kSStages); u < ns; ++u)
         mbar_wait(own_bar(RAW_QS + u % kSStages), (u / kSStages) & 1, &give_up, nullptr, kDrainLimitNs);
-      for (int u = max(0, nv - kVStages); u < nv; ++u)
-        mbar_wait(own_bar(RAW_QV + u % kVStages), (u / kVStages) & 1, &give_up, nullptr, kDrainLimitNs);
+      // copies into this CTA's value slots: for a page only one CTA copied, stand in
+      // for the other CTA's half (its arrival, or its 16 KB), then wait for the
+      // pages still open
+      const int own = (int)issued[2], peer = (int)ld_shared_cluster_u32(mapa(sa + kMiscOff + 16, r ^ 1));
+      for (int u = min(own, peer); u < max(own, peer); ++u) {
+        if (own > peer) mbar_complete_tx_local(own_bar(VQ_LAND + u % kVStages), kVStage / 2);
+        else mbar_arrive_expect_tx_local(own_bar(VQ_LAND + u % kVStages), kVStage / 2);
+      }
+      const int nc = max(own, peer);
+      for (int u = max(0, nc - kVStages); u < nc; ++u)
+        mbar_wait(own_bar(VQ_LAND + u % kVStages), (u / kVStages) & 1, &give_up, nullptr, kDrainLimitNs);
       if (r == 0 && issued[3]) mbar_wait(own_bar(Q_FULL), 0, &give_up, nullptr, kDrainLimitNs);
     } else if (r == 0) {
       for (int u = min(ns0, ns1); u < max(ns0, ns1); ++u) {
@@ -857,7 +877,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
       if (issued[3]) mbar_wait(own_bar(Q_FULL), 0, &give_up, nullptr, kDrainLimitNs);
     }
     if (issued[3]) mbar_wait(own_bar(Q_STAGE), 0, &give_up, nullptr, kDrainLimitNs);
-    if (issued[2]) mbar_wait(own_bar(RAW_V + (n - 1) % kVStages), 0, &give_up, nullptr, kDrainLimitNs);
+    if (!Q8 && issued[2]) mbar_wait(own_bar(RAW_V + (n - 1) % kVStages), 0, &give_up, nullptr, kDrainLimitNs);
   }
   cluster_arrive();
   cluster_wait();
@@ -879,8 +899,8 @@ cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t strea
   // apart), one box of 2 x 2 chunks per stage
   const bool q8 = a->kv_dtype == MLA_KV_Q8_0;
   if (q8) {
-    // q8_0: the value operand's raw codes, boxes of 64 rows x 128 codes (no
-    // swizzle); the score operand comes by bulk copies (tm_ks is not read)
+    // q8_0: the raw codes come by bulk copies and the value operand from the
+    // converted score slots; the cache maps are not read (any valid map will do)
     const uint64_t dq[2] = {kRow, rows_kv}, sq[1] = {kRow};
     const uint32_t bq[2] = {128, 64};
     if (!tma_map_nd(&tm_kv, a->kv_cache, 2, dq, sq, bq, true, 0)) return cudaErrorInvalidValue;
