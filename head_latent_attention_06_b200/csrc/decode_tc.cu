@@ -710,7 +710,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
         const int qtok = b * p.s_q + g;
         for (int c = 0; c < 8; ++c) tma_store_3d(&tm_o, sa + kSOff + c * (64 * 128), 64 * c, 64 * (int)r, qtok);
         bulk_commit_group();
-        bulk_wait_all();
+        bulk_wait_read<0>();  // the staging area may be released; the writes finish with the grid
       }
     }
     if (half == 0 && ch == 0 && row_ok) {

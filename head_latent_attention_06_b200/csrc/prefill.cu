@@ -19,7 +19,7 @@
 //            chunks of 64, accumulated in two TMEM accumulators (256 columns
 //            each).  Sharing the weight chunk between 256 tokens cuts the
 //            operand bytes per MMA by a third against one 128-token tile.
-//   attn:    FlashAttention forward per (sequence, head, 128 queries): S = Q K^T
+//   attn:    FlashAttention forward per (sequence, head, 2 x 128 queries): S = Q K^T
 //            with Q = [q_nope | q_pe] (192), K = [Kn | k_pe] (k_pe from the cache,
 //            shared by all heads), M = 128 queries, N = 128 keys; online softmax
 //            (exp2, lazy rescale of O by more than 2^8); O += P V with P in TMEM
@@ -194,28 +194,29 @@ __global__ void __launch_bounds__(kUpThreads, 1)
 }
 
 // ---------------------------------------------------------------- attention
-constexpr int kAtThreads = 256;             // warp 0 producer, warp 1 MMA, warps 4..7 softmax
+// One CTA per (sequence, head, 256 queries): two 128-query tiles A and B share
+// every K and V tile, each with its own softmax warpgroup, S (P) and O in TMEM,
+// so that the tensor pipe works on one tile while the other tile's softmax runs.
+constexpr int kAtThreads = 384;             // warp 0 producer, warp 1 MMA, warps 4..7 tile A, 8..11 tile B
 constexpr uint32_t kQChunk = 128 * 128;     // 128 rows x 64 bf16
-constexpr uint32_t kQBytes = 3 * kQChunk;   // q_nope (2 chunks) | q_pe
+constexpr uint32_t kQBytes = 3 * kQChunk;   // one tile's Q: q_nope (2 chunks) | q_pe
 constexpr uint32_t kKBytes = 3 * kQChunk;   // Kn (2 chunks) | k_pe (two pages)
 constexpr uint32_t kVBytes = 2 * kQChunk;   // V: 128 keys x 128 values, two 64-value chunks
-constexpr int kKvStages = 2;
-constexpr uint32_t kAtQOff = 0;
-constexpr uint32_t kAtKOff = kAtQOff + kQBytes;
-constexpr uint32_t kAtVOff = kAtKOff + kKvStages * kKBytes;
-constexpr uint32_t kAtBarOff = kAtVOff + kKvStages * kVBytes;
+constexpr int kVStagesAt = 2;
+constexpr uint32_t kAtQOff = 0;                              // Q of tiles A and B
+constexpr uint32_t kAtKOff = kAtQOff + 2 * kQBytes;          // one K stage
+constexpr uint32_t kAtVOff = kAtKOff + kKBytes;              // two V stages
+constexpr uint32_t kAtBarOff = kAtVOff + kVStagesAt * kVBytes;
 constexpr uint32_t kAtSmem = kAtBarOff + 256 + 1024;
 static_assert(kAtSmem <= 232448, "shared memory budget");
-// TMEM: three S / P buffers at columns 0, 128 and 256 (P, bf16, takes the first
-// 64 columns of its buffer), O at 384
-constexpr int kSBufs = 3;
-constexpr uint32_t kTmemO = 384;
+// TMEM: S (and P over it) of tile t at columns 128 t, O of tile t at 256 + 128 t
+constexpr uint32_t kTmemO = 256;
 constexpr uint32_t kAtIdescS = idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t kAtIdescPV = idesc_bf16_f32(128, 128, false, true);
 constexpr float kRescale = 8.0f;
-// barriers
-constexpr int A_Q = 0, A_KFULL = 1, A_KEMPTY = 3, A_VFULL = 5, A_VEMPTY = 7, A_SREADY = 9, A_PREADY = 12,
-              A_ODONE = 15, A_DRAIN = 18, A_NBARS = 19;
+// barriers ([2]: one per query tile or V stage)
+constexpr int A_Q = 0, A_KFULL = 1, A_KEMPTY = 2, A_VFULL = 3, A_VEMPTY = 5, A_SREADY = 7, A_PREADY = 9,
+              A_ODONE = 11, A_DRAIN = 13, A_NBARS = 14;
 
 struct AtParams {
   const __nv_bfloat16* kn;
@@ -250,11 +251,12 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   const int L_in = p.seq_lens[b];
   const bool bad_len = L_in < p.s_q || L_in > p.max_pages * kPage || L_in > p.max_len;
   const int L = bad_len ? 0 : L_in;
-  const int q0 = qt * 128;
-  const int nq = max(0, min(128, p.s_q - q0));  // query rows of this tile
-  // keys this tile's last query sees (causal) or all of them
+  const int q0 = qt * 256;                          // first query of tile A
+  const int nq = max(0, min(256, p.s_q - q0));      // query rows of the two tiles
+  // keys the CTA's last query sees (causal) or all of them; tile A runs the same
+  // tiles (its last ones fully masked under the causal rule)
   const int kmax = L == 0 ? 0 : (p.causal ? min(L, L - p.s_q + q0 + nq) : L);
-  const int n = (kmax + 127) / 128;
+  const int n = nq > 0 ? (kmax + 127) / 128 : 0;
   const uint64_t wait_ns = p.wait_ns;
 
   if (threadIdx.x == 0) {
@@ -262,13 +264,11 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     *abort_flag = 0;
     issued[0] = issued[1] = 0;
     mbar_init(bar(A_Q), 1);
+    mbar_init(bar(A_KFULL), 1);
+    mbar_init(bar(A_KEMPTY), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(A_KFULL + i), 1);
-      mbar_init(bar(A_KEMPTY + i), 1);
       mbar_init(bar(A_VFULL + i), 1);
       mbar_init(bar(A_VEMPTY + i), 1);
-    }
-    for (int i = 0; i < kSBufs; ++i) {
       mbar_init(bar(A_SREADY + i), 1);
       mbar_init(bar(A_PREADY + i), 4);
       mbar_init(bar(A_ODONE + i), 1);
@@ -287,16 +287,20 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   if (warp == 0) {
     // =========================== TMA producer ===========================
     int n_k = 0, n_v = 0;
-    if (n > 0 && nq > 0) {
+    if (n > 0) {
       const int32_t* bt = p.block_table + (size_t)b * p.max_pages;
       const size_t kv_row0 = ((size_t)b * p.H + h) * p.Lmax;
       if (lane == 0) {
-        // Q: 128 query rows (rows past s_q read as zeros), q_nope in two chunks, q_pe
+        // Q of both tiles: 256 query rows (rows past s_q read as zeros or belong to
+        // the next sequence; their outputs are not stored)
         const int tok = b * p.s_q + q0;
-        mbar_arrive_expect_tx_local(bar(A_Q), kQBytes);
-        tma_load_3d_cta(sa + kAtQOff, &tm_qn, bar(A_Q), 0, h, tok);
-        tma_load_3d_cta(sa + kAtQOff + kQChunk, &tm_qn, bar(A_Q), 64, h, tok);
-        tma_load_3d_cta(sa + kAtQOff + 2 * kQChunk, &tm_qp, bar(A_Q), 0, h, tok);
+        mbar_arrive_expect_tx_local(bar(A_Q), 2 * kQBytes);
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t dq = sa + kAtQOff + t * kQBytes;
+          tma_load_3d_cta(dq, &tm_qn, bar(A_Q), 0, h, tok + 128 * t);
+          tma_load_3d_cta(dq + kQChunk, &tm_qn, bar(A_Q), 64, h, tok + 128 * t);
+          tma_load_3d_cta(dq + 2 * kQChunk, &tm_qp, bar(A_Q), 0, h, tok + 128 * t);
+        }
       }
       auto page = [&](int idx) {
         int v = idx < p.max_pages ? bt[idx] : 0;
@@ -305,31 +309,32 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       };
       bool ok = true;
       for (int j = 0; ok && j < n; ++j) {
-        const int st = j & 1;
-        // K: Kn rows of keys 128 j .. (tokens past the length read whatever the
-        // workspace holds: their scores are masked), k_pe of the two pages
-        ok = mbar_wait_converged(bar(A_KEMPTY + st), ((j >> 1) & 1) ^ 1, abort_flag, p.status, wait_ns);
+        // V(j) into its stage once P.V(j-2) is done, then K(j) into the one K stage
+        // once both score MMAs of tile j-1 are done
+        const int vs = j & 1;
+        ok = mbar_wait_converged(bar(A_VEMPTY + vs), ((j >> 1) & 1) ^ 1, abort_flag, p.status, wait_ns);
         if (!ok) break;
         if (lane == 0) {
-          const uint32_t dst = sa + kAtKOff + st * kKBytes;
-          mbar_arrive_expect_tx_local(bar(A_KFULL + st), kKBytes);
-          tma_load_2d_cta(dst, &tm_kn, bar(A_KFULL + st), 0, (int)(kv_row0 + 128 * j));
-          tma_load_2d_cta(dst + kQChunk, &tm_kn, bar(A_KFULL + st), 64, (int)(kv_row0 + 128 * j));
-          tma_load_2d_cta(dst + 2 * kQChunk, &tm_kpe, bar(A_KFULL + st), kDc, page(2 * j) * kPage);
-          tma_load_2d_cta(dst + 2 * kQChunk + 64 * 128, &tm_kpe, bar(A_KFULL + st), kDc, page(2 * j + 1) * kPage);
-        }
-        __syncwarp();
-        n_k = j + 1;
-        ok = mbar_wait_converged(bar(A_VEMPTY + st), ((j >> 1) & 1) ^ 1, abort_flag, p.status, wait_ns);
-        if (!ok) break;
-        if (lane == 0) {
-          const uint32_t dst = sa + kAtVOff + st * kVBytes;
-          mbar_arrive_expect_tx_local(bar(A_VFULL + st), kVBytes);
-          tma_load_2d_cta(dst, &tm_v, bar(A_VFULL + st), 0, (int)(kv_row0 + 128 * j));
-          tma_load_2d_cta(dst + kQChunk, &tm_v, bar(A_VFULL + st), 64, (int)(kv_row0 + 128 * j));
+          const uint32_t dst = sa + kAtVOff + vs * kVBytes;
+          mbar_arrive_expect_tx_local(bar(A_VFULL + vs), kVBytes);
+          tma_load_2d_cta(dst, &tm_v, bar(A_VFULL + vs), 0, (int)(kv_row0 + 128 * j));
+          tma_load_2d_cta(dst + kQChunk, &tm_v, bar(A_VFULL + vs), 64, (int)(kv_row0 + 128 * j));
         }
         __syncwarp();
         n_v = j + 1;
+        ok = mbar_wait_converged(bar(A_KEMPTY), (j & 1) ^ 1, abort_flag, p.status, wait_ns);
+        if (!ok) break;
+        if (lane == 0) {
+          // K: Kn rows of keys 128 j .. (rows past the length are zeros), k_pe of the two pages
+          const uint32_t dst = sa + kAtKOff;
+          mbar_arrive_expect_tx_local(bar(A_KFULL), kKBytes);
+          tma_load_2d_cta(dst, &tm_kn, bar(A_KFULL), 0, (int)(kv_row0 + 128 * j));
+          tma_load_2d_cta(dst + kQChunk, &tm_kn, bar(A_KFULL), 64, (int)(kv_row0 + 128 * j));
+          tma_load_2d_cta(dst + 2 * kQChunk, &tm_kpe, bar(A_KFULL), kDc, page(2 * j) * kPage);
+          tma_load_2d_cta(dst + 2 * kQChunk + 64 * 128, &tm_kpe, bar(A_KFULL), kDc, page(2 * j + 1) * kPage);
+        }
+        __syncwarp();
+        n_k = j + 1;
       }
     }
     if (lane == 0) {
@@ -338,47 +343,54 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     }
   } else if (warp == 1) {
     // =========================== MMA issue ===========================
-    if (n > 0 && nq > 0) {
-      const uint64_t dq = desc_sw128(sa + kAtQOff, 16, 1024);
+    // Per K/V tile j: P.V of tile A, then of tile B; then the scores of tile j + 1
+    // for A and for B, each once P.V(j) of that tile has read its P out of the S
+    // columns the new scores overwrite.
+    if (n > 0) {
       bool ok = mbar_wait_converged(bar(A_Q), 0, abort_flag, p.status, wait_ns);
-      // S(j) = Q K(j)^T into S buffer j % 3
-      auto issue_s = [&](int j) -> bool {
-        const int st = j & 1, sb = j % kSBufs;
-        if (!mbar_wait_converged(bar(A_KFULL + st), (j >> 1) & 1, abort_flag, p.status, wait_ns)) return false;
-        tc_fence_after();
-        const uint64_t dk = desc_sw128(sa + kAtKOff + st * kKBytes, 16, 1024);
+      // S_t(j) = Q_t K(j)^T into S columns of tile t; after both tiles, K is free
+      auto issue_s = [&](int t, int j) -> bool {
+        if (t == 0) {
+          if (!mbar_wait_converged(bar(A_KFULL), j & 1, abort_flag, p.status, wait_ns)) return false;
+          tc_fence_after();
+        }
+        const uint64_t dq = desc_sw128(sa + kAtQOff + t * kQBytes, 16, 1024);
+        const uint64_t dk = desc_sw128(sa + kAtKOff, 16, 1024);
 #pragma unroll
         for (int c = 0; c < 3; ++c)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_1_elect(tmem + 128u * sb, dq + ((c * kQChunk) >> 4) + 2 * kk, dk + ((c * kQChunk) >> 4) + 2 * kk,
+            mma_1_elect(tmem + 128u * t, dq + ((c * kQChunk) >> 4) + 2 * kk, dk + ((c * kQChunk) >> 4) + 2 * kk,
                         kAtIdescS, (c | kk) != 0);
-        commit_1_elect(bar(A_KEMPTY + st));
-        commit_1_elect(bar(A_SREADY + sb));
+        commit_1_elect(bar(A_SREADY + t));
+        if (t == 1) commit_1_elect(bar(A_KEMPTY));
         return true;
       };
-      if (ok) ok = issue_s(0);
-      if (ok && n > 1) ok = issue_s(1);
+      if (ok) ok = issue_s(0, 0);
+      if (ok) ok = issue_s(1, 0);
       for (int j = 0; ok && j < n; ++j) {
-        const int st = j & 1, sb = j % kSBufs, ph = (j / kSBufs) & 1;
-        // P(j) written over S(j) in TMEM by the softmax threads
-        if (!mbar_wait_converged(bar(A_PREADY + sb), ph, abort_flag, p.status, wait_ns)) break;
-        if (!mbar_wait_converged(bar(A_VFULL + st), (j >> 1) & 1, abort_flag, p.status, wait_ns)) break;
-        tc_fence_after();
-        const uint64_t dv = desc_sw128(sa + kAtVOff + st * kVBytes, kQChunk, 1024);
-        // K = 128 keys in steps of 16: P columns 8 kk (2 bf16 each), V rows 16 kk
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_1_ts_elect(tmem + kTmemO, tmem + 128u * sb + 8u * kk, dv + ((kk * 2048) >> 4), kAtIdescPV,
-                         (j > 0 || kk > 0) ? 1u : 0u);
-        commit_1_elect(bar(A_VEMPTY + st));
-        commit_1_elect(bar(A_ODONE + sb));
-        // S(j + 2) goes where P(j - 1) was: only once P.V(j - 1) has read it
-        if (j + 2 < n) {
-          if (j >= 1 && !mbar_wait_converged(bar(A_ODONE + (j - 1) % kSBufs), ((j - 1) / kSBufs) & 1, abort_flag,
-                                             p.status, wait_ns))
+        const int vs = j & 1;
+        for (int t = 0; ok && t < 2; ++t) {
+          if (!mbar_wait_converged(bar(A_PREADY + t), j & 1, abort_flag, p.status, wait_ns)) { ok = false; break; }
+          if (t == 0 && !mbar_wait_converged(bar(A_VFULL + vs), (j >> 1) & 1, abort_flag, p.status, wait_ns)) {
+            ok = false;
             break;
-          if (!issue_s(j + 2)) break;
+          }
+          tc_fence_after();
+          const uint64_t dv = desc_sw128(sa + kAtVOff + vs * kVBytes, kQChunk, 1024);
+          // K = 128 keys in steps of 16: P columns 8 kk (2 bf16 each), V rows 16 kk
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_1_ts_elect(tmem + kTmemO + 128u * t, tmem + 128u * t + 8u * kk, dv + ((kk * 2048) >> 4),
+                           kAtIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          commit_1_elect(bar(A_ODONE + t));
+          if (t == 1) commit_1_elect(bar(A_VEMPTY + vs));
+        }
+        if (ok && j + 1 < n) {
+          for (int t = 0; ok && t < 2; ++t) {
+            if (!mbar_wait_converged(bar(A_ODONE + t), j & 1, abort_flag, p.status, wait_ns)) { ok = false; break; }
+            ok = issue_s(t, j + 1);
+          }
         }
       }
       commit_1_elect(bar(A_DRAIN));
@@ -386,20 +398,23 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       mbar_wait_converged(bar(A_DRAIN), 0, &keep, p.status, kDrainNs);
     }
   } else if (warp >= 4) {
-    // ====================== softmax / epilogue: thread = query row ======================
-    const int row = 32 * (warp - 4) + lane;  // TMEM lane of this thread's query row
-    const uint32_t tl = tmem + ((uint32_t)(32 * (warp - 4)) << 16);
-    const int qi = q0 + row;                 // query index in the chunk
+    // ================ softmax / epilogue: thread = query row of tile t ================
+    // S_t(j) is issued only after P.V_t(j-1) has completed, so O_t may be rescaled
+    // as soon as the scores of tile j are there.
+    const int t = (warp - 4) >> 2;
+    const int row = 32 * (warp & 3) + lane;  // TMEM lane of this thread's query row
+    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    const uint32_t cs = 128u * t, co = kTmemO + 128u * t;
+    const int qi = q0 + 128 * t + row;       // query index in the chunk
     const int vis = p.causal ? L - p.s_q + qi + 1 : L;  // keys this query sees
     float m_used = -CUDART_INF_F, l = 0.f;
-    for (int j = 0; j < n && nq > 0; ++j) {
-      const int sb = j % kSBufs;
-      if (!mbar_wait_converged(bar(A_SREADY + sb), (j / kSBufs) & 1, abort_flag, p.status, wait_ns)) break;
+    for (int j = 0; j < n; ++j) {
+      if (!mbar_wait_converged(bar(A_SREADY + t), j & 1, abort_flag, p.status, wait_ns)) break;
       tc_fence_after();
       // the row's 128 raw scores: four loads in flight, one wait
       uint32_t sr[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tl + 128u * sb + 32u * c, sr[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld32(tl + cs + 32u * c, sr[c]);
       tmem_wait_ld();
       const int nv = max(0, min(128, vis - 128 * j));  // visible keys of this tile
       float s[128];
@@ -428,20 +443,15 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         }
       }
       const float nref = m_used == -CUDART_INF_F ? 0.f : -m_used;
-      // O of this row may be rescaled only once P.V(j-1) has accumulated into it
       if (__any_sync(0xffffffffu, resc) && j >= 1) {
-        if (!mbar_wait_converged(bar(A_ODONE + (j - 1) % kSBufs), ((j - 1) / kSBufs) & 1, abort_flag, p.status,
-                                 wait_ns))
-          break;
-        tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
-          tmem_ld32(tl + kTmemO + 32u * c, o);
+          tmem_ld32(tl + co + 32u * c, o);
           tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st32(tl + kTmemO + 32u * c, o);
+          tmem_st32(tl + co + 32u * c, o);
         }
         tmem_wait_st();
       }
@@ -457,17 +467,17 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           l4[k & 3] += p0 + p1;
           pk[k] = pack_bf16(p0, p1);
         }
-        tmem_st32(tl + 128u * sb + 32u * c, pk);
+        tmem_st32(tl + cs + 32u * c, pk);
       }
       l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_local(bar(A_PREADY + sb));
+      if (lane == 0) mbar_arrive_local(bar(A_PREADY + t));
     }
     // ---- epilogue: o = O / l, lse
-    if (n > 0 && nq > 0) {
-      mbar_wait_converged(bar(A_ODONE + (n - 1) % kSBufs), ((n - 1) / kSBufs) & 1, abort_flag, p.status, wait_ns);
+    if (n > 0) {
+      mbar_wait_converged(bar(A_ODONE + t), (n - 1) & 1, abort_flag, p.status, wait_ns);
       tc_fence_after();
     }
     const bool alive = __shfl_sync(0xffffffffu, *abort_flag, 0) == 0;
@@ -475,7 +485,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     const float inv = empty ? 0.f : 1.f / l;
     // tcgen05.ld is a warp-collective instruction: every lane loads (the
     // condition is warp-uniform), only the rows of real queries are stored
-    const bool live = n > 0 && nq > 0 && alive;
+    const bool live = n > 0 && alive;
     const bool mine = qi < p.s_q && nq > 0;
     const size_t orow = ((size_t)b * p.s_q + qi) * p.H + h;
     __nv_bfloat16* dst = p.out + orow * kDv;
@@ -483,7 +493,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     for (int c = 0; c < 4; ++c) {
       uint32_t o[32];
       if (live) {
-        tmem_ld32(tl + kTmemO + 32u * c, o);
+        tmem_ld32(tl + co + 32u * c, o);
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -505,12 +515,11 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) {
-    // a wait that ran out may leave loads in flight: wait (bounded) for the last
-    // load of each stage and for Q
+    // a wait that ran out may leave loads in flight: wait (bounded) for Q and for
+    // the last load of each ring
     int give_up = 0;
-    if (n > 0 && nq > 0) mbar_wait(bar(A_Q), 0, &give_up, nullptr, kDrainNs);
-    for (int j = max(0, (int)issued[0] - 2); j < (int)issued[0]; ++j)
-      mbar_wait(bar(A_KFULL + (j & 1)), (j >> 1) & 1, &give_up, nullptr, kDrainNs);
+    if (n > 0) mbar_wait(bar(A_Q), 0, &give_up, nullptr, kDrainNs);
+    if (issued[0] > 0) mbar_wait(bar(A_KFULL), (issued[0] - 1) & 1, &give_up, nullptr, kDrainNs);
     for (int j = max(0, (int)issued[1] - 2); j < (int)issued[1]; ++j)
       mbar_wait(bar(A_VFULL + (j & 1)), (j >> 1) & 1, &give_up, nullptr, kDrainNs);
   }
@@ -586,7 +595,7 @@ cudaError_t launch_prefill(const mla_prefill_args_t* a, cudaStream_t stream) {
   at.causal = a->causal;
   at.scale_log2 = a->softmax_scale * kLog2e;
   at.wait_ns = device_wait_limit_ns();
-  return launch_pdl(prefill_attn_kernel, dim3((a->s_q + 127) / 128, a->H, a->B), dim3(kAtThreads), kAtSmem, stream,
+  return launch_pdl(prefill_attn_kernel, dim3((a->s_q + 255) / 256, a->H, a->B), dim3(kAtThreads), kAtSmem, stream,
                     tm_qn, tm_qp, tm_kn, tm_v, tm_c, at);
 }
 
