@@ -13,6 +13,9 @@ Draw recipe (fixed; changing it changes every stored expectation):
 * q8_0 cache: each block of 32 consecutive values of a row gets the scale
   ``d = amax(block) / 127`` rounded to fp16, and int8 codes ``round(x / d)``
   (nearest even, in fp32, clamped to [-127, 127]; 0 for an all-zero block);
+* q4_0 cache: the same with ``d = amax(block) / 7`` and codes in [-7, 7], each
+  stored as the 4-bit number code + 8, value 2j of a row in the low half of
+  byte j and value 2j + 1 in the high half (288 bytes a row);
 * rows of a sequence's last page at positions >= its length hold finite values
   50x larger than the real rows, so that a kernel that forgets to mask them
   produces a visibly wrong answer.
@@ -41,6 +44,7 @@ TAIL_GAIN = 50.0
 FP8_MAX = 448.0
 Q8_BLOCK = 32     # q8_0: values per scale block
 Q8_LEVELS = 127   # q8_0: largest code
+Q4_LEVELS = 7     # q4_0: largest code
 
 
 @dataclass
@@ -50,7 +54,7 @@ class WorkloadSpec:
     H: int
     s_q: int
     lens: Optional[Sequence[int]]  # explicit lengths; None => ragged draw
-    kv_dtype: str = "bf16"  # "bf16" | "fp8" | "q8_0"
+    kv_dtype: str = "bf16"  # "bf16" | "fp8" | "q8_0" | "q4_0"
     causal: bool = False
     seed: int = 0
     permute_pages: bool = True
@@ -90,6 +94,10 @@ PRESETS = {
     "q8": WorkloadSpec("q8", B=64, H=128, s_q=1, lens=[4096] * 64, kv_dtype="q8_0", seed=5,
                        note="DeepSeek-V3-shaped: batch 64, 128 heads, 4096 tokens, q8_0 cache "
                             "(int8 codes, fp16 scale per 32 values)"),
+    # the same over the 4-bit blockwise cache
+    "q4": WorkloadSpec("q4", B=64, H=128, s_q=1, lens=[4096] * 64, kv_dtype="q4_0", seed=6,
+                       note="DeepSeek-V3-shaped: batch 64, 128 heads, 4096 tokens, q4_0 cache "
+                            "(4-bit codes, fp16 scale per 32 values)"),
 }
 
 
@@ -108,7 +116,7 @@ class Workload:
     w_uk: torch.Tensor            # bf16 [H][128][512]   k = W_UK[h] . c
     w_uv: torch.Tensor            # bf16 [H][128][512]   v = W_UV[h] . c
     kv_cache: torch.Tensor        # bf16 or float8_e4m3fn [num_pages][64][576]
-    kv_scale: Optional[torch.Tensor]  # fp32 [num_pages][64] (fp8), fp16 [num_pages][64][18] (q8_0)
+    kv_scale: Optional[torch.Tensor]  # fp32 [num_pages][64] (fp8), fp16 [num_pages][64][18] (q8_0, q4_0)
     raw_rows: Optional[torch.Tensor] = None  # fp32 [num_pages][64][576] draws (keep_raw only)
     softmax_scale: float = SOFTMAX_SCALE
     extra: dict = field(default_factory=dict)
@@ -145,7 +153,8 @@ class Workload:
 
 def row_bytes(kv_dtype: str) -> int:
     """Bytes one cached token occupies: 576 values, plus their scales."""
-    return {"bf16": 2 * ROW, "fp8": ROW + 4, "q8_0": ROW + 2 * (ROW // Q8_BLOCK)}[kv_dtype]
+    return {"bf16": 2 * ROW, "fp8": ROW + 4, "q8_0": ROW + 2 * (ROW // Q8_BLOCK),
+            "q4_0": ROW // 2 + 2 * (ROW // Q8_BLOCK)}[kv_dtype]
 
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
@@ -179,14 +188,25 @@ def _quantise_rows_e4m3(rows: torch.Tensor):
     return q, scale.squeeze(-1).to(torch.float32)
 
 
-def _quantise_rows_q8_0(rows: torch.Tensor):
+def _quantise_rows_blocks(rows: torch.Tensor, levels: int):
     blocks = rows.reshape(*rows.shape[:-1], ROW // Q8_BLOCK, Q8_BLOCK)
-    d = (blocks.abs().amax(dim=-1) / Q8_LEVELS).to(torch.float16)
+    d = (blocks.abs().amax(dim=-1) / levels).to(torch.float16)
     df = d.to(torch.float32)
     safe = torch.where(df > 0, df, torch.ones_like(df))
-    q = torch.round(blocks / safe[..., None]).clamp_(-Q8_LEVELS, Q8_LEVELS)
+    q = torch.round(blocks / safe[..., None]).clamp_(-levels, levels)
     q = torch.where(df[..., None] > 0, q, torch.zeros_like(q))
     return q.to(torch.int8).reshape(rows.shape), d
+
+
+def _quantise_rows_q8_0(rows: torch.Tensor):
+    return _quantise_rows_blocks(rows, Q8_LEVELS)
+
+
+def _quantise_rows_q4_0(rows: torch.Tensor):
+    """(packed uint8 [..., 288], fp16 scales [..., 18])."""
+    q, d = _quantise_rows_blocks(rows, Q4_LEVELS)
+    n = (q.to(torch.int16) + 8).to(torch.uint8)
+    return n[..., 0::2] | (n[..., 1::2] << 4), d
 
 
 def make_workload(spec: WorkloadSpec, keep_raw: bool = False) -> Workload:
@@ -223,11 +243,15 @@ def make_workload(spec: WorkloadSpec, keep_raw: bool = False) -> Workload:
     # stored at their physical page.  Tail rows of a last page get TAIL_GAIN.
     fp8 = spec.kv_dtype == "fp8"
     q8 = spec.kv_dtype == "q8_0"
+    q4 = spec.kv_dtype == "q4_0"
     if fp8:
         kv_cache = torch.zeros(num_pages, PAGE, ROW, dtype=torch.float8_e4m3fn)
         kv_scale = torch.ones(num_pages, PAGE, dtype=torch.float32)
     elif q8:
         kv_cache = torch.zeros(num_pages, PAGE, ROW, dtype=torch.int8)
+        kv_scale = torch.zeros(num_pages, PAGE, ROW // Q8_BLOCK, dtype=torch.float16)
+    elif q4:
+        kv_cache = torch.zeros(num_pages, PAGE, ROW // 2, dtype=torch.uint8)
         kv_scale = torch.zeros(num_pages, PAGE, ROW // Q8_BLOCK, dtype=torch.float16)
     else:
         kv_cache = torch.zeros(num_pages, PAGE, ROW, dtype=torch.bfloat16)
@@ -252,6 +276,10 @@ def make_workload(spec: WorkloadSpec, keep_raw: bool = False) -> Workload:
                 kv_scale[idx] = sc
             elif q8:
                 q, sc = _quantise_rows_q8_0(rows)
+                kv_cache[idx] = q
+                kv_scale[idx] = sc
+            elif q4:
+                q, sc = _quantise_rows_q4_0(rows)
                 kv_cache[idx] = q
                 kv_scale[idx] = sc
             else:

@@ -18,6 +18,8 @@ def from_workload(w) -> OracleInputs:
         kv, scale = bf16_bits(w.kv_cache), None
     elif kind == "q8_0":
         kv, scale = int8_bits(w.kv_cache), f16_bits(w.kv_scale)
+    elif kind == "q4_0":
+        kv, scale = w.kv_cache.contiguous().numpy(), f16_bits(w.kv_scale)
     else:
         kv, scale = fp8_bits(w.kv_cache), w.kv_scale.numpy()
     return OracleInputs(bf16_bits(w.q_nope), bf16_bits(w.q_pe), bf16_bits(w.w_uk),

@@ -28,6 +28,12 @@ Readings taken where the pages are silent (each one is listed with the design):
   row), codes = the fp32 quotient ``value / scale`` rounded to nearest even and
   saturated at +-448.  The decision takes fp32 inputs, so the fp64 row is first
   rounded to fp32.
+* q8_0 and q4_0 caches: blocks of 32 values, one fp16 scale ``d = amax / levels``
+  (127 or 7, computed in fp32), codes = the fp32 quotients ``value / d`` rounded
+  to nearest even and clamped to +-levels (0 for an all-zero block).  q4_0 codes
+  are stored as the 4-bit number code + 8, value 2j of the row in the low half of
+  byte j and value 2j + 1 in the high half (the docs name the type, not its
+  byte layout).
 
 Pinned by ``tests/test_cache_write_oracle.py``: the encoders against torch's
 casts, RoPE against closed forms and its relative-position identity, the paged
@@ -120,21 +126,34 @@ def quantise_row_e4m3(row: np.ndarray) -> Tuple[np.ndarray, np.float32]:
     return f64_to_e4m3fn(np.clip(q.astype(np.float64), -E4M3_MAX, E4M3_MAX)), scale
 
 
+def _quantise_row_blocks(row: np.ndarray, levels: int) -> Tuple[np.ndarray, np.ndarray]:
+    r32 = np.asarray(row, dtype=np.float64).astype(np.float32).reshape(-1, 32)
+    amax = np.max(np.abs(r32), axis=1)
+    d16 = (amax / np.float32(levels)).astype(np.float32).astype(np.float16)
+    d32 = d16.astype(np.float32)
+    safe = np.where(d32 > 0, d32, np.float32(1.0))
+    q = np.rint((r32 / safe[:, None]).astype(np.float32))
+    q = np.clip(q, -levels, levels)
+    q = np.where(d32[:, None] > 0, q, 0)
+    return q.astype(np.int8).reshape(-1), d16
+
+
 def quantise_row_q8_0(row: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
     """One 576-value row -> (int8 codes [576], fp16 scales [18]) of the q8_0 format
     (ik_llama.cpp docs "FlashMLA", section "KV cache with MLA"; blocks of 32
     values, d = amax / 127 rounded to fp16, codes round(x / d) in [-127, 127]).
     The row is taken at fp32 precision and amax / 127 and the quotients are fp32
     IEEE operations, as for the e4m3 row."""
-    r32 = np.asarray(row, dtype=np.float64).astype(np.float32).reshape(-1, 32)
-    amax = np.max(np.abs(r32), axis=1)
-    d16 = (amax / np.float32(127.0)).astype(np.float32).astype(np.float16)
-    d32 = d16.astype(np.float32)
-    safe = np.where(d32 > 0, d32, np.float32(1.0))
-    q = np.rint((r32 / safe[:, None]).astype(np.float32))
-    q = np.clip(q, -127, 127)
-    q = np.where(d32[:, None] > 0, q, 0)
-    return q.astype(np.int8).reshape(-1), d16
+    return _quantise_row_blocks(row, 127)
+
+
+def quantise_row_q4_0(row: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """One 576-value row -> (packed codes uint8 [288], fp16 scales [18]) of the
+    q4_0 format: as q8_0 with d = amax / 7 and codes in [-7, 7]; byte j holds
+    code 2j + 8 in its low four bits and code 2j+1 + 8 in its high four bits."""
+    q, d16 = _quantise_row_blocks(row, 7)
+    n = (q.astype(np.int64) + 8).astype(np.uint8)
+    return (n[0::2] | (n[1::2] << 4)).astype(np.uint8), d16
 
 
 def slot_of(block_table: np.ndarray, seq_lens: np.ndarray, s_q: int, b: int, i: int,
@@ -158,13 +177,14 @@ def write_kv(h: np.ndarray, w_dkv: np.ndarray, w_kr: np.ndarray, kv: np.ndarray,
     returns (kv, kv_scale).
 
     h [B][s_q][d_h] (fp64 values), w_dkv [512][d_h], w_kr [64][d_h]; kv holds raw
-    bits [num_pages][64][576] (uint16 bf16, uint8 e4m3, int8 q8_0 codes); kv_scale
-    is fp32 [num_pages][64] for e4m3, fp16 [num_pages][64][18] for q8_0.  Every
+    bits [num_pages][64][576] (uint16 bf16, uint8 e4m3, int8 q8_0 codes) or
+    [num_pages][64][288] (uint8 packed q4_0 codes); kv_scale is fp32
+    [num_pages][64] for e4m3, fp16 [num_pages][64][18] for q8_0 and q4_0.  Every
     row other than the new tokens' is left as it was."""
-    assert kv_dtype in ("bf16", "fp8", "q8_0")
+    assert kv_dtype in ("bf16", "fp8", "q8_0", "q4_0")
     B = h.shape[0]
     kv = np.array(kv, copy=True)
-    if kv_dtype == "q8_0":
+    if kv_dtype in ("q8_0", "q4_0"):
         kv_scale = np.array(kv_scale, dtype=np.float16, copy=True)
     else:
         kv_scale = None if kv_scale is None else np.array(kv_scale, dtype=np.float32, copy=True)
@@ -179,6 +199,8 @@ def write_kv(h: np.ndarray, w_dkv: np.ndarray, w_kr: np.ndarray, kv: np.ndarray,
                 kv[page, row] = f64_to_bf16(full)
             elif kv_dtype == "q8_0":
                 kv[page, row], kv_scale[page, row] = quantise_row_q8_0(full)
+            elif kv_dtype == "q4_0":
+                kv[page, row], kv_scale[page, row] = quantise_row_q4_0(full)
             else:
                 kv[page, row], kv_scale[page, row] = quantise_row_e4m3(full)
     return kv, kv_scale

@@ -89,14 +89,19 @@ class OracleInputs:
 
     q_nope [B][s_q][H][128] and q_pe [B][s_q][H][64] as bf16 bits; w_uk, w_uv
     [H][128][512] bf16 bits; kv [num_pages][64][576] as bf16 (uint16), e4m3
-    (uint8) or q8_0 (int8 codes, as uint8) bits; kv_scale fp32 [num_pages][64]
-    for e4m3, fp16 bits [num_pages][64][18] (one scale per 32-value block) for
-    q8_0, else None; block_table int [B][max_pages]; seq_lens int [B] (lengths
-    include the s_q new tokens).
+    (uint8) or q8_0 (int8 codes, as uint8) bits, or [num_pages][64][288] packed
+    q4_0 codes (uint8); kv_scale fp32 [num_pages][64] for e4m3, fp16 bits
+    [num_pages][64][18] (one scale per 32-value block) for q8_0 and q4_0, else
+    None; block_table int [B][max_pages]; seq_lens int [B] (lengths include the
+    s_q new tokens).
 
-    q8_0 (ik_llama.cpp docs "FlashMLA", section "KV cache with MLA": the
-    recommended quantised MLA cache): value = code * the block's scale, blocks of
-    32 consecutive values of the 576-value row.
+    q8_0 and q4_0 (ik_llama.cpp docs "FlashMLA", section "KV cache with MLA":
+    q8_0 is the recommended quantised MLA cache, lower-bit types are used with a
+    Hadamard rotation): value = code * the block's scale, blocks of 32
+    consecutive values of the 576-value row.  The docs fix no byte layout for
+    q4_0; the reading taken here: codes in [-7, 7] stored as the 4-bit number
+    code + 8, value 2j of the row in the low half of byte j and value 2j + 1 in
+    its high half (288 bytes a row).
     """
 
     def __init__(self, q_nope, q_pe, w_uk, w_uv, kv, kv_dtype, kv_scale, block_table,
@@ -107,7 +112,7 @@ class OracleInputs:
         self.w_uv = bf16_to_f64(w_uv)
         self.kv = np.asarray(kv)
         self.kv_dtype = kv_dtype
-        if kv_dtype == "q8_0":
+        if kv_dtype in ("q8_0", "q4_0"):
             self.kv_scale = f16_to_f64(kv_scale)
         else:
             self.kv_scale = None if kv_scale is None else np.asarray(kv_scale, dtype=np.float64)
@@ -116,7 +121,7 @@ class OracleInputs:
         self.softmax_scale = float(softmax_scale)
         self.causal = bool(causal)
         self.B, self.s_q, self.H, _ = self.q_nope.shape
-        assert kv_dtype in ("bf16", "fp8", "q8_0")
+        assert kv_dtype in ("bf16", "fp8", "q8_0", "q4_0")
 
     def visible(self, b: int, i: int) -> int:
         """Number of cached tokens query i of sequence b attends to."""
@@ -132,11 +137,18 @@ class OracleInputs:
             return np.zeros((0, D_C + D_R))
         npg = (n + PAGE - 1) // PAGE
         pages = self.block_table[b, :npg]
-        raw = self.kv[pages].reshape(npg * PAGE, D_C + D_R)[:n]
+        raw = self.kv[pages].reshape(npg * PAGE, -1)[:n]
         if self.kv_dtype == "bf16":
             return bf16_to_f64(raw)
         if self.kv_dtype == "q8_0":
             codes = raw.astype(np.uint8).view(np.int8).astype(np.float64)          # [n][576]
+            block = self.kv_scale[pages].reshape(npg * PAGE, -1)[:n]               # [n][18]
+            return codes * np.repeat(block, Q8_BLOCK, axis=1)
+        if self.kv_dtype == "q4_0":
+            byte = raw.astype(np.int64)                                            # [n][288]
+            codes = np.empty((n, D_C + D_R))
+            codes[:, 0::2] = (byte & 0xF) - 8
+            codes[:, 1::2] = (byte >> 4) - 8
             block = self.kv_scale[pages].reshape(npg * PAGE, -1)[:n]               # [n][18]
             return codes * np.repeat(block, Q8_BLOCK, axis=1)
         scale = self.kv_scale[pages].reshape(npg * PAGE)[:n]

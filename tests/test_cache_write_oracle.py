@@ -11,7 +11,10 @@ none of which re-types the oracle's own formulas.
 * the paged write by brute force (only the new rows change, page order is
   addressing only) and its error cases;
 * the whole write read back through the decode oracle: one cached token gives
-  ``o = W_UV c`` with ``c = W_DKV h`` (closed form).
+  ``o = W_UV c`` with ``c = W_DKV h`` (closed form);
+* the q8_0 and q4_0 row quantisers against the low-bit oracle's blockwise
+  quantiser, q4_0's zero block, extremes and packing by hand, and the paged
+  q8_0 / q4_0 writes by brute force.
 """
 
 import numpy as np
@@ -262,4 +265,63 @@ def test_q8_0_write_touches_only_the_new_rows():
     full = np.concatenate([c[1], cw.rope(kr, np.array([65]), 10000.0)[1]])
     got = kv2[1, 1].astype(np.float64) * np.repeat(sc2[1, 1].astype(np.float64), 32)
     step = np.repeat(sc2[1, 1].astype(np.float64), 32)
+    assert np.all(np.abs(got - full) <= 0.5 * step + 1e-3 * np.abs(full) + 1e-9)
+
+
+def _unpack_q4(packed: np.ndarray) -> np.ndarray:
+    """Codes of a packed q4_0 row: value 2j in the low four bits of byte j, value
+    2j + 1 in the high four, each stored as code + 8."""
+    b = packed.astype(np.int64)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.int64)
+    out[..., 0::2] = (b & 15) - 8
+    out[..., 1::2] = (b >> 4) - 8
+    return out
+
+
+def test_q4_0_row_quantisation_matches_the_blockwise_format():
+    """The cache write's q4_0 row (fp32 arithmetic, packed) against the low-bit
+    oracle's blockwise quantiser (fp64): scales equal, codes equal except where an
+    fp32 quotient falls on the other side of a rounding boundary."""
+    from oracle import lowbit_cache as lb
+    rng = np.random.default_rng(13)
+    diff = 0
+    for _ in range(200):
+        row = rng.standard_normal(576) * rng.uniform(0.01, 50.0)
+        row32 = row.astype(np.float32).astype(np.float64)
+        packed, d = cw.quantise_row_q4_0(row)
+        assert packed.shape == (288,) and packed.dtype == np.uint8
+        codes = _unpack_q4(packed)
+        ref_codes, ref_d = lb.quantise_blocks(row32, "q4_0")
+        assert np.array_equal(d.astype(np.float64), ref_d)
+        diff += int((codes != ref_codes).sum())
+        assert np.abs(codes - ref_codes).max() <= 1
+    assert diff <= 2e-4 * 200 * 576
+
+
+def test_q4_0_zero_block_and_extremes():
+    row = np.zeros(576)
+    row[32:64] = np.linspace(-3.5, 7.0, 32)          # block 1: amax 7 -> d = 1
+    packed, d = cw.quantise_row_q4_0(row)
+    codes = _unpack_q4(packed)
+    assert d[0] == 0 and np.all(codes[:32] == 0)      # an all-zero block: zero codes
+    assert d[1] == 1.0 and codes[63] == 7 and codes[32] == -4  # -3.5 rounds to even
+    assert packed[0] == 0x88                          # two zero codes: 8 | 8 << 4
+
+
+def test_q4_0_write_touches_only_the_new_rows():
+    rng = np.random.default_rng(14)
+    B, s_q, d_h, P = 2, 2, 64, 6
+    h = rng.standard_normal((B, s_q, d_h))
+    w_dkv, w_kr = rng.standard_normal((512, d_h)) / 8, rng.standard_normal((64, d_h)) / 8
+    kv = rng.integers(0, 256, size=(P, 64, 288)).astype(np.uint8)
+    sc = rng.random((P, 64, 18)).astype(np.float16)
+    bt = np.array([[3, 1], [0, 5]])
+    lens = np.array([66, 10])
+    kv2, sc2 = cw.write_kv(h, w_dkv, w_kr, kv, sc, "q4_0", bt, lens, s_q)
+    changed = np.argwhere((kv2 != kv).any(axis=2) | (sc2 != sc).any(axis=2))
+    assert sorted(map(tuple, changed)) == [(0, 8), (0, 9), (1, 0), (1, 1)]
+    c, kr = cw.compress(h[0], w_dkv, w_kr)
+    full = np.concatenate([c[1], cw.rope(kr, np.array([65]), 10000.0)[1]])
+    step = np.repeat(sc2[1, 1].astype(np.float64), 32)
+    got = _unpack_q4(kv2[1, 1]) * step
     assert np.all(np.abs(got - full) <= 0.5 * step + 1e-3 * np.abs(full) + 1e-9)

@@ -9,7 +9,11 @@
   fp16 rounding of the scale), block extremes on the outermost code, zero blocks,
   blocks independent of one another;
 * the pages' claim that the rotation helps at low bit widths, on rows with an
-  outlier: the q4_0 error after rotate -> quantise -> rotate back is smaller.
+  outlier: the q4_0 error after rotate -> quantise -> rotate back is smaller;
+* the decode oracle's q8_0 and q4_0 caches: rows read back as the blockwise
+  dequantisation of the raw draw, a hand-made q4_0 row pins the byte layout, a
+  q4_0 cache equals a q8_0 cache holding the same codes, and the absorbed form
+  equals the definition over both.
 """
 
 import numpy as np
@@ -139,6 +143,79 @@ def test_q8_0_cache_rows_are_the_blockwise_dequantisation():
 def test_q8_0_decode_absorbed_equals_the_definition():
     import oracle
     w = _q8_workload(lens=(1, 200), H=16)
+    inp = oracle.from_workload(w)
+    a = om.decode_absorbed(inp)
+    d = om.decode_nonabsorbed(inp)
+    for key in ("o", "o_lat", "lse"):
+        assert np.allclose(a[key], d[key], rtol=1e-10, atol=1e-12)
+
+
+# ---------------------------------------------------------------- q4_0 cache in the decode oracle
+
+def _q4_workload(lens=(70, 130), H=16, seed=3):
+    from mla_inputs import WorkloadSpec, make_workload
+    return make_workload(WorkloadSpec("q4", B=len(lens), H=H, s_q=1, lens=list(lens), kv_dtype="q4_0",
+                                      seed=seed), keep_raw=True)
+
+
+def test_q4_0_byte_layout():
+    """One hand-made row: byte 0 = 0x1F holds code 15 - 8 = 7 (value 0, low four
+    bits) and 1 - 8 = -7 (value 1, high four bits); byte 0x88 is two zeros."""
+    kv = np.full((1, 64, 288), 0x88, dtype=np.uint8)
+    kv[0, 0, 0] = 0x1F
+    kv[0, 0, 17] = 0xA3                              # values 34, 35: 3 - 8, 10 - 8
+    sc = np.zeros((1, 64, 18), dtype=np.float16)
+    sc[0, 0, :] = 0.5
+    sc[0, 0, 1] = 2.0
+    z = np.zeros((1, 1, 16, 128), dtype=np.uint16)
+    inp = om.OracleInputs(z, np.zeros((1, 1, 16, 64), np.uint16), np.zeros((16, 128, 512), np.uint16),
+                          np.zeros((16, 128, 512), np.uint16), kv, "q4_0", sc.view(np.uint16),
+                          np.zeros((1, 1), np.int64), np.array([1]), 1.0, False)
+    row = inp.rows(0, 1)[0]
+    want = np.zeros(576)
+    want[0], want[1] = 3.5, -3.5
+    want[34], want[35] = -10.0, 4.0
+    assert np.array_equal(row, want)
+
+
+def test_q4_0_cache_rows_are_the_blockwise_dequantisation():
+    """The decode oracle reads a q4_0 row as code * block scale: the values the
+    low-bit oracle's quantiser gives for the raw fp32 draw."""
+    import oracle
+    w = _q4_workload()
+    inp = oracle.from_workload(w)
+    raw = w.raw_rows.double().numpy()
+    for b, L in enumerate(w.lens):
+        C = inp.rows(b, L)
+        for j in (0, 31, L - 1):
+            pg, rr = int(w.block_table[b, j // 64]), j % 64
+            codes, d = lb.quantise_blocks(raw[pg, rr], "q4_0")
+            assert np.array_equal(C[j], lb.dequantise_blocks(codes, d))
+
+
+def test_q4_0_equals_q8_0_on_the_same_codes():
+    """A q4_0 cache and a q8_0 cache holding the same codes (all within [-7, 7])
+    and scales give the same attention: the 4-bit storage is only addressing."""
+    import oracle
+    from mla_inputs import WorkloadSpec, make_workload
+    w = make_workload(WorkloadSpec("q8", B=2, H=16, s_q=1, lens=[70, 130], kv_dtype="q8_0", seed=8))
+    inp8 = oracle.from_workload(w)
+    codes = np.clip(inp8.kv.view(np.int8).astype(np.int64), -7, 7)
+    inp8.kv = codes.astype(np.int8).view(np.uint8)
+    n = (codes + 8).astype(np.uint8)
+    kv4 = n[..., 0::2] | (n[..., 1::2] << 4)
+    from mla_inputs import bf16_bits, f16_bits
+    inp4 = om.OracleInputs(bf16_bits(w.q_nope), bf16_bits(w.q_pe), bf16_bits(w.w_uk), bf16_bits(w.w_uv),
+                           kv4, "q4_0", f16_bits(w.kv_scale), w.block_table.numpy(), w.seq_lens.numpy(),
+                           w.softmax_scale, False)
+    a, b = om.decode_absorbed(inp8), om.decode_absorbed(inp4)
+    for key in ("o", "o_lat", "lse"):
+        assert np.array_equal(a[key], b[key])
+
+
+def test_q4_0_decode_absorbed_equals_the_definition():
+    import oracle
+    w = _q4_workload(lens=(1, 200), H=16)
     inp = oracle.from_workload(w)
     a = om.decode_absorbed(inp)
     d = om.decode_nonabsorbed(inp)
