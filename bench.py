@@ -51,6 +51,8 @@ MEASURED_TRAFFIC = {
     "long128": (608_454_912, "decode_tc.cu", "7bb76fcc659538c8"),
     # one launch of the q8_0 workload (the same kernel file, its q8_0 variant)
     "q8": (175_534_592, "decode_tc.cu", "7bb76fcc659538c8"),
+    # one launch of the q4_0 workload (the q4_0 variant)
+    "q4": (98_002_688, "decode_tc.cu", "30109a2e70d165f7"),
     # both prefill kernels on one sequence of the chunked-prefill workload:
     # 1,153,470,976 bytes, times the 4 sequences of the full workload (traffic
     # grows with the sequences processed)
@@ -305,7 +307,8 @@ WRITE_METRIC = "MLA cache write GB/s (latent + RoPE key into the paged cache) & 
 def run_write_kv(args):
     """Times mla_write_kv for the new tokens of one decode step of the workload:
     hidden states of width d_h -> latent c = W_DKV h and rotated RoPE key -> their
-    rows of the paged cache (bf16, or e4m3 with per-row scales).  One GPU; the
+    rows of the paged cache (bf16, e4m3 with per-row scales, or q8_0 / q4_0 with
+    per-block scales).  One GPU; the
     two launches are replayed from a CUDA graph with L2 flushed before each."""
     import torch
     import head_latent_attention_06_b200 as mla
@@ -358,7 +361,8 @@ def run_write_kv(args):
     line = {"metric": WRITE_METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16 in, fp32 accumulate, " + {"bf16": "bf16", "fp8": "e4m3", "q8_0": "q8_0"}[spec.kv_dtype]
+            "dtype": "bf16 in, fp32 accumulate, " + {"bf16": "bf16", "fp8": "e4m3", "q8_0": "q8_0",
+                                                      "q4_0": "q4_0"}[spec.kv_dtype]
                      + " cache",
             "data": "synthetic (seeded N(0,1) hidden states, N(0,1/d_h) weights)", "config": cfg,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
@@ -693,6 +697,7 @@ def main(argv=None):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": {"fp8": "e4m3 cache, e4m3 x e4m3 MMA (two-term operand split)",
                   "q8_0": "q8_0 cache (int8 codes x fp16 block scales formed in bf16), bf16 MMA",
+                  "q4_0": "q4_0 cache (4-bit codes x fp16 block scales formed in bf16), bf16 MMA",
                   "bf16": "bf16"}[spec.kv_dtype],
         "data": "synthetic (seeded, N(0,1) activations and cache, N(0,1/512) weights)",
         "config": _config_dict(args.config, w, st.num_splits),

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(PKG, "libmla_b200.so")
 
 D_C, D_R, D_N, D_V, PAGE = 512, 64, 128, 128, 64
 MAX_SPLITS = 128
-KV_BF16, KV_FP8_E4M3, KV_Q8_0 = 0, 1, 2
+KV_BF16, KV_FP8_E4M3, KV_Q8_0, KV_Q4_0 = 0, 1, 2, 3
 Q8_BLOCKS = (D_C + D_R) // 32   # q8_0: scale blocks of a 576-value row
 
 STATUS = {
@@ -32,7 +32,7 @@ EXPORTS = ("mla_absorb_q", "mla_decode_workspace_size", "mla_decode_num_splits",
            "mla_decode_paged", "mla_combine_splits", "mla_up_proj_v", "mla_get_status",
            "mla_status_string", "mla_decode_paged_noalloc", "mla_noalloc_init",
            "mla_get_status_noalloc", "mla_write_kv_workspace_size", "mla_write_kv",
-           "mla_set_decode_kernel", "mla_set_device_wait_limit", "mla_prefill_workspace_size",
+           "mla_set_decode_kernel", "mla_set_device_wait_limit", "mla_fold_hadamard", "mla_prefill_workspace_size",
            "mla_prefill")
 
 DECODE_AUTO, DECODE_WARP_MMA = 0, 1
@@ -123,6 +123,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_prefill_workspace_size.argtypes = [pp, ctypes.POINTER(ctypes.c_size_t)]
     lib.mla_prefill.argtypes = [pp, vp]
     lib.mla_get_status.argtypes = [vp, vp]
+    lib.mla_fold_hadamard.argtypes = [vp, i32, vp, vp, i32, vp]
     lib.mla_status_string.argtypes = [ctypes.c_int]
     lib.mla_status_string.restype = ctypes.c_char_p
     for name in EXPORTS:
@@ -207,16 +208,33 @@ def mla_up_proj_v(o_lat, w_uv, out, stream=None):
                                                  w_uv.shape[1], w_uv.shape[2], _stream(stream)))
 
 
+def mla_fold_hadamard(w_dkv=None, w_uk=None, w_uv=None, stream=None):
+    """Folds the orthonormal 512-point Hadamard rotation into the weights, in place:
+    w_dkv [576][d_h] (rows 0..511 -> H W_DKV), w_uk and w_uv [H][128][512] (each row
+    -> row H); bf16 on the device, any of them may be None."""
+    import torch
+    H = (w_uk if w_uk is not None else w_uv).shape[0] if (w_uk is not None or w_uv is not None) else 0
+    d_h = w_dkv.shape[1] if w_dkv is not None else 0
+    _want([(w_dkv, "w_dkv", torch.bfloat16, (D_C + D_R, d_h), True),
+           (w_uk, "w_uk", torch.bfloat16, (H, D_N, D_C), True),
+           (w_uv, "w_uv", torch.bfloat16, (H, D_V, D_C), True)])
+    _check("mla_fold_hadamard", load().mla_fold_hadamard(_ptr(w_dkv), d_h, _ptr(w_uk), _ptr(w_uv), H,
+                                                         _stream(stream)))
+
+
 def _cache_kind(kv_cache):
-    """(kv_dtype code, scale dtype, scale shape tail) of a cache tensor's dtype:
-    bf16 values; float8_e4m3fn codes with fp32 row scales [pages][64]; int8 q8_0
-    codes with fp16 block scales [pages][64][18]."""
+    """(kv_dtype code, scale dtype, scale shape tail, row width) of a cache tensor's
+    dtype: bf16 values; float8_e4m3fn codes with fp32 row scales [pages][64]; int8
+    q8_0 codes with fp16 block scales [pages][64][18]; uint8 q4_0 bytes (two codes
+    a byte, 288 a row) with fp16 block scales [pages][64][18]."""
     import torch
     if kv_cache.dtype == torch.float8_e4m3fn:
-        return KV_FP8_E4M3, torch.float32, ()
+        return KV_FP8_E4M3, torch.float32, (), D_C + D_R
     if kv_cache.dtype == torch.int8:
-        return KV_Q8_0, torch.float16, (Q8_BLOCKS,)
-    return KV_BF16, None, ()
+        return KV_Q8_0, torch.float16, (Q8_BLOCKS,), D_C + D_R
+    if kv_cache.dtype == torch.uint8:
+        return KV_Q4_0, torch.float16, (Q8_BLOCKS,), (D_C + D_R) // 2
+    return KV_BF16, None, (), D_C + D_R
 
 
 def make_decode_args(*, q_lat, q_pe, kv_cache, kv_scale, block_table, seq_lens, o_lat, lse,
@@ -224,19 +242,20 @@ def make_decode_args(*, q_lat, q_pe, kv_cache, kv_scale, block_table, seq_lens, 
                      max_seq_len=0) -> DecodeArgs:
     """Fill a ``DecodeArgs`` from device tensors.  Shapes: q_lat [B][s_q][H][512],
     q_pe [B][s_q][H][64], kv_cache [num_pages][64][576] (bf16, float8_e4m3fn or
-    int8 for q8_0), kv_scale [num_pages][64] fp32 (e4m3), [num_pages][64][18] fp16
-    (q8_0) or None (bf16), block_table [B][max_pages] int32, seq_lens [B] int32,
-    o_lat like q_lat, lse [B][s_q][H] fp32 or None."""
+    int8 for q8_0) or [num_pages][64][288] uint8 (q4_0), kv_scale [num_pages][64]
+    fp32 (e4m3), [num_pages][64][18] fp16 (q8_0, q4_0) or None (bf16), block_table
+    [B][max_pages] int32, seq_lens [B] int32, o_lat like q_lat, lse [B][s_q][H]
+    fp32 or None."""
     import torch
     bf16, f32, i32 = torch.bfloat16, torch.float32, torch.int32
     if q_lat.dim() != 4 or kv_cache.dim() != 3 or block_table.dim() != 2:
         raise ValueError("q_lat must be [B][s_q][H][512], kv_cache [pages][64][576], block_table [B][pages]")
     B, s_q, H, _ = q_lat.shape
     P = kv_cache.shape[0]
-    kind, sc_dtype, sc_tail = _cache_kind(kv_cache)
+    kind, sc_dtype, sc_tail, width = _cache_kind(kv_cache)
     _want([(q_lat, "q_lat", bf16, (B, s_q, H, D_C), False),
            (q_pe, "q_pe", bf16, (B, s_q, H, D_R), False),
-           (kv_cache, "kv_cache", (bf16, torch.float8_e4m3fn, torch.int8), (P, PAGE, D_C + D_R), False),
+           (kv_cache, "kv_cache", (bf16, torch.float8_e4m3fn, torch.int8, torch.uint8), (P, PAGE, width), False),
            (kv_scale, "kv_scale", sc_dtype or f32, (P, PAGE) + sc_tail, kind == KV_BF16),
            (block_table, "block_table", i32, (B, block_table.shape[1]), False),
            (seq_lens, "seq_lens", i32, (B,), False),
@@ -314,19 +333,19 @@ def make_write_kv_args(*, h, w_dkv, kv_cache, kv_scale, block_table, seq_lens, w
                        rope_base=10000.0) -> WriteKvArgs:
     """Fill a ``WriteKvArgs`` from device tensors.  Shapes: h [B][s_q][d_h] bf16,
     w_dkv [576][d_h] bf16 (W_DKV rows, then W_KR rows), kv_cache [num_pages][64][576]
-    (bf16, float8_e4m3fn or int8 for q8_0), kv_scale [num_pages][64] fp32 (e4m3),
-    [num_pages][64][18] fp16 (q8_0) or None (bf16), block_table [B][max_pages]
-    int32, seq_lens [B] int32."""
+    (bf16, float8_e4m3fn or int8 for q8_0) or [num_pages][64][288] uint8 (q4_0),
+    kv_scale [num_pages][64] fp32 (e4m3), [num_pages][64][18] fp16 (q8_0, q4_0) or
+    None (bf16), block_table [B][max_pages] int32, seq_lens [B] int32."""
     import torch
     bf16, f32, i32 = torch.bfloat16, torch.float32, torch.int32
     if h.dim() != 3 or kv_cache.dim() != 3 or block_table.dim() != 2:
         raise ValueError("h must be [B][s_q][d_h], kv_cache [pages][64][576], block_table [B][pages]")
     B, s_q, d_h = h.shape
     P = kv_cache.shape[0]
-    kind, sc_dtype, sc_tail = _cache_kind(kv_cache)
+    kind, sc_dtype, sc_tail, width = _cache_kind(kv_cache)
     _want([(h, "h", bf16, (B, s_q, d_h), False),
            (w_dkv, "w_dkv", bf16, (D_C + D_R, d_h), False),
-           (kv_cache, "kv_cache", (bf16, torch.float8_e4m3fn, torch.int8), (P, PAGE, D_C + D_R), False),
+           (kv_cache, "kv_cache", (bf16, torch.float8_e4m3fn, torch.int8, torch.uint8), (P, PAGE, width), False),
            (kv_scale, "kv_scale", sc_dtype or f32, (P, PAGE) + sc_tail, kind == KV_BF16),
            (block_table, "block_table", i32, (B, block_table.shape[1]), False),
            (seq_lens, "seq_lens", i32, (B,), False),

@@ -23,6 +23,7 @@ int write_kv_k_split(int n_tok, int d_h);
 cudaError_t launch_write_kv(const mla_write_kv_args_t*, cudaStream_t);
 size_t prefill_workspace_bytes(int B, int H, int Lmax);
 cudaError_t launch_prefill(const mla_prefill_args_t*, cudaStream_t);
+cudaError_t launch_fold_hadamard(void*, int, void*, void*, int, cudaStream_t);
 }  // namespace mla
 
 using namespace mla;
@@ -50,7 +51,8 @@ mla_status_t check_decode_shape(const mla_decode_args_t* a) {
     return MLA_ERR_INVALID_VALUE;
   if (a->d_c != kDc || a->d_r != kDr || a->page_size != kPage) return MLA_ERR_UNSUPPORTED;
   if (a->H % 16 != 0 || a->H > 128 || a->s_q > MLA_MAX_S_Q) return MLA_ERR_UNSUPPORTED;
-  if (a->kv_dtype != MLA_KV_BF16 && a->kv_dtype != MLA_KV_FP8_E4M3 && a->kv_dtype != MLA_KV_Q8_0)
+  if (a->kv_dtype != MLA_KV_BF16 && a->kv_dtype != MLA_KV_FP8_E4M3 && a->kv_dtype != MLA_KV_Q8_0 &&
+      a->kv_dtype != MLA_KV_Q4_0)
     return MLA_ERR_UNSUPPORTED;
   if (a->num_splits < 0 || a->num_splits > MLA_MAX_SPLITS) return MLA_ERR_INVALID_VALUE;
   if (a->max_seq_len < 0) return MLA_ERR_INVALID_VALUE;
@@ -116,7 +118,8 @@ mla_status_t check_write_kv_shape(const mla_write_kv_args_t* a) {
     return MLA_ERR_INVALID_VALUE;
   if ((int64_t)a->B * a->s_q > (1 << 24)) return MLA_ERR_INVALID_VALUE;
   if (a->d_c != kDc || a->d_r != kDr || a->page_size != kPage || a->d_h % 64 != 0) return MLA_ERR_UNSUPPORTED;
-  if (a->kv_dtype != MLA_KV_BF16 && a->kv_dtype != MLA_KV_FP8_E4M3 && a->kv_dtype != MLA_KV_Q8_0)
+  if (a->kv_dtype != MLA_KV_BF16 && a->kv_dtype != MLA_KV_FP8_E4M3 && a->kv_dtype != MLA_KV_Q8_0 &&
+      a->kv_dtype != MLA_KV_Q4_0)
     return MLA_ERR_UNSUPPORTED;
   if (!(a->rope_base > 0.f) || !isfinite(a->rope_base)) return MLA_ERR_INVALID_VALUE;
   return MLA_OK;
@@ -246,6 +249,13 @@ mla_status_t mla_write_kv(const mla_write_kv_args_t* a, void* stream) {
       (reinterpret_cast<uintptr_t>(a->kv_scale) & 3u))
     return MLA_ERR_MISALIGNED;
   return from_cuda(launch_write_kv(a, (cudaStream_t)stream));
+}
+
+mla_status_t mla_fold_hadamard(void* w_dkv, int32_t d_h, void* w_uk, void* w_uv, int32_t H, void* stream) {
+  if (H < 0 || (w_dkv && d_h <= 0)) return MLA_ERR_INVALID_VALUE;
+  if (H > 128 || (w_dkv && d_h % 64 != 0)) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(w_dkv) || !aligned16(w_uk) || !aligned16(w_uv)) return MLA_ERR_MISALIGNED;
+  return from_cuda(launch_fold_hadamard(w_dkv, d_h, w_uk, w_uv, H, (cudaStream_t)stream));
 }
 
 mla_status_t mla_prefill_workspace_size(const mla_prefill_args_t* a, size_t* bytes) {

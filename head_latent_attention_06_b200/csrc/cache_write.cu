@@ -7,7 +7,8 @@
 //   row    = c || k_pe  -> row pos % 64 of page block_table[b][pos / 64], stored as
 //            bf16 (round to nearest even) or as e4m3 codes with one fp32 scale per
 //            row, scale = amax / 448 (ik_llama.cpp docs "FlashMLA", "KV cache with MLA":
-//            the latent cache may be quantised)
+//            the latent cache may be quantised), or blockwise q8_0 / q4_0 codes
+//            with one fp16 scale per 32 values
 // RoPE turns value pair (2i, 2i+1) by pos * base^(-2i/64).
 //
 // Two kernels.  The down-projection [n_tok x d_h] . [d_h x 576] is bound by
@@ -223,25 +224,32 @@ __global__ void __launch_bounds__(128) kv_finish_kernel(const FinishParams p) {
     __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(p.kv) + slot * kRow + 2 * lane;
 #pragma unroll
     for (int j = 0; j < 9; ++j) *reinterpret_cast<uint32_t*>(row + 64 * j) = pack_bf16(v[j].x, v[j].y);
-  } else if constexpr (KIND == 2) {
-    // q8_0: block 2j + lane / 16 is values 64j + 32 (lane / 16) .. +31, two per
-    // lane of its half-warp; scale d = amax / 127 rounded to fp16, codes the fp32
-    // quotients by d rounded to nearest even and clamped to [-127, 127]
-    int8_t* row = reinterpret_cast<int8_t*>(p.kv) + slot * kRow + 2 * lane;
+  } else if constexpr (KIND == 2 || KIND == 3) {
+    // q8_0 / q4_0: block 2j + lane / 16 is values 64j + 32 (lane / 16) .. +31, two
+    // per lane of its half-warp; scale d = amax / levels (127 or 7) rounded to
+    // fp16, codes the fp32 quotients by d rounded to nearest even and clamped to
+    // [-levels, levels].  q4_0 stores code + 8 in four bits: values 64j + 2 lane
+    // and 64j + 2 lane + 1 share byte 32j + lane (low half, high half).
+    constexpr float levels = KIND == 2 ? 127.f : 7.f;
     __half* sc = static_cast<__half*>(p.kv_scale) + slot * (kRow / 32);
 #pragma unroll
     for (int j = 0; j < 9; ++j) {
       float amax = fmaxf(fabsf(v[j].x), fabsf(v[j].y));
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      const __half d = __float2half_rn(__fdiv_rn(amax, 127.f));
+      const __half d = __float2half_rn(__fdiv_rn(amax, levels));
       const float df = __half2float(d);
       int c0 = 0, c1 = 0;
       if (df > 0.f) {
-        c0 = (int)fminf(fmaxf(rintf(__fdiv_rn(v[j].x, df)), -127.f), 127.f);
-        c1 = (int)fminf(fmaxf(rintf(__fdiv_rn(v[j].y, df)), -127.f), 127.f);
+        c0 = (int)fminf(fmaxf(rintf(__fdiv_rn(v[j].x, df)), -levels), levels);
+        c1 = (int)fminf(fmaxf(rintf(__fdiv_rn(v[j].y, df)), -levels), levels);
       }
-      *reinterpret_cast<uint16_t*>(row + 64 * j) = (uint16_t)((uint8_t)c0 | ((uint16_t)(uint8_t)c1 << 8));
+      if constexpr (KIND == 2) {
+        int8_t* row = reinterpret_cast<int8_t*>(p.kv) + slot * kRow + 2 * lane;
+        *reinterpret_cast<uint16_t*>(row + 64 * j) = (uint16_t)((uint8_t)c0 | ((uint16_t)(uint8_t)c1 << 8));
+      } else {
+        p.kv[slot * (kRow / 2) + 32 * j + lane] = (uint8_t)((c0 + 8) | ((c1 + 8) << 4));
+      }
       if ((lane & 15) == 0) sc[2 * j + (lane >> 4)] = d;
     }
   } else {
@@ -313,6 +321,7 @@ cudaError_t launch_write_kv(const mla_write_kv_args_t* a, cudaStream_t stream) {
   const dim3 fgrid((n_tok + 3) / 4);
   if (a->kv_dtype == MLA_KV_FP8_E4M3) return launch_pdl(kv_finish_kernel<1>, fgrid, dim3(128), 0, stream, p);
   if (a->kv_dtype == MLA_KV_Q8_0) return launch_pdl(kv_finish_kernel<2>, fgrid, dim3(128), 0, stream, p);
+  if (a->kv_dtype == MLA_KV_Q4_0) return launch_pdl(kv_finish_kernel<3>, fgrid, dim3(128), 0, stream, p);
   return launch_pdl(kv_finish_kernel<0>, fgrid, dim3(128), 0, stream, p);
 }
 

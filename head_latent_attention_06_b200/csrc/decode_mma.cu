@@ -2,16 +2,17 @@
 //
 // This is the portable formulation of the decode step: legacy warp MMAs
 // (mma.sync, fp32 accumulation) with cp.async staging.  It handles every
-// supported shape (any H multiple of 16, any s_q, bf16, e4m3 or q8_0 cache) and
-// is the path for shapes the tensor-memory kernels do not take: the q8_0 cache,
-// an e4m3 scale array not on 16 bytes.
+// supported shape (any H multiple of 16, any s_q, bf16, e4m3, q8_0 or q4_0
+// cache) and is the path for shapes the tensor-memory kernels do not take: a
+// scale array not on 16 bytes.
 //
 // Cache formats.  bf16: the rows as they are.  e4m3: codes converted exactly to
 // bf16 in shared memory, the per-token scale folded into S and into P.  q8_0
 // (ik_llama.cpp docs "FlashMLA", section "KV cache with MLA"): int8 codes with
 // one fp16 scale per 32-value block; each value is formed as code * scale in
 // fp32 and rounded to bf16 in shared memory (relative error 2^-9, against the
-// format's own step of up to 1/254 of the block's largest value).
+// format's own step of up to 1/254 of the block's largest value).  q4_0: the
+// same with 4-bit codes, two a byte (value 2j in the low half of byte j).
 //
 // For one sequence b, the rows of the attention problem are the (query i,
 // head h) pairs, r = i * H + h.  A CTA owns 64 rows and one split (a range of
@@ -41,7 +42,7 @@ struct DecodeParams {
   const __nv_bfloat16* q_lat;
   const __nv_bfloat16* q_pe;
   const uint8_t* kv;
-  const void* kv_scale;  // e4m3: fp32 [pages][64]; q8_0: fp16 [pages][64][18]
+  const void* kv_scale;  // e4m3: fp32 [pages][64]; q8_0, q4_0: fp16 [pages][64][18]
   const int32_t* block_table;
   const int32_t* seq_lens;
   __nv_bfloat16* o_lat;
@@ -53,17 +54,21 @@ struct DecodeParams {
   float scale_log2;  // softmax_scale * log2(e)
 };
 
-// KIND: 0 bf16 cache, 1 e4m3 (+ fp32 token scales), 2 q8_0 (+ fp16 block scales)
+// KIND: 0 bf16 cache, 1 e4m3 (+ fp32 token scales), 2 q8_0 (+ fp16 block
+// scales), 3 q4_0 (+ fp16 block scales)
 constexpr int kQ8Blocks = kRow / 32;  // 18 scale blocks per row
+// stored bytes of one cache row
+template <int KIND>
+__host__ __device__ constexpr int row_bytes() { return KIND == 0 ? 2 * kRow : KIND == 3 ? kRow / 2 : kRow; }
 
 template <int KIND>
 struct Smem {
   static constexpr size_t q_bytes = (size_t)ROWS * CP * 2;
-  static constexpr size_t stage_bytes = KIND ? (size_t)TT * kRow : (size_t)TT * CP * 2;
+  static constexpr size_t stage_bytes = KIND ? (size_t)TT * row_bytes<KIND>() : (size_t)TT * CP * 2;
   static constexpr size_t conv_bytes = KIND ? (size_t)TT * CP * 2 : 0;
   static constexpr size_t p_bytes = (size_t)ROWS * PP * 2;
   static constexpr size_t red_bytes = 2 * ROWS * sizeof(float);
-  static constexpr size_t sc_bytes = NSTAGE * TT * (KIND == 2 ? kQ8Blocks * 2 : sizeof(float));
+  static constexpr size_t sc_bytes = NSTAGE * TT * (KIND >= 2 ? kQ8Blocks * 2 : sizeof(float));
   static constexpr size_t q_off = 0;
   static constexpr size_t stage_off = q_off + q_bytes;
   static constexpr size_t conv_off = stage_off + NSTAGE * stage_bytes;
@@ -126,11 +131,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_mma_kernel(DecodeParams p)
   auto load_tile = [&](int t, int stage) {
     unsigned char* st = stages + stage * SM::stage_bytes;
     const int jb = t * TT;
-    constexpr int VPR = CODED ? kRow / 16 : kRow / 8;  // 16-byte vectors per token row
+    constexpr int RB = row_bytes<KIND>();
+    constexpr int VPR = RB / 16;  // 16-byte vectors per token row
     for (int v = tid; v < TT * VPR; v += NTHREADS) {
       int r = v / VPR, c = v % VPR;
       int j = jb + r;
-      unsigned char* dst = CODED ? st + r * kRow + c * 16 : st + (r * CP + c * 8) * 2;
+      unsigned char* dst = CODED ? st + r * RB + c * 16 : st + (r * CP + c * 8) * 2;
       bool ok = j < j_end;
       int page = ok ? bt[j / kPage] : 0;
       if (ok && (page < 0 || page >= p.num_pages)) {
@@ -139,7 +145,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_mma_kernel(DecodeParams p)
       }
       if (ok) {
         size_t rowi = (size_t)page * kPage + (j % kPage);
-        cp_async16(dst, p.kv + rowi * kRow * (CODED ? 1 : 2) + c * 16);
+        cp_async16(dst, p.kv + rowi * RB + c * 16);
       } else {
         *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
       }
@@ -154,7 +160,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_mma_kernel(DecodeParams p)
       }
       scs[stage * TT + tid] = s;
     }
-    if (KIND == 2) {
+    if (KIND >= 2) {
       // the 18 fp16 block scales of each row: nine 4-byte words (36 bytes)
       for (int v = tid; v < TT * (kQ8Blocks / 2); v += NTHREADS) {
         const int r = v / (kQ8Blocks / 2), w = v % (kQ8Blocks / 2);
@@ -215,8 +221,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_mma_kernel(DecodeParams p)
       __nv_bfloat16* conv = reinterpret_cast<__nv_bfloat16*>(smem + SM::conv_off);
       for (int v = tid; v < TT * (kRow / 8); v += NTHREADS) {
         int r = v / (kRow / 8), c = (v % (kRow / 8)) * 8;
-        uint2 in = *reinterpret_cast<const uint2*>(raw + r * kRow + c);
         uint4 o;
+        if (KIND == 3) {
+          // 8 four-bit codes (code + 8) of one 32-value block times its scale
+          const float d = __half2float(qsc[((size_t)stage * TT + r) * kQ8Blocks + (c >> 5)]);
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(raw + r * (kRow / 2) + c / 2);
+          uint32_t out[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int lo = (int)((w >> (8 * k)) & 15u) - 8, hi = (int)((w >> (8 * k + 4)) & 15u) - 8;
+            out[k] = pack_bf16((float)lo * d, (float)hi * d);
+          }
+          o = make_uint4(out[0], out[1], out[2], out[3]);
+          *reinterpret_cast<uint4*>(conv + r * CP + c) = o;
+          continue;
+        }
+        uint2 in = *reinterpret_cast<const uint2*>(raw + r * kRow + c);
         if (KIND == 1) {
           o.x = e4m3x2_to_bf16x2((uint16_t)(in.x & 0xFFFF));
           o.y = e4m3x2_to_bf16x2((uint16_t)(in.x >> 16));
@@ -420,14 +440,19 @@ cudaError_t launch_decode_mma(const mla_decode_args_t* a, int splits, cudaStream
     e2 = cudaFuncSetAttribute(decode_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)Smem<1>::total);
     if (e2 != cudaSuccess) return e2;
-    return cudaFuncSetAttribute(decode_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)Smem<2>::total);
+    e2 = cudaFuncSetAttribute(decode_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)Smem<2>::total);
+    if (e2 != cudaSuccess) return e2;
+    return cudaFuncSetAttribute(decode_mma_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)Smem<3>::total);
   });
   if (e != cudaSuccess) return e;
   if (a->kv_dtype == MLA_KV_FP8_E4M3)
     return launch_pdl(decode_mma_kernel<1>, grid, dim3(NTHREADS), Smem<1>::total, stream, p);
   if (a->kv_dtype == MLA_KV_Q8_0)
     return launch_pdl(decode_mma_kernel<2>, grid, dim3(NTHREADS), Smem<2>::total, stream, p);
+  if (a->kv_dtype == MLA_KV_Q4_0)
+    return launch_pdl(decode_mma_kernel<3>, grid, dim3(NTHREADS), Smem<3>::total, stream, p);
   return launch_pdl(decode_mma_kernel<0>, grid, dim3(NTHREADS), Smem<0>::total, stream, p);
 }
 

@@ -1,4 +1,4 @@
-// Paged latent-attention decode over a bf16 or q8_0 cache on the 5th-generation
+// Paged latent-attention decode over a bf16, q8_0 or q4_0 cache on the 5th-generation
 // tensor cores (sm_100a): tcgen05 MMAs over a CTA pair, accumulators in tensor
 // memory (TMEM), cache pages streamed by TMA.  16 to 128 heads (fewer heads pad
 // the 128-row tile with zero rows: the step stays bound by the cache stream, so
@@ -46,8 +46,9 @@
 // P.V of t.  The output rescale is lazy: the reference maximum moves only when
 // the tile maximum exceeds it by more than 2^8, so O in TMEM is rarely touched.
 //
-// q8_0 cache (ik_llama.cpp docs "FlashMLA", section "KV cache with MLA": int8
-// codes with one fp16 scale per 32 values): the same MMAs on bf16 operands.  The
+// q8_0 and q4_0 caches (ik_llama.cpp docs "FlashMLA", section "KV cache with
+// MLA": int8 or 4-bit codes with one fp16 scale per 32 values): the same MMAs on
+// bf16 operands.  The
 // producer brings the CTA's raw codes (and their block scales) into the back half
 // of its score slot; four converter warps (12..15, 512 threads in all) read them
 // into registers, meet at a named barrier, and write the values code * scale
@@ -59,6 +60,8 @@
 // CTA that holds their columns (four to itself, four to the peer; the 128-byte
 // swizzle depends on the row mod 8 only, so the layout survives the move), and a
 // converter thread relays the landing of its CTA's value slot to the even CTA.
+// q4_0 rows are 288 bytes (two codes a byte, 9 KB of raw codes per slot); a
+// converter splits each byte into its low half (value 2j) and high half (2j + 1).
 //
 // Every mbarrier wait is bounded (MLA_ERR_DEVICE_TIMEOUT in the status word);
 // after one runs out every role leaves its loop, issued MMAs are drained, the
@@ -137,6 +140,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 // q8_0: fp16 block scales beside the ring (32 rows x 18 per score slot); raw
 // codes in the back half of each score slot
 constexpr uint32_t kQ8RowBytes = kRow;                  // 576 int8 codes
+constexpr uint32_t kQ4RowBytes = kRow / 2;              // q4_0: 576 codes, two per byte
 constexpr uint32_t kQ8ScRow = 18 * 2;                   // 36 bytes of scales per row
 constexpr uint32_t kQ8RawS = 32 * kQ8RowBytes;          // 18432: the CTA's 32 rows
 constexpr uint32_t kQ8ScS = 32 * kQ8ScRow;              // 1152
@@ -145,6 +149,7 @@ constexpr uint32_t kSmemBytesQ8 = kQ8ScOff + kSStages * kQ8ScS + 1024;
 static_assert(kSmemBytesQ8 <= 232448, "shared memory budget (q8_0)");
 static_assert(kQ8ScOff % 16 == 0 && kQ8ScS % 16 == 0, "bulk copies into the scale area start on 16 bytes");
 static_assert(kSStage == 2 * kQ8RawS, "raw codes fill the back half of a score slot");
+static_assert(kQ4RowBytes % 16 == 0, "q4_0 rows start on 16 bytes");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 256;                     // S buffers at columns 256, 288
 constexpr uint32_t kTmemQ = 320;                     // Q chunks 0..5: columns 320..511 (2 bf16 each)
@@ -159,7 +164,7 @@ struct TcParams {
   const __nv_bfloat16* q_lat;
   const __nv_bfloat16* q_pe;
   const uint8_t* kv;
-  const uint8_t* kv_scale;  // q8_0: fp16 [pages][64][18], 16-byte aligned
+  const uint8_t* kv_scale;  // q8_0, q4_0: fp16 [pages][64][18], 16-byte aligned
   const int32_t* block_table;
   const int32_t* seq_lens;
   __nv_bfloat16* o_lat;
@@ -178,9 +183,15 @@ struct TcParams {
 MLA_DEVI float q8_code(uint32_t word_flipped, int k) {
   return __int_as_float((int)__byte_perm(word_flipped, 0x4B000000u, 0x7440u + k)) - 8388736.0f;
 }
+// q4_0 value of one code: byte k of a word of 4-bit numbers (code + 8, one per
+// byte after the split into low and high halves) under the exponent of 2^23.
+MLA_DEVI float q4_code(uint32_t nibbles, int k) {
+  return __int_as_float((int)__byte_perm(nibbles, 0x4B000000u, 0x7440u + k)) - 8388616.0f;
+}
 
-template <bool Q8>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kThreads, 1)
+// KV: 0 bf16 cache; 1 q8_0 and 2 q4_0 caches, expanded to bf16 by converter warps
+template <int KV>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KV != 0 ? kThreadsQ8 : kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qpe,
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_kv,
                      const __grid_constant__ CUtensorMap tm_o, const TcParams p) {
@@ -189,6 +200,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
   const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
   uint8_t* sm = smem_raw + pad;
   const uint32_t sa = raw_addr + pad;
+  constexpr bool Q8 = KV != 0;  // a blockwise cache (q8_0 or q4_0) through the converter warps
+  constexpr bool Q4 = KV == 2;
+  constexpr uint32_t kRawRow = Q4 ? kQ4RowBytes : kQ8RowBytes;  // stored bytes of a cache row
+  constexpr uint32_t kRawS = 32 * kRawRow;                       // the CTA's 32 rows of a page
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t r = cluster_ctarank();
@@ -298,7 +313,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
       // the CTA's half page (32 contiguous rows) of tile u, into L2 ahead of its TMA
       auto prefetch = [&](int u) {
         const int pg = page_of(u, blk_p, pg_p);
-        constexpr uint32_t kRowBytes = Q8 ? kQ8RowBytes : kRow * 2;
+        constexpr uint32_t kRowBytes = Q8 ? kRawRow : kRow * 2;
         if (lane == 0) prefetch_l2_bulk(p.kv + ((size_t)pg * kPage + 32 * r) * kRowBytes, 32 * kRowBytes);
       };
       auto load_s = [&](int u) -> bool {
@@ -314,8 +329,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
           if (!mbar_wait_converged(own_bar(SRC_FREE + st), ph, abort_flag, p.status, wait_ns)) return false;
           if (lane == 0) {
             const size_t row0 = (size_t)pg * kPage + 32 * r;
-            mbar_arrive_expect_tx_local(own_bar(RAW_QS + st), kQ8RawS + kQ8ScS);
-            bulk_load_cta(dst + kQ8RawS, p.kv + row0 * kQ8RowBytes, kQ8RawS, own_bar(RAW_QS + st));
+            mbar_arrive_expect_tx_local(own_bar(RAW_QS + st), kRawS + kQ8ScS);
+            bulk_load_cta(dst + kQ8RawS, p.kv + row0 * kRawRow, kRawS, own_bar(RAW_QS + st));
             bulk_load_cta(sa + kQ8ScOff + st * kQ8ScS, p.kv_scale + row0 * kQ8ScRow, kQ8ScS,
                           own_bar(RAW_QS + st));
           }
@@ -722,7 +737,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
     }
     tc_fence_before();
   } else if constexpr (Q8) {
-    // ====================== q8_0 converters (warps 12..15) ======================
+    // ================= q8_0 / q4_0 converters (warps 12..15) =================
     // Per page: the score slot (this CTA's 32 rows x 576 values, 9 chunks of
     // 32 rows x 128 bytes, 128-byte swizzle) and the value slot (64 rows x the
     // CTA's latent chunks 2r, 2r+1, 4+2r, 5+2r, 4 chunks of 64 rows x 128 bytes).
@@ -739,11 +754,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
         const bool got = mbar_wait_converged(own_bar(RAW_QS + st), (u / kSStages) & 1, abort_flag, p.status, wait_ns);
         if (!named_bar_and(6, 32 * kConvWarps, got)) return false;
         const uint32_t slot = sa + kSOff + st * kSStage;
+        // unit i of a thread: values k0 .. k0+15 of one row (16 bytes of q8_0
+        // codes, 8 bytes of q4_0 codes)
         uint4 raw[9];
 #pragma unroll
         for (int i = 0; i < 9; ++i) {
           const int q = ct + 128 * i, row = q / 36, k0 = 16 * (q % 36);
-          raw[i] = lds128(slot + kQ8RawS + row * kQ8RowBytes + k0);
+          if constexpr (Q4) {
+            const uint2 h = lds64(slot + kQ8RawS + row * kRawRow + (k0 >> 1));
+            raw[i] = make_uint4(h.x, h.y, 0u, 0u);
+          } else {
+            raw[i] = lds128(slot + kQ8RawS + row * kRawRow + k0);
+          }
         }
         named_bar_sync(6, 32 * kConvWarps);
 #pragma unroll
@@ -751,12 +773,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Q8 ? kThreadsQ8 : kT
           const int q = ct + 128 * i, row = q / 36, k0 = 16 * (q % 36);
           const bool live = tok0 + 32 * (int)r + row < j_end;
           const float d = live ? __half2float(scs[(st * 32 + row) * 18 + (k0 >> 5)]) : 0.f;
-          const uint32_t w[4] = {raw[i].x ^ 0x80808080u, raw[i].y ^ 0x80808080u, raw[i].z ^ 0x80808080u,
-                                 raw[i].w ^ 0x80808080u};
           uint32_t o[8];
+          if constexpr (Q4) {
+            // byte m of a word holds values 2m (low half) and 2m + 1 (high half)
+            const uint32_t lo[2] = {raw[i].x & 0x0F0F0F0Fu, raw[i].y & 0x0F0F0F0Fu};
+            const uint32_t hi[2] = {(raw[i].x >> 4) & 0x0F0F0F0Fu, (raw[i].y >> 4) & 0x0F0F0F0Fu};
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            o[k] = pack_bf16(q8_code(w[k >> 1], 2 * (k & 1)) * d, q8_code(w[k >> 1], 2 * (k & 1) + 1) * d);
+            for (int k = 0; k < 8; ++k)
+              o[k] = pack_bf16(q4_code(lo[k >> 2], k & 3) * d, q4_code(hi[k >> 2], k & 3) * d);
+          } else {
+            const uint32_t w[4] = {raw[i].x ^ 0x80808080u, raw[i].y ^ 0x80808080u, raw[i].z ^ 0x80808080u,
+                                   raw[i].w ^ 0x80808080u};
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              o[k] = pack_bf16(q8_code(w[k >> 1], 2 * (k & 1)) * d, q8_code(w[k >> 1], 2 * (k & 1) + 1) * d);
+          }
           const int c = k0 >> 6, unit = (k0 & 63) >> 3;
           const uint32_t base = slot + c * kChunkS + row * 128;
           sts128(base + (((unit) ^ (row & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
@@ -897,11 +928,12 @@ cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t strea
   // score operand: (64 values, rows, 9 chunks 128 bytes apart), one box per stage;
   // value operand: (64 values, rows, 4 chunks 128 bytes apart, 2 groups 512 bytes
   // apart), one box of 2 x 2 chunks per stage
-  const bool q8 = a->kv_dtype == MLA_KV_Q8_0;
-  if (q8) {
-    // q8_0: the raw codes come by bulk copies and the value operand from the
+  const bool q8 = a->kv_dtype == MLA_KV_Q8_0, q4 = a->kv_dtype == MLA_KV_Q4_0;
+  if (q8 || q4) {
+    // q8_0, q4_0: the raw codes come by bulk copies and the value operand from the
     // converted score slots; the cache maps are not read (any valid map will do)
-    const uint64_t dq[2] = {kRow, rows_kv}, sq[1] = {kRow};
+    const uint64_t rb = q4 ? kQ4RowBytes : kQ8RowBytes;
+    const uint64_t dq[2] = {rb, rows_kv}, sq[1] = {rb};
     const uint32_t bq[2] = {128, 64};
     if (!tma_map_nd(&tm_kv, a->kv_cache, 2, dq, sq, bq, true, 0)) return cudaErrorInvalidValue;
     tm_ks = tm_kv;
@@ -944,15 +976,22 @@ cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t strea
   };
   if (q8) {
     static PerDeviceOnce attrs_q8;
-    cudaError_t e = once_per_device(attrs_q8, [&]() { return set_attrs(decode_tc_kernel<true>, kSmemBytesQ8); });
+    cudaError_t e = once_per_device(attrs_q8, [&]() { return set_attrs(decode_tc_kernel<1>, kSmemBytesQ8); });
     if (e != cudaSuccess) return e;
-    return launch_pdl(decode_tc_kernel<true>, grid, dim3(kThreadsQ8), kSmemBytesQ8, stream, tm_q, tm_qpe, tm_ks,
+    return launch_pdl(decode_tc_kernel<1>, grid, dim3(kThreadsQ8), kSmemBytesQ8, stream, tm_q, tm_qpe, tm_ks,
+                      tm_kv, tm_o, p);
+  }
+  if (q4) {
+    static PerDeviceOnce attrs_q4;
+    cudaError_t e = once_per_device(attrs_q4, [&]() { return set_attrs(decode_tc_kernel<2>, kSmemBytesQ8); });
+    if (e != cudaSuccess) return e;
+    return launch_pdl(decode_tc_kernel<2>, grid, dim3(kThreadsQ8), kSmemBytesQ8, stream, tm_q, tm_qpe, tm_ks,
                       tm_kv, tm_o, p);
   }
   static PerDeviceOnce attrs;
-  cudaError_t e = once_per_device(attrs, [&]() { return set_attrs(decode_tc_kernel<false>, kSmemBytes); });
+  cudaError_t e = once_per_device(attrs, [&]() { return set_attrs(decode_tc_kernel<0>, kSmemBytes); });
   if (e != cudaSuccess) return e;
-  return launch_pdl(decode_tc_kernel<false>, grid, dim3(kThreads), kSmemBytes, stream, tm_q, tm_qpe, tm_ks, tm_kv,
+  return launch_pdl(decode_tc_kernel<0>, grid, dim3(kThreads), kSmemBytes, stream, tm_q, tm_qpe, tm_ks, tm_kv,
                     tm_o, p);
 }
 
@@ -962,10 +1001,10 @@ cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t strea
 // an e4m3 cache) take these arguments.
 bool decode_tc_supported(const mla_decode_args_t* a) {
   // any head count up to 128 (rows beyond H pad the 128-row tile); a bf16 cache,
-  // or an e4m3 or q8_0 cache whose scale array starts on 16 bytes (bulk copies)
+  // or an e4m3, q8_0 or q4_0 cache whose scale array starts on 16 bytes (bulk copies)
   if (a->H % 16 != 0 || a->H > 128) return false;
   if (a->kv_dtype == MLA_KV_BF16) return true;
-  return (a->kv_dtype == MLA_KV_FP8_E4M3 || a->kv_dtype == MLA_KV_Q8_0) &&
+  return (a->kv_dtype == MLA_KV_FP8_E4M3 || a->kv_dtype == MLA_KV_Q8_0 || a->kv_dtype == MLA_KV_Q4_0) &&
          (reinterpret_cast<uintptr_t>(a->kv_scale) & 15u) == 0;
 }
 

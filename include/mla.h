@@ -64,8 +64,13 @@ typedef enum {
 
 /* Cache formats of a 576-value row: bf16 values; e4m3 codes with one fp32 scale
  * per row (value = code * scale); q8_0 int8 codes with one fp16 scale per block
- * of 32 consecutive values (value = code * block scale, 18 blocks a row). */
-typedef enum { MLA_KV_BF16 = 0, MLA_KV_FP8_E4M3 = 1, MLA_KV_Q8_0 = 2 } mla_kv_dtype_t;
+ * of 32 consecutive values (value = code * block scale, 18 blocks a row); q4_0
+ * the same with codes in [-7, 7], each stored as the 4-bit number code + 8, value
+ * 2j of the row in the low four bits of byte j and value 2j + 1 in the high four
+ * (288 bytes a row).  q8_0 and q4_0 follow ik_llama.cpp docs "FlashMLA", section
+ * "KV cache with MLA" (q8_0 the recommended MLA cache; below 6 bits a Hadamard
+ * rotation, see mla_fold_hadamard). */
+typedef enum { MLA_KV_BF16 = 0, MLA_KV_FP8_E4M3 = 1, MLA_KV_Q8_0 = 2, MLA_KV_Q4_0 = 3 } mla_kv_dtype_t;
 
 /* Supported dimensions: d_c = 512, d_r = 64, d_n = d_v = 128, page_size = 64,
  * H a multiple of 16 up to 128, 1 <= s_q <= MLA_MAX_S_Q.  s_q > 1 covers
@@ -101,10 +106,11 @@ typedef struct {
   const void* q_pe;               /* bf16 [B][s_q][H][d_r], RoPE already applied */
   const void* kv_cache;           /* [num_pages][page_size][d_c + d_r]: row = c || k_pe,
                                      bf16 (MLA_KV_BF16), e4m3 (MLA_KV_FP8_E4M3) or int8
-                                     (MLA_KV_Q8_0) */
+                                     (MLA_KV_Q8_0); q4_0: [num_pages][page_size][288] bytes */
   const void* kv_scale;           /* e4m3: fp32 [num_pages][page_size], the scale of the whole
-                                     row; q8_0: fp16 [num_pages][page_size][18], the scale of
-                                     each 32-value block, 4-byte aligned; NULL for bf16 */
+                                     row; q8_0, q4_0: fp16 [num_pages][page_size][18], the scale
+                                     of each 32-value block, 4-byte aligned (q4_0: 16-byte
+                                     aligned); NULL for bf16 */
   const int32_t* block_table;     /* int32 [B][max_pages_per_seq]: physical page of each
                                      64-token logical page */
   const int32_t* seq_lens;        /* int32 [B], device: cached tokens of sequence b, including
@@ -216,10 +222,11 @@ typedef struct {
                                      n_tok = B * s_q, token t = b * s_q + i */
   const void* w_dkv;              /* bf16 [d_c + d_r][d_h]: rows 0 .. d_c-1 are W_DKV, rows
                                      d_c .. d_c+d_r-1 the RoPE key's projection W_KR */
-  void* kv_cache;                 /* [num_pages][page_size][d_c + d_r], bf16 or e4m3; only the
+  void* kv_cache;                 /* [num_pages][page_size][d_c + d_r], bf16, e4m3 or q8_0
+                                     codes, or [num_pages][page_size][288] q4_0 bytes; only the
                                      new tokens' rows are written */
   void* kv_scale;                 /* written at the new rows: e4m3: fp32 [num_pages][page_size];
-                                     q8_0: fp16 [num_pages][page_size][18]; NULL for bf16 */
+                                     q8_0, q4_0: fp16 [num_pages][page_size][18]; NULL for bf16 */
   const int32_t* block_table;     /* int32 [B][max_pages_per_seq]: physical page of each
                                      64-token logical page */
   const int32_t* seq_lens;        /* int32 [B], device: lengths including the s_q new tokens */
@@ -254,6 +261,8 @@ mla_status_t mla_write_kv_workspace_size(const mla_write_kv_args_t* args, size_t
  * q8_0 cache (the format those docs recommend): per block of 32 values, d =
  * amax / 127 (computed in fp32) rounded to fp16, codes = the fp32 quotients
  * value / d rounded to nearest even, clamped to +-127 (0 for an all-zero block).
+ * q4_0 cache: the same with d = amax / 7 and codes clamped to +-7, packed two
+ * to a byte as the cache format above states.
  * The projections accumulate in fp32.  No other cache row is touched.  A length
  * below s_q or beyond the block table (MLA_ERR_BAD_SEQ_LEN) or a page id outside
  * the cache (MLA_ERR_BAD_BLOCK_TABLE) is recorded in the workspace's status word
@@ -316,6 +325,28 @@ mla_status_t mla_prefill_workspace_size(const mla_prefill_args_t* args, size_t* 
  * (MLA_ERR_BAD_BLOCK_TABLE) goes to the workspace's status word.
  */
 mla_status_t mla_prefill(const mla_prefill_args_t* args, void* stream);
+
+/*
+ * mla_fold_hadamard — folds the Hadamard rotation of the latent space into the
+ * weights, in place (ik_llama.cpp docs "FlashMLA", section "KV cache with MLA":
+ * below 6 bits a Hadamard transform of the cache before quantisation recovers
+ * quality).  With H the orthonormal Sylvester-Hadamard matrix of size d_c = 512
+ * (entries +-2^-4.5, symmetric, H H = I):
+ *   w_dkv : bf16 [d_c + d_r][d_h]; its first 512 rows W_DKV become H W_DKV (each
+ *           column transformed), so mla_write_kv stores the rotated latent H c;
+ *           the d_r RoPE rows are left as they are
+ *   w_uk  : bf16 [H_heads][d_n][d_c]; every row becomes row * H (W_UK[h] H)
+ *   w_uv  : bf16 [H_heads][d_v][d_c]; every row becomes row * H (W_UV[h] H)
+ * Attention over the rotated cache with the folded weights equals attention
+ * over the plain cache with the plain weights (H is orthonormal), and the
+ * rotation spreads a large latent channel over every block of 32, which is
+ * what a blockwise 4-bit cache needs.  Each vector is transformed in fp32 and
+ * rounded once to bf16.  Any of the three pointers may be NULL (skipped);
+ * pointers 16-byte aligned; d_h a positive multiple of 64 when w_dkv is given;
+ * H_heads 0 .. 128 (d_n = d_v = 128).  Folding twice restores the weights up
+ * to bf16 rounding.  Apply it once, before the weights are used.
+ */
+mla_status_t mla_fold_hadamard(void* w_dkv, int32_t d_h, void* w_uk, void* w_uv, int32_t H, void* stream);
 
 /* Waits for `stream`, returns the sticky device status word of `workspace`
  * (MLA_OK if no device-side problem was recorded) and clears it. */

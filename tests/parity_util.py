@@ -15,7 +15,7 @@ from oracle import mla_oracle as om
 
 # q8_0: each value is formed in bf16 from its code and block scale, so the bf16
 # cache's bounds apply (against the oracle's exact dequantised values)
-TOL = {"bf16": (2e-2, 1e-2), "fp8": (6e-2, 3e-2), "q8_0": (2e-2, 1e-2)}
+TOL = {"bf16": (2e-2, 1e-2), "fp8": (6e-2, 3e-2), "q8_0": (2e-2, 1e-2), "q4_0": (2e-2, 1e-2)}
 
 
 def errors(got: np.ndarray, ref: np.ndarray):

@@ -88,7 +88,8 @@ def test_auto_split_count(lib):
 @pytest.mark.parametrize("field,value,code", [
     ("d_c", 256, UNSUPPORTED), ("d_r", 32, UNSUPPORTED), ("page_size", 32, UNSUPPORTED),
     ("H", 24, UNSUPPORTED), ("H", 256, UNSUPPORTED), ("s_q", 1025, UNSUPPORTED),
-    ("kv_dtype", 5, UNSUPPORTED), ("H", 0, INVALID), ("s_q", 0, INVALID), ("B", -1, INVALID),
+    ("kv_dtype", 4, UNSUPPORTED), ("kv_dtype", -1, UNSUPPORTED), ("H", 0, INVALID), ("s_q", 0, INVALID),
+    ("B", -1, INVALID),
     ("num_splits", 129, INVALID), ("max_pages_per_seq", 0, INVALID),
 ])
 def test_decode_rejects_bad_shapes(lib, field, value, code):
@@ -231,7 +232,8 @@ def test_prefill_workspace_holds_keys_and_values(lib):
 
 @pytest.mark.parametrize("field,value,code", [
     ("d_c", 256, UNSUPPORTED), ("d_r", 32, UNSUPPORTED), ("page_size", 32, UNSUPPORTED),
-    ("kv_dtype", 1, UNSUPPORTED), ("kv_dtype", 2, UNSUPPORTED), ("H", 129, UNSUPPORTED),
+    ("kv_dtype", 1, UNSUPPORTED), ("kv_dtype", 2, UNSUPPORTED), ("kv_dtype", 3, UNSUPPORTED),
+    ("H", 129, UNSUPPORTED),
     ("H", 0, INVALID), ("s_q", 0, INVALID), ("B", -1, INVALID), ("max_pages_per_seq", 0, INVALID),
     ("max_seq_len", 1023, INVALID), ("softmax_scale", float("nan"), INVALID),
     ("max_seq_len", 1 << 30, UNSUPPORTED), ("B", 65536, UNSUPPORTED),
@@ -269,3 +271,26 @@ def test_prefill_with_empty_batch_enqueues_nothing(lib):
     a = _pargs(B=0)
     a.workspace, a.workspace_bytes = 0x20000, 256
     assert lib.mla_prefill(ctypes.byref(a), None) == OK
+
+
+def test_q4_0_cache_is_accepted_and_needs_scales(lib):
+    a = _args(kv_dtype=3)
+    n = ctypes.c_size_t(0)
+    assert lib.mla_decode_workspace_size(ctypes.byref(a), ctypes.byref(n)) == OK
+    a.workspace, a.workspace_bytes = 0x20000, 1 << 30
+    a.kv_scale = None
+    assert lib.mla_decode_paged(ctypes.byref(a), None) == INVALID
+    a.kv_scale = 0x30002                                                   # fp16 scales: 4-byte aligned
+    assert lib.mla_decode_paged(ctypes.byref(a), None) == MISALIGNED
+
+
+def test_fold_hadamard_argument_checks(lib):
+    f = lib.mla_fold_hadamard
+    p = 0x10000
+    assert f(None, 0, None, None, 0, None) == OK                   # nothing to fold
+    assert f(p, 7168, p, p, -1, None) == INVALID
+    assert f(p, 0, None, None, 0, None) == INVALID                 # w_dkv needs d_h > 0
+    assert f(p, 100, None, None, 0, None) == UNSUPPORTED           # d_h a multiple of 64
+    assert f(None, 0, p, p, 129, None) == UNSUPPORTED
+    assert f(p + 8, 7168, None, None, 0, None) == MISALIGNED
+    assert f(None, 0, p, p + 4, 16, None) == MISALIGNED
