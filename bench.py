@@ -577,6 +577,13 @@ def main(argv=None):
     g_absorb = st.capture(st.absorb)
     g_decode = st.capture(lambda: mla.mla_decode_paged(st.args))
     g_tail = st.capture(lambda: (mla.mla_combine_splits(st.args), st.up_project()))
+    # the same step through mla_decode_step (one launch where the shape allows)
+    from head_latent_attention_06_b200.step import FusedStep
+    fst = FusedStep(q_nope=st.q_nope, q_pe=st.q_pe, w_uk=st.w_uk, w_uv=st.w_uv, kv_cache=st._keep[0],
+                    kv_scale=st._keep[1], block_table=st._keep[2], seq_lens=st._keep[3], causal=w.causal,
+                    softmax_scale=w.softmax_scale, num_splits=args.splits,
+                    max_seq_len=max(w.lens) if w.lens else 0, fuse=1)
+    g_fused = fst.capture()
 
     def timed(graph, ev):
         flush_l2()
@@ -593,7 +600,7 @@ def main(argv=None):
     def new_events():
         return [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
 
-    evs, ev_abs, ev_dec, ev_tail = new_events(), new_events(), new_events(), new_events()
+    evs, ev_abs, ev_dec, ev_tail, ev_fused = new_events(), new_events(), new_events(), new_events(), new_events()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -610,9 +617,16 @@ def main(argv=None):
             timed(g_decode, ev_dec[k])
             timed(g_tail, ev_tail[k])
         torch.cuda.synchronize()
+        for k in range(args.steps):
+            timed(g_fused, ev_fused[k])
+        torch.cuda.synchronize()
     assert mla.mla_get_status(st.workspace) == 0
+    assert mla.mla_get_status(fst.workspace) == 0
+    g_step.replay()
+    torch.cuda.synchronize()
+    fused_same = bool(torch.equal(fst.out, st.out))
     ms = lambda ev: [e[0].elapsed_time(e[1]) for e in ev]
-    step_ms, dec_ms, absorb_ms, tail_ms = ms(evs), ms(ev_dec), ms(ev_abs), ms(ev_tail)
+    step_ms, dec_ms, absorb_ms, tail_ms, fused_ms = ms(evs), ms(ev_dec), ms(ev_abs), ms(ev_tail), ms(ev_fused)
     total_ms = reduce_max(sum(step_ms))
     dec_avg_ms = reduce_max(sum(dec_ms) / len(dec_ms))
     ms_per_step = total_ms / args.steps
@@ -706,6 +720,11 @@ def main(argv=None):
         "decode_us": round(dec_avg_ms * 1e3, 2),
         "absorb_us": round(1e3 * sum(absorb_ms) / len(absorb_ms), 2),
         "combine_up_proj_us": round(1e3 * sum(tail_ms) / len(tail_ms), 2),
+        # mla_decode_step with fuse = 1: the same step in one call (one launch
+        # where the shape allows), timed the same way; its output equals the
+        # four-kernel step's bit for bit
+        "fused_step": {"us": round(1e3 * reduce_max(sum(fused_ms)) / len(fused_ms), 2),
+                       "launches": fst.launches, "same_output": fused_same},
         "roofline": {
             # the binding side: cache bytes at the HBM copy bandwidth, or the
             # algorithmic FLOPs at the tensor peak of the MMA kind used

@@ -33,7 +33,7 @@ EXPORTS = ("mla_absorb_q", "mla_decode_workspace_size", "mla_decode_num_splits",
            "mla_status_string", "mla_decode_paged_noalloc", "mla_noalloc_init",
            "mla_get_status_noalloc", "mla_write_kv_workspace_size", "mla_write_kv",
            "mla_set_decode_kernel", "mla_set_device_wait_limit", "mla_fold_hadamard", "mla_prefill_workspace_size",
-           "mla_prefill")
+           "mla_prefill", "mla_decode_step_workspace_size", "mla_decode_step_launches", "mla_decode_step")
 
 DECODE_AUTO, DECODE_WARP_MMA = 0, 1
 
@@ -92,6 +92,23 @@ class PrefillArgs(ctypes.Structure):
     ]
 
 
+class StepArgs(ctypes.Structure):
+    """Mirror of ``mla_step_args_t`` (field order and types must match)."""
+    _fields_ = [
+        ("q_nope", ctypes.c_void_p), ("q_pe", ctypes.c_void_p),
+        ("w_uk", ctypes.c_void_p), ("w_uv", ctypes.c_void_p),
+        ("kv_cache", ctypes.c_void_p), ("kv_scale", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+        ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("B", ctypes.c_int32), ("s_q", ctypes.c_int32), ("H", ctypes.c_int32),
+        ("d_c", ctypes.c_int32), ("d_r", ctypes.c_int32), ("page_size", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
+        ("kv_dtype", ctypes.c_int32), ("causal", ctypes.c_int32), ("num_splits", ctypes.c_int32),
+        ("max_seq_len", ctypes.c_int32), ("softmax_scale", ctypes.c_float), ("fuse", ctypes.c_int32),
+    ]
+
+
 _lib: Optional[ctypes.CDLL] = None
 
 
@@ -123,6 +140,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_prefill_workspace_size.argtypes = [pp, ctypes.POINTER(ctypes.c_size_t)]
     lib.mla_prefill.argtypes = [pp, vp]
     lib.mla_get_status.argtypes = [vp, vp]
+    ps = ctypes.POINTER(StepArgs)
+    lib.mla_decode_step_workspace_size.argtypes = [ps, ctypes.POINTER(ctypes.c_size_t)]
+    lib.mla_decode_step_launches.argtypes = [ps, ctypes.POINTER(ctypes.c_int32)]
+    lib.mla_decode_step.argtypes = [ps, vp]
     lib.mla_fold_hadamard.argtypes = [vp, i32, vp, vp, i32, vp]
     lib.mla_status_string.argtypes = [ctypes.c_int]
     lib.mla_status_string.restype = ctypes.c_char_p
@@ -376,6 +397,71 @@ def mla_write_kv(args: WriteKvArgs, stream=None):
     _check("mla_write_kv", load().mla_write_kv(ctypes.byref(args), _stream(stream)))
 
 
+def make_step_args(*, q_nope, q_pe, w_uk, w_uv, kv_cache, kv_scale, block_table, seq_lens, out, lse,
+                   workspace=None, causal=False, softmax_scale, num_splits=0, max_seq_len=0,
+                   fuse=0) -> StepArgs:
+    """Fill a ``StepArgs`` (the whole decode step, ``mla_decode_step``) from device
+    tensors.  Shapes: q_nope [B][s_q][H][128], q_pe [B][s_q][H][64], w_uk and w_uv
+    [H][128][512] bf16; the cache, scales, block table and lengths as for
+    ``make_decode_args``; out [B][s_q][H][128] bf16, lse [B][s_q][H] fp32 or None;
+    fuse: 0 automatic, 1 one launch wherever possible, -1 never."""
+    import torch
+    bf16, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    if q_nope.dim() != 4 or kv_cache.dim() != 3 or block_table.dim() != 2:
+        raise ValueError("q_nope must be [B][s_q][H][128], kv_cache [pages][64][row], block_table [B][pages]")
+    B, s_q, H, _ = q_nope.shape
+    P = kv_cache.shape[0]
+    kind, sc_dtype, sc_tail, width = _cache_kind(kv_cache)
+    _want([(q_nope, "q_nope", bf16, (B, s_q, H, D_N), False),
+           (q_pe, "q_pe", bf16, (B, s_q, H, D_R), False),
+           (w_uk, "w_uk", bf16, (H, D_N, D_C), False),
+           (w_uv, "w_uv", bf16, (H, D_V, D_C), False),
+           (kv_cache, "kv_cache", (bf16, torch.float8_e4m3fn, torch.int8, torch.uint8), (P, PAGE, width), False),
+           (kv_scale, "kv_scale", sc_dtype or f32, (P, PAGE) + sc_tail, kind == KV_BF16),
+           (block_table, "block_table", i32, (B, block_table.shape[1]), False),
+           (seq_lens, "seq_lens", i32, (B,), False),
+           (out, "out", bf16, (B, s_q, H, D_V), False),
+           (lse, "lse", f32, (B, s_q, H), True),
+           (workspace, "workspace", torch.uint8, None, True)])
+    a = StepArgs()
+    a.q_nope, a.q_pe, a.w_uk, a.w_uv = _ptr(q_nope), _ptr(q_pe), _ptr(w_uk), _ptr(w_uv)
+    a.kv_cache, a.kv_scale = _ptr(kv_cache), _ptr(kv_scale)
+    a.block_table, a.seq_lens = _ptr(block_table), _ptr(seq_lens)
+    a.out, a.lse = _ptr(out), _ptr(lse)
+    a.B, a.s_q, a.H = B, s_q, H
+    a.d_c, a.d_r, a.page_size = D_C, D_R, PAGE
+    a.num_pages = P
+    a.max_pages_per_seq = block_table.shape[1]
+    a.kv_dtype = kind
+    a.causal = int(bool(causal))
+    a.num_splits = int(num_splits)
+    a.max_seq_len = int(max_seq_len)
+    a.softmax_scale = float(softmax_scale)
+    a.fuse = int(fuse)
+    if workspace is not None:
+        a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    return a
+
+
+def mla_decode_step_workspace_size(args: StepArgs) -> int:
+    n = ctypes.c_size_t(0)
+    _check("mla_decode_step_workspace_size",
+           load().mla_decode_step_workspace_size(ctypes.byref(args), ctypes.byref(n)))
+    return int(n.value)
+
+
+def mla_decode_step_launches(args: StepArgs) -> int:
+    """Kernel launches one mla_decode_step call makes (1: fused)."""
+    n = ctypes.c_int32(0)
+    _check("mla_decode_step_launches", load().mla_decode_step_launches(ctypes.byref(args), ctypes.byref(n)))
+    return int(n.value)
+
+
+def mla_decode_step(args: StepArgs, stream=None):
+    """The whole decode step (absorption, decode, split merge, up-projection)."""
+    _check("mla_decode_step", load().mla_decode_step(ctypes.byref(args), _stream(stream)))
+
+
 def make_prefill_args(*, q_nope, q_pe, w_uk, w_uv, kv_cache, block_table, seq_lens, out, lse,
                       max_seq_len, workspace=None, causal=True, softmax_scale) -> PrefillArgs:
     """Fill a ``PrefillArgs`` from device tensors.  Shapes: q_nope [B][s_q][H][128],
@@ -444,6 +530,8 @@ def alloc_workspace(args, device="cuda"):
     import torch
     if isinstance(args, WriteKvArgs):
         n = mla_write_kv_workspace_size(args)
+    elif isinstance(args, StepArgs):
+        n = mla_decode_step_workspace_size(args)
     elif isinstance(args, PrefillArgs):
         n = mla_prefill_workspace_size(args)
     else:

@@ -24,6 +24,9 @@ cudaError_t launch_write_kv(const mla_write_kv_args_t*, cudaStream_t);
 size_t prefill_workspace_bytes(int B, int H, int Lmax);
 cudaError_t launch_prefill(const mla_prefill_args_t*, cudaStream_t);
 cudaError_t launch_fold_hadamard(void*, int, void*, void*, int, cudaStream_t);
+bool decode_step_fusable(const mla_decode_args_t*, int splits);
+size_t decode_step_flag_bytes();
+cudaError_t launch_decode_step_fused(const mla_decode_args_t*, const StepOperands*, cudaStream_t);
 }  // namespace mla
 
 using namespace mla;
@@ -153,6 +156,62 @@ namespace mla {
 uint64_t device_wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 }  // namespace mla
 
+// ---- the whole step: the decode's arguments with q_lat and o_lat in the step's
+// workspace, laid out after the decode's own part and the step's flags
+namespace {
+struct StepLayout {
+  size_t flags_off, q_lat_off, o_lat_off, total;
+};
+
+mla_decode_args_t step_decode_args(const mla_step_args_t* s) {
+  mla_decode_args_t d;
+  memset(&d, 0, sizeof(d));
+  d.q_pe = s->q_pe;
+  d.kv_cache = s->kv_cache;
+  d.kv_scale = s->kv_scale;
+  d.block_table = s->block_table;
+  d.seq_lens = s->seq_lens;
+  d.lse = s->lse;
+  d.workspace = s->workspace;
+  d.workspace_bytes = s->workspace_bytes;
+  d.B = s->B;
+  d.s_q = s->s_q;
+  d.H = s->H;
+  d.d_c = s->d_c;
+  d.d_r = s->d_r;
+  d.page_size = s->page_size;
+  d.num_pages = s->num_pages;
+  d.max_pages_per_seq = s->max_pages_per_seq;
+  d.kv_dtype = s->kv_dtype;
+  d.causal = s->causal;
+  d.num_splits = s->num_splits;
+  d.max_seq_len = s->max_seq_len;
+  d.softmax_scale = s->softmax_scale;
+  return d;
+}
+
+StepLayout step_layout(const mla_decode_args_t* d, int splits) {
+  StepLayout L;
+  const size_t lat = (size_t)d->B * d->s_q * d->H * kDc * 2;
+  L.flags_off = align_up(workspace_bytes(d, splits), 256);
+  L.q_lat_off = align_up(L.flags_off + decode_step_flag_bytes(), 256);
+  L.o_lat_off = align_up(L.q_lat_off + lat, 256);
+  L.total = align_up(L.o_lat_off + lat, 256);
+  return L;
+}
+
+// One launch: forced (fuse = 1) wherever the fused kernel takes the shape; by
+// default only where it measured faster than the four launches chained by
+// programmatic dependent launch: the q8_0 and q4_0 caches, whose decode is
+// bound by its converter warps, with a grid covering at least half the SMs
+// (with fewer CTAs the projection tiles queue up on them).
+bool step_fused(const mla_step_args_t* s, const mla_decode_args_t* d, int splits) {
+  if (s->fuse < 0 || !use_tc(d) || !decode_step_fusable(d, splits)) return false;
+  if (s->fuse > 0) return true;
+  return d->kv_dtype != MLA_KV_BF16 && 4 * d->B * d->s_q >= device_sm_count();
+}
+}  // namespace
+
 extern "C" {
 
 mla_status_t mla_absorb_q(const void* q_nope, const void* w_uk, void* q_lat, int32_t n_tok,
@@ -249,6 +308,61 @@ mla_status_t mla_write_kv(const mla_write_kv_args_t* a, void* stream) {
       (reinterpret_cast<uintptr_t>(a->kv_scale) & 3u))
     return MLA_ERR_MISALIGNED;
   return from_cuda(launch_write_kv(a, (cudaStream_t)stream));
+}
+
+mla_status_t mla_decode_step_workspace_size(const mla_step_args_t* a, size_t* bytes) {
+  if (!a) return MLA_ERR_INVALID_VALUE;
+  const mla_decode_args_t d = step_decode_args(a);
+  mla_status_t st = check_decode_shape(&d);
+  if (st != MLA_OK) return st;
+  if (!bytes) return MLA_ERR_INVALID_VALUE;
+  *bytes = step_layout(&d, choose_splits(&d)).total;
+  return MLA_OK;
+}
+
+mla_status_t mla_decode_step_launches(const mla_step_args_t* a, int32_t* launches) {
+  if (!a) return MLA_ERR_INVALID_VALUE;
+  const mla_decode_args_t d = step_decode_args(a);
+  mla_status_t st = check_decode_shape(&d);
+  if (st != MLA_OK) return st;
+  if (!launches) return MLA_ERR_INVALID_VALUE;
+  const int splits = choose_splits(&d);
+  *launches = a->B == 0 ? 0 : step_fused(a, &d, splits) ? 1 : splits > 1 ? 4 : 3;
+  return MLA_OK;
+}
+
+mla_status_t mla_decode_step(const mla_step_args_t* a, void* stream) {
+  if (!a) return MLA_ERR_INVALID_VALUE;
+  mla_decode_args_t d = step_decode_args(a);
+  mla_status_t st = check_decode_shape(&d);
+  if (st != MLA_OK) return st;
+  const int splits = choose_splits(&d);
+  const StepLayout L = step_layout(&d, splits);
+  if (!a->workspace) return MLA_ERR_INVALID_VALUE;
+  if (!aligned16(a->workspace)) return MLA_ERR_MISALIGNED;
+  if (a->workspace_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (a->B == 0) return MLA_OK;
+  if (!a->q_nope || !a->w_uk || !a->w_uv || !a->out) return MLA_ERR_INVALID_VALUE;
+  if (!aligned16(a->q_nope) || !aligned16(a->w_uk) || !aligned16(a->w_uv) || !aligned16(a->out))
+    return MLA_ERR_MISALIGNED;
+  unsigned char* ws = static_cast<unsigned char*>(a->workspace);
+  d.q_lat = ws + L.q_lat_off;
+  d.o_lat = ws + L.o_lat_off;
+  st = check_decode_ptrs(&d, splits);
+  if (st != MLA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int n_tok = a->B * a->s_q;
+  if (step_fused(a, &d, splits)) {
+    const StepOperands fx = {a->q_nope, a->w_uk, a->w_uv, a->out, reinterpret_cast<uint32_t*>(ws + L.flags_off)};
+    return from_cuda(launch_decode_step_fused(&d, &fx, s));
+  }
+  cudaError_t e = launch_absorb_q(a->q_nope, a->w_uk, ws + L.q_lat_off, n_tok, a->H, s);
+  if (e == cudaSuccess)
+    e = use_tc(&d) ? (d.kv_dtype == MLA_KV_FP8_E4M3 ? launch_decode_f8(&d, splits, s) : launch_decode_tc(&d, splits, s))
+                   : launch_decode_mma(&d, splits, s);
+  if (e == cudaSuccess && splits > 1) e = launch_combine(&d, splits, s);
+  if (e == cudaSuccess) e = launch_up_proj_v(d.o_lat, a->w_uv, a->out, n_tok, a->H, s);
+  return from_cuda(e);
 }
 
 mla_status_t mla_fold_hadamard(void* w_dkv, int32_t d_h, void* w_uk, void* w_uv, int32_t H, void* stream) {

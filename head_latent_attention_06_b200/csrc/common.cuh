@@ -23,6 +23,17 @@ constexpr int kDn = 128;
 constexpr int kDv = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 
+// The fused decode step's operands beyond the decode's own (q_lat and o_lat are
+// then buffers of the step's workspace): q_nope, W_UK, W_UV, the output, and the
+// flags between the step's phases.
+struct StepOperands {
+  const void* q_nope;
+  const void* w_uk;
+  const void* w_uv;
+  void* out;
+  uint32_t* flags;
+};
+
 // Layout of the decode workspace: a 256-byte header holding the sticky status
 // word, then fp32 partial outputs [n_tok][H][S][d_c] and partial lse
 // [n_tok][H][S], each 256-byte aligned.

@@ -72,6 +72,7 @@
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
+#include "proj_tile.cuh"
 #include "sm100.cuh"
 #include "tma_host.cuh"
 
@@ -175,7 +176,112 @@ struct TcParams {
   int B, s_q, H, num_pages, max_pages, causal, splits;
   float scale_log2;
   uint64_t wait_ns;
+  // fused step only: the absorption's output (q_lat, read back through tm_q),
+  // the up-projection's output, and the flags between the phases (workspace)
+  __nv_bfloat16* q_lat_out;
+  __nv_bfloat16* out;
+  uint32_t* ready;       // [token blocks]: absorption tiles done
+  uint32_t* done;        // [token blocks]: decode CTAs whose o_lat rows are written
+  uint32_t* exit_count;  // CTAs that have finished
+  int n_tok;
 };
+
+// ---------------------------------------------------------------- fused step
+// The decode step in one launch (every CTA of the grid resident at once: the
+// host launches it only when the grid fits the SMs): each CTA first takes a
+// share of the query absorption (tiles of 64 tokens x one head x 128 latent
+// columns, three groups of four warps per CTA), then decodes its work unit as
+// the standalone kernel does, its producer waiting until every absorption tile
+// of its token block is written before it requests Q; after its epilogue each
+// CTA counts its o_lat rows as written, and finally takes a share of the value
+// up-projection (tiles of 64 tokens x one head x 32 output columns), each tile
+// waiting until every decode CTA of its token block has counted.  The weights
+// are read once per token block, not once per query token.  The last CTA to
+// finish clears the flags for the next launch.
+constexpr int kPhaseGroups = 3;                 // groups of four warps (warps 0..11)
+constexpr uint32_t kPhaseRing = 48 * 1024;      // shared memory of one group
+constexpr int kMaxStepBlocks = 16;              // token blocks of 64 the flags hold
+static_assert(kPhaseGroups * kPhaseRing <= kPOff, "projection rings below the P buffers");
+static_assert(proj::Cfg<kDn, kDc, 128, true, 2>::RING <= kPhaseRing &&
+                  proj::Cfg<kDc, kDv, 32, false, 4>::RING <= kPhaseRing,
+              "a projection tile fits its group's ring");
+
+MLA_DEVI bool group_any(int bar_id, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(bar_id)
+      : "memory");
+  return r != 0;
+}
+
+// One projection phase of the fused step (ABSORB: q_lat = W_UK^T q_nope; else
+// out = W_UV o_lat) over all CTAs of the grid.  Every thread of the CTA calls it.
+template <bool ABSORB>
+MLA_DEVI void step_phase(const CUtensorMap* tm_x, const CUtensorMap* tm_w, const TcParams& p, uint32_t sa,
+                         uint8_t* sm) {
+  const int warp = threadIdx.x >> 5;
+  const int group = warp / 4;
+  const uint32_t bars = sa + kPOff;  // per group: 4 stage barriers
+  if (threadIdx.x == 0) {
+    for (int g = 0; g < kPhaseGroups; ++g)
+      for (int s = 0; s < 4; ++s) mbar_init(bars + 64 * g + 8 * s, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (group < kPhaseGroups) {
+    const int gtid = threadIdx.x - 128 * group, bar_id = 13 + group;
+    const int cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    const int n_ctas = gridDim.x * gridDim.y * gridDim.z;
+    const int n_blocks = (p.n_tok + 63) / 64;
+    const int n_tiles = n_blocks * p.H * 4;  // 4 column slices: 512 / 128 or 128 / 32
+    const uint32_t ring = sa + group * kPhaseRing;
+    uint8_t* ring_g = sm + group * kPhaseRing;
+    const uint32_t bar0 = bars + 64 * group;
+    int abort = 0;
+    uint32_t iter = 0;
+    for (int tau = cta * kPhaseGroups + group; tau < n_tiles; tau += n_ctas * kPhaseGroups, ++iter) {
+      const int tb = tau / (p.H * 4), rem = tau - tb * (p.H * 4), h = rem >> 2, sl = rem & 3;
+      if constexpr (ABSORB) {
+        proj::tile<kDn, kDc, 128, true, 2>(tm_x, tm_w, p.q_lat_out, p.n_tok, p.H, 64 * tb, h, 128 * sl, ring,
+                                           ring_g, bar0, iter, gtid, bar_id, []() {}, abort, p.status);
+        // the tile's stores (every thread of the group, ordered by the tile's last
+        // group barrier) are published before the count
+        if (gtid == 0) {
+          fence_proxy_async_all();
+          __threadfence();
+          red_release_gpu_add(p.ready + tb, 1u);
+        }
+      } else {
+        const uint32_t need = 2u * (uint32_t)min(64, p.n_tok - 64 * tb);
+        // a wait that runs out is recorded and the tile goes on (on rows that may
+        // not be written yet): every copy it requests still lands before the CTA
+        // moves on, as on the normal path
+        proj::tile<kDc, kDv, 32, false, 4>(tm_x, tm_w, p.out, p.n_tok, p.H, 64 * tb, h, 32 * sl, ring, ring_g,
+                                           bar0, iter, gtid, bar_id,
+                                           [&]() {
+                                             if (!wait_counter_geq(p.done + tb, need, p.wait_ns))
+                                               set_status(p.status, MLA_ERR_DEVICE_TIMEOUT);
+                                             fence_proxy_async_all();
+                                           },
+                                           abort, p.status);
+      }
+      // a group that gave up leaves together (its stage barriers are out of step)
+      if (group_any(bar_id, abort != 0)) break;
+    }
+  }
+  // generic stores into shared memory before the asynchronous proxy writes there again
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int g = 0; g < kPhaseGroups; ++g)
+      for (int s = 0; s < 4; ++s) mbar_inval(bars + 64 * g + 8 * s);
+  __syncthreads();
+}
 
 // q8_0 value of one code: the byte with its sign bit flipped, put under the
 // exponent of 2^23, is 2^23 + 128 + code exactly; subtracting gives the code,
@@ -189,12 +295,16 @@ MLA_DEVI float q4_code(uint32_t nibbles, int k) {
   return __int_as_float((int)__byte_perm(nibbles, 0x4B000000u, 0x7440u + k)) - 8388616.0f;
 }
 
-// KV: 0 bf16 cache; 1 q8_0 and 2 q4_0 caches, expanded to bf16 by converter warps
-template <int KV>
+// KV: 0 bf16 cache; 1 q8_0 and 2 q4_0 caches, expanded to bf16 by converter warps.
+// FUSED: the whole decode step (absorption, decode, up-projection) in one launch;
+// tm_qn, tm_wuk, tm_ol, tm_wuv are its projection operands (unused otherwise).
+template <int KV, bool FUSED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KV != 0 ? kThreadsQ8 : kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qpe,
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_kv,
-                     const __grid_constant__ CUtensorMap tm_o, const TcParams p) {
+                     const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_qn,
+                     const __grid_constant__ CUtensorMap tm_wuk, const __grid_constant__ CUtensorMap tm_ol,
+                     const __grid_constant__ CUtensorMap tm_wuv, const TcParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
@@ -272,6 +382,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KV != 0 ? kThreadsQ8
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_trigger();
+  if constexpr (FUSED) {
+    // q_nope, the weights and the workspace may come from or be read by the
+    // kernels before this one
+    pdl_wait();
+    step_phase<true>(&tm_qn, &tm_wuk, p, sa, sm);
+  }
 
   // ---- the work unit: tiles [t0, t1) of sequence b, query g
   const bool bad_len = L_in < 0 || L_in > p.max_pages * kPage;
@@ -398,7 +514,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KV != 0 ? kThreadsQ8
       // the same moment, and these two gate the first score MMA; the L2
       // prefetch of the next pages only after them
       bool ok = load_s(0);
-      pdl_wait();
+      if constexpr (FUSED) {
+        // every absorption tile of this token's block written (by any CTA).  A wait
+        // that runs out is recorded and Q is requested all the same (both CTAs of
+        // the pair then keep the same count of copies on the pair's barriers).
+        if (lane == 0) {
+          if (!wait_counter_geq(p.ready + (b * p.s_q + g) / 64, 4u * (uint32_t)p.H, wait_ns))
+            set_status(p.status, MLA_ERR_DEVICE_TIMEOUT);
+          fence_proxy_async_all();
+        }
+        __syncwarp();
+      } else {
+        pdl_wait();
+      }
       if (lane == 0) {
         // 3-D maps (values, heads, query tokens): heads >= H come in as zeros.
         // Chunks 6.. (the MMA's shared-memory A operand) into the Q region; chunks
@@ -725,7 +853,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KV != 0 ? kThreadsQ8
         const int qtok = b * p.s_q + g;
         for (int c = 0; c < 8; ++c) tma_store_3d(&tm_o, sa + kSOff + c * (64 * 128), 64 * c, 64 * (int)r, qtok);
         bulk_commit_group();
-        bulk_wait_read<0>();  // the staging area may be released; the writes finish with the grid
+        if constexpr (FUSED) {
+          // the rows are read by other CTAs of this grid: written, then counted
+          bulk_wait_all();
+          fence_proxy_async_all();
+          __threadfence();
+          red_release_gpu_add(p.done + qtok / 64, 1u);
+        } else {
+          bulk_wait_read<0>();  // the staging area may be released; the writes finish with the grid
+        }
       }
     }
     if (half == 0 && ch == 0 && row_ok) {
@@ -913,10 +1049,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KV != 0 ? kThreadsQ8
   cluster_arrive();
   cluster_wait();
   if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
+  if constexpr (FUSED) {
+    __syncthreads();
+    step_phase<false>(&tm_ol, &tm_wuv, p, sa, sm);
+    // the last CTA out clears the flags for the next launch (every CTA is past
+    // its last use of them once it has counted itself here)
+    if (threadIdx.x == 0) {
+      __threadfence();
+      const uint32_t n_ctas = gridDim.x * gridDim.y * gridDim.z;
+      if (atomicAdd(p.exit_count, 1u) == n_ctas - 1) {
+        const int n_blocks = (p.n_tok + 63) / 64;
+        for (int i = 0; i < n_blocks; ++i) {
+          p.ready[i] = 0u;
+          p.done[i] = 0u;
+        }
+        *p.exit_count = 0u;
+        __threadfence();
+      }
+    }
+  }
 }
 
 // ---------------------------------------------------------------- host side
-cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t stream) {
+// One instance's launch: the kernel attributes once per device, then the launch.
+template <int KV, bool F>
+cudaError_t launch_inst(dim3 grid, const CUtensorMap (&m)[9], const TcParams& p, cudaStream_t stream) {
+  constexpr uint32_t threads = KV != 0 ? kThreadsQ8 : kThreads;
+  constexpr uint32_t smem = KV != 0 ? kSmemBytesQ8 : kSmemBytes;
+  static PerDeviceOnce attrs;
+  cudaError_t e = once_per_device(attrs, [&]() {
+    cudaError_t e2 = cudaFuncSetAttribute(decode_tc_kernel<KV, F>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)smem);
+    if (e2 != cudaSuccess) return e2;
+    return cudaFuncSetAttribute(decode_tc_kernel<KV, F>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  });
+  if (e != cudaSuccess) return e;
+  return launch_pdl(decode_tc_kernel<KV, F>, grid, dim3(threads), smem, stream, m[0], m[1], m[2], m[3], m[4], m[5],
+                    m[6], m[7], m[8], p);
+}
+
+// fx: the fused step's extra operands (nullptr: the decode alone)
+cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t stream,
+                      const StepOperands* fx = nullptr) {
   CUtensorMap tm_q, tm_qpe, tm_ks, tm_kv, tm_o;  // tm_o: o_lat, the single-split result
   const uint64_t rows_kv = (uint64_t)a->num_pages * kPage;
   const int n_tok = a->B * a->s_q;
@@ -968,31 +1142,35 @@ cudaError_t launch_tc(const mla_decode_args_t* a, int splits, cudaStream_t strea
   p.splits = splits;
   p.scale_log2 = a->softmax_scale * kLog2e;
   p.wait_ns = device_wait_limit_ns();
-  dim3 grid(2 * splits, a->s_q, a->B);
-  auto set_attrs = [](auto kern, uint32_t smem) {
-    cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e2 != cudaSuccess) return e2;
-    return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-  };
-  if (q8) {
-    static PerDeviceOnce attrs_q8;
-    cudaError_t e = once_per_device(attrs_q8, [&]() { return set_attrs(decode_tc_kernel<1>, kSmemBytesQ8); });
-    if (e != cudaSuccess) return e;
-    return launch_pdl(decode_tc_kernel<1>, grid, dim3(kThreadsQ8), kSmemBytesQ8, stream, tm_q, tm_qpe, tm_ks,
-                      tm_kv, tm_o, p);
+  p.n_tok = n_tok;
+  p.q_lat_out = nullptr;
+  p.out = nullptr;
+  p.ready = p.done = p.exit_count = nullptr;
+  // the fused step's projection operands: absorption X = q_nope (values, heads,
+  // tokens; 64-token boxes) and W_UK (512 columns, H x 128 rows); up-projection
+  // X = o_lat and W_UV (512 columns, H x 128 rows, 32-row boxes)
+  CUtensorMap m[9] = {tm_q, tm_qpe, tm_ks, tm_kv, tm_o, tm_q, tm_q, tm_q, tm_q};
+  if (fx) {
+    if (!tma_map_3d(&m[5], fx->q_nope, kDn, a->H, n_tok, kDn * 2, (uint64_t)a->H * kDn * 2, 64, 1, proj::TM) ||
+        !tma_map_2d(&m[6], fx->w_uk, kDc, (uint64_t)a->H * kDn, kDc * 2, 64, proj::TK) ||
+        !tma_map_3d(&m[7], a->o_lat, kDc, a->H, n_tok, kDc * 2, (uint64_t)a->H * kDc * 2, 64, 1, proj::TM) ||
+        !tma_map_2d(&m[8], fx->w_uv, kDc, (uint64_t)a->H * kDv, kDc * 2, 64, 32))
+      return cudaErrorInvalidValue;
+    p.q_lat_out = static_cast<__nv_bfloat16*>(const_cast<void*>(a->q_lat));
+    p.out = static_cast<__nv_bfloat16*>(fx->out);
+    p.ready = fx->flags;
+    p.done = fx->flags + kMaxStepBlocks;
+    p.exit_count = fx->flags + 2 * kMaxStepBlocks;
   }
-  if (q4) {
-    static PerDeviceOnce attrs_q4;
-    cudaError_t e = once_per_device(attrs_q4, [&]() { return set_attrs(decode_tc_kernel<2>, kSmemBytesQ8); });
-    if (e != cudaSuccess) return e;
-    return launch_pdl(decode_tc_kernel<2>, grid, dim3(kThreadsQ8), kSmemBytesQ8, stream, tm_q, tm_qpe, tm_ks,
-                      tm_kv, tm_o, p);
+  const dim3 grid(2 * splits, a->s_q, a->B);
+  if (fx) {
+    if (q8) return launch_inst<1, true>(grid, m, p, stream);
+    if (q4) return launch_inst<2, true>(grid, m, p, stream);
+    return launch_inst<0, true>(grid, m, p, stream);
   }
-  static PerDeviceOnce attrs;
-  cudaError_t e = once_per_device(attrs, [&]() { return set_attrs(decode_tc_kernel<0>, kSmemBytes); });
-  if (e != cudaSuccess) return e;
-  return launch_pdl(decode_tc_kernel<0>, grid, dim3(kThreads), kSmemBytes, stream, tm_q, tm_qpe, tm_ks, tm_kv,
-                    tm_o, p);
+  if (q8) return launch_inst<1, false>(grid, m, p, stream);
+  if (q4) return launch_inst<2, false>(grid, m, p, stream);
+  return launch_inst<0, false>(grid, m, p, stream);
 }
 
 }  // namespace
@@ -1012,6 +1190,54 @@ int decode_tc_clusters_per_split(const mla_decode_args_t* a) { return a->B * a->
 
 cudaError_t launch_decode_tc(const mla_decode_args_t* a, int splits, cudaStream_t stream) {
   return launch_tc(a, splits, stream);
+}
+
+// CTA pairs of the fused kernel the current device holds at once (0 if unknown),
+// queried once per device: the GPCs decide how many pairs fit, not the SM count.
+int fused_cluster_capacity(bool coded) {
+  static PerDeviceOnce once[2];
+  static std::atomic<int> cap[2][PerDeviceOnce::kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= PerDeviceOnce::kMaxDevices) return 0;
+  once_per_device(once[coded], [&]() {
+    auto kern = coded ? decode_tc_kernel<1, true> : decode_tc_kernel<0, true>;
+    const uint32_t smem = coded ? kSmemBytesQ8 : kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(coded ? kThreadsQ8 : kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e == cudaSuccess) cap[coded][dev].store(n, std::memory_order_relaxed);
+    return e;
+  });
+  return cap[coded][dev].load(std::memory_order_relaxed);
+}
+
+// The fused step takes one split, a cache this kernel reads, a grid whose CTA
+// pairs the device holds all at once (one pair per query token) and token
+// blocks the flags hold.
+bool decode_step_fusable(const mla_decode_args_t* a, int splits) {
+  const int n_tok = a->B * a->s_q;
+  if (!(splits == 1 && a->kv_dtype != MLA_KV_FP8_E4M3 && decode_tc_supported(a) && n_tok > 0 &&
+        (n_tok + 63) / 64 <= kMaxStepBlocks))
+    return false;
+  return n_tok <= fused_cluster_capacity(a->kv_dtype != MLA_KV_BF16);
+}
+
+size_t decode_step_flag_bytes() { return 3 * kMaxStepBlocks * sizeof(uint32_t); }
+
+cudaError_t launch_decode_step_fused(const mla_decode_args_t* a, const StepOperands* fx, cudaStream_t stream) {
+  return launch_tc(a, 1, stream, fx);
 }
 
 }  // namespace mla

@@ -307,6 +307,29 @@ MLA_DEVI void sts128(uint32_t addr, uint4 v) {
                : "memory");
 }
 
+// Flags between CTAs of one grid: an acquire load, a release add, and a bounded
+// wait for a counter to reach a value (false once limit_ns has passed).
+MLA_DEVI uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+MLA_DEVI void red_release_gpu_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+MLA_DEVI bool wait_counter_geq(const uint32_t* ctr, uint32_t target, uint64_t limit_ns) {
+  if (ld_acquire_gpu(ctr) >= target) return true;
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    if (globaltimer() - t0 > limit_ns) return false;
+  }
+}
+// orders this thread's accesses of either proxy (generic, async) before its later ones
+MLA_DEVI void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
+MLA_DEVI void mbar_inval(uint32_t addr) { asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(addr) : "memory"); }
+
 MLA_DEVI void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ---------------------------------------------------------------- descriptors

@@ -2,18 +2,19 @@
 
 ``DecodeStep``: absorb -> paged decode -> combine -> up-project (the absorbed
 form); it owns the intermediate device buffers (q_lat, o_lat, lse, out and the
-workspace) and replays the four calls on the current stream.  ``PrefillStep``:
-the explicit form for long chunks of new tokens (one call, two kernels).
-Neither does arithmetic of its own.
+workspace) and replays the four calls on the current stream.  ``FusedStep``: the
+same step through ``mla_decode_step`` (one call; one launch where the shape
+allows).  ``PrefillStep``: the explicit form for long chunks of new tokens (one
+call, two kernels).  None does arithmetic of its own.
 """
 
 from __future__ import annotations
 
 import torch
 
-from . import (D_C, D_N, D_V, alloc_workspace, make_decode_args, make_prefill_args, mla_absorb_q,
-               mla_combine_splits, mla_decode_num_splits, mla_decode_paged, mla_prefill,
-               mla_up_proj_v)
+from . import (D_C, D_N, D_V, alloc_workspace, make_decode_args, make_prefill_args, make_step_args,
+               mla_absorb_q, mla_combine_splits, mla_decode_num_splits, mla_decode_paged,
+               mla_decode_step, mla_decode_step_launches, mla_prefill, mla_up_proj_v)
 
 
 class DecodeStep:
@@ -79,6 +80,51 @@ def step_from_workload(w, device="cuda", num_splits=0):
                       block_table=d(w.block_table), seq_lens=d(w.seq_lens), causal=w.causal,
                       softmax_scale=w.softmax_scale, num_splits=num_splits,
                       max_seq_len=max(w.lens) if w.lens else 0)
+
+
+class FusedStep:
+    """The decode step through one ``mla_decode_step`` call: owns out, lse and the
+    workspace (which holds q_lat, o_lat and the step's flags)."""
+
+    def __init__(self, *, q_nope, q_pe, w_uk, w_uv, kv_cache, kv_scale, block_table, seq_lens,
+                 causal, softmax_scale, num_splits=0, max_seq_len=0, out=None, fuse=0):
+        B, s_q, H, _ = q_nope.shape
+        dev = q_nope.device
+        self.B, self.s_q, self.H = B, s_q, H
+        self.lse = torch.empty(B, s_q, H, dtype=torch.float32, device=dev)
+        self.out = out if out is not None else torch.empty(B, s_q, H, D_V, dtype=torch.bfloat16,
+                                                           device=dev)
+        self.args = make_step_args(q_nope=q_nope, q_pe=q_pe, w_uk=w_uk, w_uv=w_uv, kv_cache=kv_cache,
+                                   kv_scale=kv_scale, block_table=block_table, seq_lens=seq_lens,
+                                   out=self.out, lse=self.lse, causal=causal,
+                                   softmax_scale=softmax_scale, num_splits=num_splits,
+                                   max_seq_len=max_seq_len, fuse=fuse)
+        self.workspace = alloc_workspace(self.args, device=dev)
+        self.launches = mla_decode_step_launches(self.args)
+        self._keep = (q_nope, q_pe, w_uk, w_uv, kv_cache, kv_scale, block_table, seq_lens)
+
+    def run(self, stream=None):
+        mla_decode_step(self.args, stream)
+        return self.out
+
+    def capture(self):
+        """One CUDA graph of the step (see ``DecodeStep.capture``)."""
+        self.run()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.run()
+        return g
+
+
+def fused_from_workload(w, device="cuda", num_splits=0, fuse=0):
+    """Copy a ``mla_inputs.Workload`` to the device and build its ``FusedStep``."""
+    d = lambda t: None if t is None else t.to(device, non_blocking=False).contiguous()
+    return FusedStep(q_nope=d(w.q_nope), q_pe=d(w.q_pe), w_uk=d(w.w_uk), w_uv=d(w.w_uv),
+                     kv_cache=d(w.kv_cache), kv_scale=d(w.kv_scale),
+                     block_table=d(w.block_table), seq_lens=d(w.seq_lens), causal=w.causal,
+                     softmax_scale=w.softmax_scale, num_splits=num_splits,
+                     max_seq_len=max(w.lens) if w.lens else 0, fuse=fuse)
 
 
 class PrefillStep:

@@ -327,6 +327,66 @@ mla_status_t mla_prefill_workspace_size(const mla_prefill_args_t* args, size_t* 
 mla_status_t mla_prefill(const mla_prefill_args_t* args, void* stream);
 
 /*
+ * Arguments of mla_decode_step / mla_decode_step_workspace_size /
+ * mla_decode_step_launches: the whole decode step from the query's two parts to
+ * the output.  Zero-initialise the struct, then fill every field.
+ */
+typedef struct {
+  const void* q_nope;             /* bf16 [B][s_q][H][d_n] */
+  const void* q_pe;               /* bf16 [B][s_q][H][d_r], RoPE already applied */
+  const void* w_uk;               /* bf16 [H][d_n][d_c] */
+  const void* w_uv;               /* bf16 [H][d_v][d_c] */
+  const void* kv_cache;           /* as in mla_decode_args_t */
+  const void* kv_scale;           /* as in mla_decode_args_t */
+  const int32_t* block_table;     /* int32 [B][max_pages_per_seq] */
+  const int32_t* seq_lens;        /* int32 [B], device, including the s_q new tokens */
+  void* out;                      /* bf16 [B][s_q][H][d_v], written */
+  float* lse;                     /* fp32 [B][s_q][H], natural log, written; may be NULL */
+  void* workspace;                /* device scratch, >= mla_decode_step_workspace_size() bytes,
+                                     16-byte aligned, zero before the first use (its first 16
+                                     bytes hold the sticky status word; it also holds q_lat,
+                                     o_lat and the step's flags) */
+  size_t workspace_bytes;
+  int32_t B, s_q, H;
+  int32_t d_c, d_r, page_size;
+  int32_t num_pages;
+  int32_t max_pages_per_seq;
+  int32_t kv_dtype;               /* mla_kv_dtype_t */
+  int32_t causal;
+  int32_t num_splits;             /* 0 = automatic, as for mla_decode_paged */
+  int32_t max_seq_len;
+  float softmax_scale;
+  int32_t fuse;                   /* 0: one launch where it measured faster (a q8_0 or q4_0
+                                     cache whose grid covers at least half the SMs); 1: one
+                                     launch wherever the shape allows it; -1: never */
+} mla_step_args_t;
+
+/* Bytes of workspace mla_decode_step needs (host only). */
+mla_status_t mla_decode_step_workspace_size(const mla_step_args_t* args, size_t* bytes);
+
+/* Kernel launches mla_decode_step makes for these arguments (host only): 1 when
+ * the step runs fused, else 3 (one split) or 4. */
+mla_status_t mla_decode_step_launches(const mla_step_args_t* args, int32_t* launches);
+
+/*
+ * mla_decode_step — the decode step in one call: o = W_UV attention(W_UK^T
+ * q_nope, q_pe; cache), the same function as mla_absorb_q, mla_decode_paged,
+ * mla_combine_splits and mla_up_proj_v in sequence (snowgate thread 35: a
+ * fused dequantise-and-multiply decode; nnets.ru article, section "Суть MLA",
+ * for the absorbed form).  With a bf16, q8_0 or q4_0 cache, one split and at
+ * most one query token per CTA pair the device holds at once, it can be one
+ * launch (see `fuse`): every CTA first takes a
+ * share of the query absorption (so W_UK is read once per 64 query tokens,
+ * not once per token), decodes its unit once the absorption tiles of its
+ * tokens are written, then takes a share of the up-projection once the decode
+ * rows it needs are written (flags in the workspace; every wait bounded, a
+ * wait that runs out records MLA_ERR_DEVICE_TIMEOUT).  Otherwise it enqueues
+ * the four kernels above on `stream`.  Results are identical either way.  After
+ * a recorded device timeout, zero the workspace before the next call.
+ */
+mla_status_t mla_decode_step(const mla_step_args_t* args, void* stream);
+
+/*
  * mla_fold_hadamard — folds the Hadamard rotation of the latent space into the
  * weights, in place (ik_llama.cpp docs "FlashMLA", section "KV cache with MLA":
  * below 6 bits a Hadamard transform of the cache before quantisation recovers

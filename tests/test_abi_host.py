@@ -294,3 +294,71 @@ def test_fold_hadamard_argument_checks(lib):
     assert f(None, 0, p, p, 129, None) == UNSUPPORTED
     assert f(p + 8, 7168, None, None, 0, None) == MISALIGNED
     assert f(None, 0, p, p + 4, 16, None) == MISALIGNED
+
+
+def _sargs(B=2, s_q=1, H=128, splits=0, max_len=4096, **kw):
+    a = mla.StepArgs()
+    fake = 0x10000
+    for f in ("q_nope", "q_pe", "w_uk", "w_uv", "kv_cache", "block_table", "seq_lens", "out", "lse"):
+        setattr(a, f, fake)
+    a.B, a.s_q, a.H = B, s_q, H
+    a.d_c, a.d_r, a.page_size = 512, 64, 64
+    a.num_pages, a.max_pages_per_seq = 128, 64
+    a.kv_dtype, a.causal, a.num_splits, a.max_seq_len = 0, 0, splits, max_len
+    a.softmax_scale = 0.0722
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_step_workspace_holds_the_decode_flags_and_both_latents(lib):
+    # the decode's part (256 bytes at one split), 256 bytes of flags, then q_lat and
+    # o_lat (B * s_q * H * 512 bf16 each, 256-byte aligned)
+    lat = 2 * 1 * 128 * 512 * 2
+    assert mla.mla_decode_step_workspace_size(_sargs(splits=1)) == 256 + 256 + 2 * lat
+    four = mla.mla_decode_step_workspace_size(_sargs(splits=4))
+    assert four == mla.mla_decode_workspace_size(_args(splits=4)) + 256 + 2 * lat
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("d_c", 256, UNSUPPORTED), ("H", 24, UNSUPPORTED), ("s_q", 1025, UNSUPPORTED), ("kv_dtype", 4, UNSUPPORTED),
+    ("H", 0, INVALID), ("B", -1, INVALID), ("num_splits", 129, INVALID),
+])
+def test_step_rejects_bad_shapes(lib, field, value, code):
+    a = _sargs(**{field: value})
+    a.workspace, a.workspace_bytes = 0x20000, 1 << 40
+    assert lib.mla_decode_step(ctypes.byref(a), None) == code
+    n = ctypes.c_size_t(0)
+    assert lib.mla_decode_step_workspace_size(ctypes.byref(a), ctypes.byref(n)) == code
+    k = ctypes.c_int32(0)
+    assert lib.mla_decode_step_launches(ctypes.byref(a), ctypes.byref(k)) == code
+
+
+def test_step_rejects_bad_pointers_and_workspace(lib):
+    a = _sargs()
+    assert lib.mla_decode_step(ctypes.byref(a), None) == INVALID              # no workspace
+    a.workspace, a.workspace_bytes = 0x20008, 1 << 40
+    assert lib.mla_decode_step(ctypes.byref(a), None) == MISALIGNED
+    a.workspace, a.workspace_bytes = 0x20000, 1024
+    assert lib.mla_decode_step(ctypes.byref(a), None) == WS_SMALL
+    a.workspace_bytes = 1 << 40
+    for f in ("q_nope", "w_uk", "w_uv", "out", "q_pe", "kv_cache"):
+        setattr(a, f, None)
+        assert lib.mla_decode_step(ctypes.byref(a), None) == INVALID, f
+        setattr(a, f, 0x10008)
+        assert lib.mla_decode_step(ctypes.byref(a), None) == MISALIGNED, f
+        setattr(a, f, 0x10000)
+    a.kv_dtype, a.kv_scale = 3, None                                         # q4_0 needs scales
+    assert lib.mla_decode_step(ctypes.byref(a), None) == INVALID
+
+
+def test_step_with_empty_batch_enqueues_nothing(lib):
+    a = _sargs(B=0)
+    a.workspace, a.workspace_bytes = 0x20000, 1024
+    assert lib.mla_decode_step(ctypes.byref(a), None) == OK
+    assert mla.mla_decode_step_launches(a) == 0
+    # without a device the step is never fused: the four-kernel sequence (three at one split)
+    assert mla.mla_decode_step_launches(_sargs(splits=1)) in (1, 3)
+    assert mla.mla_decode_step_launches(_sargs(splits=4)) == 4
+    assert mla.mla_decode_step_launches(_sargs(splits=1, kv_dtype=1)) == 3   # e4m3: never fused
+    assert mla.mla_decode_step_launches(_sargs(splits=1, fuse=-1)) == 3
