@@ -42,21 +42,21 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # file and the device headers it includes, as they were when the capture was
 # taken: reported as the roofline's ``traffic`` only while they are unchanged.
 MEASURED_TRAFFIC = {
-    # ncu --set full, one launch of the V3 workload
-    "v3": (315_394_304, "decode_tc.cu", "7bb76fcc659538c8"),
+    # ncu (dram__bytes_read.sum + dram__bytes_write.sum), one launch of the V3 workload
+    "v3": (314_853_888, "decode_tc.cu", "37924f04a4a9e143"),
     # one launch of the fp8 workload
-    "fp8": (773_442_560, "decode_f8.cu", "39cb32945b83f43e"),
+    "fp8": (774_229_504, "decode_f8.cu", "39ec40f7a33f3d1f"),
     # one launch of each long-context workload
-    "long16": (607_938_304, "decode_tc.cu", "7bb76fcc659538c8"),
-    "long128": (608_454_912, "decode_tc.cu", "7bb76fcc659538c8"),
-    # one launch of the q8_0 workload (the same kernel file, its q8_0 variant)
-    "q8": (175_534_592, "decode_tc.cu", "7bb76fcc659538c8"),
-    # one launch of the q4_0 workload (the q4_0 variant)
-    "q4": (98_002_688, "decode_tc.cu", "30109a2e70d165f7"),
+    "long16": (607_507_200, "decode_tc.cu", "37924f04a4a9e143"),
+    "long128": (608_263_168, "decode_tc.cu", "37924f04a4a9e143"),
+    # one launch of the q8_0 and the q4_0 workloads (the same kernel file, its
+    # blockwise instances)
+    "q8": (173_468_672, "decode_tc.cu", "37924f04a4a9e143"),
+    "q4": (97_926_656, "decode_tc.cu", "37924f04a4a9e143"),
     # both prefill kernels on one sequence of the chunked-prefill workload:
-    # 1,153,470,976 bytes, times the 4 sequences of the full workload (traffic
+    # 1,148,841,984 bytes, times the 4 sequences of the full workload (traffic
     # grows with the sequences processed)
-    "prefill": (4 * 1_153_470_976, "prefill.cu", "5faab4bd87ffdac2"),
+    "prefill": (4 * 1_148_841_984, "prefill.cu", "740bfda2cf634d5e"),
 }
 KERNEL_HEADERS = ("sm100.cuh", "common.cuh", "tma_host.cuh")
 
