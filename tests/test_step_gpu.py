@@ -140,3 +140,21 @@ def test_automatic_choice_of_one_launch(cuda_lib):
         w = make_workload(WorkloadSpec("fa", B=B, H=128, s_q=1, lens=[64] * B, kv_dtype=kv, seed=57))
         st = fused_from_workload(w, num_splits=1, fuse=fuse)
         assert st.launches == want, (kv, B, fuse, st.launches)
+
+
+def test_fused_step_two_token_blocks_and_empty_sequences(cuda_lib):
+    """More than 64 query tokens: the projection tiles and flags of a second token
+    block (two of its 64 rows real, the rest past the end), and sequences with no
+    cached token (o = 0, lse = -inf) inside the one launch."""
+    B = 66
+    lens = [0 if b % 17 == 5 else 64 + 37 * b for b in range(B)]
+    w = make_workload(WorkloadSpec("f2b", B=B, H=32, s_q=1, lens=lens, seed=58))
+    st = _fused(cuda_lib, w, splits=1)
+    if st.launches != 1:
+        pytest.skip(f"the device holds fewer than {B} CTA pairs of the fused kernel at once")
+    rows = [(b, 0) for b in (0, 5, 22, 63, 64, 65)]
+    ref = oracle_of(w, rows=rows, absorbed=True)
+    bi = tuple(np.array(x) for x in zip(*rows))
+    check_close("o", to_np(st.out)[bi], ref["o"][bi], "bf16")
+    check_lse(to_np(st.lse)[bi], ref["lse"][bi], TOL["bf16"][0])
+    assert torch.equal(st.out, _four(cuda_lib, w, splits=1).out)
