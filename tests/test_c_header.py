@@ -38,6 +38,17 @@ int main(void) {
   w.num_pages = 4096; w.max_pages_per_seq = 64; w.kv_dtype = MLA_KV_BF16; w.rope_base = 10000.f;
   if (mla_write_kv_workspace_size(&w, &bytes) != MLA_OK || bytes < 256) return 6;
   if (strcmp(mla_status_string(MLA_ERR_MISALIGNED), "MLA_ERR_MISALIGNED") != 0) return 7;
+  mla_step_args_t s;
+  memset(&s, 0, sizeof s);
+  s.B = 64; s.s_q = 1; s.H = 128; s.d_c = MLA_D_C; s.d_r = MLA_D_R; s.page_size = MLA_PAGE_SIZE;
+  s.num_pages = 4096; s.max_pages_per_seq = 64; s.kv_dtype = MLA_KV_Q4_0; s.max_seq_len = 4096;
+  s.softmax_scale = 0.0722f; s.fuse = -1;
+  /* one split: the decode's 256 bytes, the step's flags, q_lat and o_lat */
+  if (mla_decode_step_workspace_size(&s, &bytes) != MLA_OK || bytes != 512 + 2 * 64 * 128 * 512 * 2) return 8;
+  int32_t launches = 0;
+  if (mla_decode_step_launches(&s, &launches) != MLA_OK || launches != 3) return 9;
+  if (mla_decode_step(&s, 0) != MLA_ERR_INVALID_VALUE) return 10;     /* no workspace */
+  if (mla_fold_hadamard(0, 0, 0, 0, 0, 0) != MLA_OK) return 11;       /* nothing to fold */
   printf("ok\n");
   return 0;
 }
