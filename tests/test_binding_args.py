@@ -101,3 +101,51 @@ def test_projection_calls_check_shapes_before_the_device():
         mla.mla_up_proj_v(x, w, torch.zeros(4, H, 128, dtype=bf16))
     with pytest.raises(ValueError, match="out: dtype"):
         mla.mla_up_proj_v(x, w, torch.zeros(3, H, 128, dtype=f32))
+
+
+def _step_tensors(B=2, s_q=1, H=16, P=8, kind="bf16"):
+    cache = {"bf16": torch.zeros(P, 64, 576, dtype=bf16), "q8_0": torch.zeros(P, 64, 576, dtype=torch.int8),
+             "q4_0": torch.zeros(P, 64, 288, dtype=torch.uint8)}[kind]
+    scale = None if kind == "bf16" else torch.ones(P, 64, 18, dtype=torch.float16)
+    return dict(
+        q_nope=torch.zeros(B, s_q, H, 128, dtype=bf16), q_pe=torch.zeros(B, s_q, H, 64, dtype=bf16),
+        w_uk=torch.zeros(H, 128, 512, dtype=bf16), w_uv=torch.zeros(H, 128, 512, dtype=bf16),
+        kv_cache=cache, kv_scale=scale, block_table=torch.zeros(B, 4, dtype=i32), seq_lens=torch.ones(B, dtype=i32),
+        out=torch.zeros(B, s_q, H, 128, dtype=bf16), lse=torch.zeros(B, s_q, H, dtype=f32))
+
+
+def test_step_args_need_device_tensors():
+    with pytest.raises(ValueError, match="q_nope must be a CUDA tensor"):
+        mla.make_step_args(**_step_tensors(), softmax_scale=0.07)
+
+
+@pytest.mark.parametrize("field,bad,msg", [
+    ("q_nope", torch.zeros(2, 1, 16, 128, dtype=f32), "q_nope: dtype"),
+    ("w_uk", torch.zeros(16, 128, 256, dtype=bf16), "w_uk: shape"),
+    ("w_uv", torch.zeros(8, 128, 512, dtype=bf16), "w_uv: shape"),
+    ("out", torch.zeros(2, 1, 16, 512, dtype=bf16), "out: shape"),
+    ("kv_cache", torch.zeros(8, 64, 576, dtype=torch.uint8), "kv_cache: shape"),   # uint8 is q4_0: 288 a row
+])
+def test_step_args_reject_bad_tensors(field, bad, msg):
+    t = _step_tensors()
+    t[field] = bad
+    with pytest.raises(ValueError, match=msg):
+        mla.make_step_args(**t, softmax_scale=0.07)
+
+
+@pytest.mark.parametrize("kind", ["q8_0", "q4_0"])
+def test_step_args_blockwise_cache_needs_fp16_block_scales(kind):
+    t = _step_tensors(kind=kind)
+    t["kv_scale"] = None
+    with pytest.raises(ValueError, match="kv_scale is required"):
+        mla.make_step_args(**t, softmax_scale=0.07)
+    t["kv_scale"] = torch.ones(8, 64, dtype=torch.float16)
+    with pytest.raises(ValueError, match="kv_scale: shape"):
+        mla.make_step_args(**t, softmax_scale=0.07)
+
+
+def test_fold_hadamard_checks_its_weights():
+    with pytest.raises(ValueError, match="w_uk: shape"):
+        mla.mla_fold_hadamard(w_uk=torch.zeros(4, 128, 256, dtype=bf16))
+    with pytest.raises(ValueError, match="w_dkv must be a CUDA tensor"):
+        mla.mla_fold_hadamard(w_dkv=torch.zeros(576, 128, dtype=bf16))
